@@ -1,0 +1,355 @@
+/*
+ * moe_oracle.c -- plain, slow CPU oracle of the MoE expert-FFN layer.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path links, loads or calls
+ * this file; only the test suite, the smoke check and the benchmark's CPU
+ * baseline do. It shares no code with the CUDA library.
+ *
+ * What the layer computes (its plain definition):
+ *
+ *   out[t] = sum_{j<k} w[t,j] * FFN_{e[t,j]}(x[t])
+ *   FFN_e(x) = W_d[e] * (silu(W_g[e] x) (.) (W_u[e] x)),  silu(g) = g / (1 + exp(-g))
+ *
+ * Sources:
+ *  - InfiniLM PR #500, "T2-1-3 Qwen3-MoE inference optimisation" report,
+ *    §2.1 (Qwen3-MoE routing: top-k softmax, no shared expert, no bias) and
+ *    §2.2 (bucket the routing indices into per-expert counts and a
+ *    permutation; gather the activations by that permutation; three grouped
+ *    GEMMs gate/up/down with SwiGLU between them; scale by the routing
+ *    weights and scatter back to the tokens).
+ *  - FlashInfer PR #7196 analysis ("CuTe DSL W4A16 MoE optimisation and
+ *    bit-exact tests"), §1 (moe_finalize: slot 0 is a round-to-nearest fp32
+ *    multiply, later slots are round-to-nearest fp32 FMAs in slot order, no
+ *    flush-to-zero, signed zero kept) and §2-§3 (W4A16: int4 weights decoded
+ *    to bf16 with a per-group scale before the MMA).
+ *
+ * Precision: dot products accumulate in double, are rounded once to fp32 (the
+ * "fp32-accumulated" value), and the layer's bf16 rounding points are kept
+ * where the layer has them: act = bf16(silu(g) * u), y = bf16(down output),
+ * out = bf16(finalize accumulator). Finalize is emulated exactly in fp32.
+ * Build flags: -O2 -ffp-contract=off, no fast-math; FTZ/DAZ are cleared at
+ * each entry point that does fp32 arithmetic.
+ *
+ * Readings of points the sources leave open (each also stated where used):
+ *  R1 top-k selects on the softmax probabilities (monotone in the logits);
+ *     equal probabilities go to the lower expert id; slot order is
+ *     descending probability.
+ *  R2 weights are renormalised over the k selected experts.
+ *  R3 rows [0,I) of W_gu[e] are the gate projection and rows [I,2I) the up
+ *     projection.
+ *  R4 the permutation is stable: within one expert, pairs p = t*k + j keep
+ *     ascending p (ascending token).
+ *  R5 perm[r] = pair id p; inv_perm[p] = r.
+ *  R6 the routing weight is applied in finalize only; y is the unscaled
+ *     bf16 down-projection output.
+ *  R7 int4: the low nibble of byte b is K index 2b, the high nibble 2b+1,
+ *     two's complement in [-8,7]; one bf16 scale per 128 consecutive K
+ *     elements of a row; w = bf16(q * scale).
+ *  R8 bf16 rounding is round-to-nearest-even; NaN stays NaN.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+#if defined(__x86_64__) || defined(__i386__)
+#include <xmmintrin.h>
+#endif
+
+/* ---- scalar helpers ----------------------------------------------------- */
+
+static void no_ftz_daz(void) {
+#if defined(__x86_64__) || defined(__i386__)
+    /* MXCSR bit 15 = FTZ, bit 6 = DAZ. */
+    _mm_setcsr(_mm_getcsr() & ~(0x8000u | 0x0040u));
+#endif
+}
+
+static float bf16_to_f32(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* Round-to-nearest-even fp32 -> bf16 (R8). */
+static uint16_t f32_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7fffffffu) > 0x7f800000u) return (uint16_t)((u >> 16) | 0x0040u);
+    u += 0x7fffu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+/* Sign-extended nibble n (0..15) as the int4 value (R7). */
+static int int4_value(unsigned n) { return (n & 8u) ? (int)n - 16 : (int)n; }
+
+/* w = bf16(q * scale); the fp32 product is exact (<= 12 significant bits). */
+static uint16_t dequant_one(const uint8_t *row_q, const uint16_t *row_s, int kidx) {
+    unsigned byte = row_q[kidx >> 1];
+    unsigned nib = (kidx & 1) ? (byte >> 4) : (byte & 15u);
+    float q = (float)int4_value(nib);
+    float s = bf16_to_f32(row_s[kidx / 128]);
+    return f32_to_bf16(q * s);
+}
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}
+
+/* ---- step 1: routing ------------------------------------------------------
+ * Softmax over all E logits, keep the k most probable experts (R1), then
+ * renormalise their probabilities to sum to one (R2). InfiniLM PR #500 §2.1,
+ * §2.4 (op::topksoftmax); the renormalisation is Qwen3's norm_topk_prob.
+ * Returns 0, or -1 on bad sizes.
+ */
+int oracle_route(const float *logits, int T, int E, int k, int32_t *ids, float *w) {
+    if (T < 0 || E < 1 || k < 1 || k > E) return -1;
+    int bad = 0;
+#pragma omp parallel for schedule(static)
+    for (int t = 0; t < T; ++t) {
+        const float *l = logits + (size_t)t * E;
+        double *p = (double *)malloc(sizeof(double) * (size_t)E);
+        char *taken = (char *)calloc((size_t)E, 1);
+        if (!p || !taken) { bad = 1; free(p); free(taken); continue; }
+        double m = -INFINITY;
+        for (int e = 0; e < E; ++e) if ((double)l[e] > m) m = (double)l[e];
+        double z = 0.0;
+        for (int e = 0; e < E; ++e) { p[e] = exp((double)l[e] - m); z += p[e]; }
+        for (int e = 0; e < E; ++e) p[e] /= z;
+        double s = 0.0;
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                if (taken[e]) continue;
+                if (best < 0 || p[e] > p[best]) best = e;   /* strict: ties keep the lower id */
+            }
+            taken[best] = 1;
+            ids[(size_t)t * k + j] = best;
+            s += p[best];
+        }
+        for (int j = 0; j < k; ++j)
+            w[(size_t)t * k + j] = (float)(p[ids[(size_t)t * k + j]] / s);
+        free(p);
+        free(taken);
+    }
+    return bad ? -1 : 0;
+}
+
+/* ---- step 2: bucketing ----------------------------------------------------
+ * Counting sort of the flat pair list p = t*k + j by expert id, stable in p
+ * (R4, R5). InfiniLM PR #500 §2.2 step 1. Returns 0, or -1 if an id is out of
+ * range (outputs are then undefined).
+ */
+int oracle_permute(const int32_t *ids, int P, int E, int32_t *counts, int32_t *offsets,
+                   int32_t *perm, int32_t *inv_perm) {
+    if (P < 0 || E < 1) return -1;
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int p = 0; p < P; ++p) {
+        if (ids[p] < 0 || ids[p] >= E) return -1;
+        counts[ids[p]]++;
+    }
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int32_t *fill = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    if (!fill) return -1;
+    for (int e = 0; e < E; ++e) fill[e] = offsets[e];
+    for (int p = 0; p < P; ++p) {
+        int r = fill[ids[p]]++;
+        perm[r] = p;
+        inv_perm[p] = r;
+    }
+    free(fill);
+    return 0;
+}
+
+/* ---- step 3: gather -------------------------------------------------------
+ * hidden_perm[r] = hidden[perm[r] / k]. InfiniLM PR #500 §2.2 step 2.
+ */
+void oracle_gather(const uint16_t *hidden, const int32_t *perm, int P, int H, int k,
+                   uint16_t *hidden_perm) {
+    for (int r = 0; r < P; ++r)
+        memcpy(hidden_perm + (size_t)r * H, hidden + (size_t)(perm[r] / k) * H, sizeof(uint16_t) * (size_t)H);
+}
+
+/* ---- step 7: W4A16 weight decoding -----------------------------------------
+ * out[r][c] = bf16(q[r][c] * scale[r][c/128]) (R7). FlashInfer PR #7196
+ * analysis §2 (W4A16: 4-bit weights, 16-bit activations) and §3 (exact
+ * reference covering bf16 weight decoding).
+ */
+void oracle_dequant_int4(const uint8_t *q, const uint16_t *scales, int rows, int K, uint16_t *out) {
+    no_ftz_daz();
+    for (int r = 0; r < rows; ++r)
+        for (int c = 0; c < K; ++c)
+            out[(size_t)r * K + c] = dequant_one(q + (size_t)r * (K / 2), scales + (size_t)r * (K / 128), c);
+}
+
+/* ---- steps 4-5: one expert's FFN on one activation row ---------------------
+ * act[i] = bf16(silu(g_i) * u_i),  g = W_g x, u = W_u x  (R3), InfiniLM PR
+ * #500 §2.2 (gate/up grouped GEMM, then SwiGLU);
+ * y[h] = bf16(sum_i act[i] * W_d[h][i]) (R6), the down grouped GEMM.
+ * Weights are bf16 (fmt 0) or int4 + scales (fmt 1, decoded per element).
+ */
+static float weight_at(int fmt, const void *w, const uint16_t *s, int K, int row, int col) {
+    if (fmt == 0) return bf16_to_f32(((const uint16_t *)w)[(size_t)row * K + col]);
+    return bf16_to_f32(dequant_one((const uint8_t *)w + (size_t)row * (K / 2), s + (size_t)row * (K / 128), col));
+}
+
+void oracle_expert_ffn(int fmt, const uint16_t *x, const void *w_gu, const uint16_t *w_gu_s,
+                       const void *w_d, const uint16_t *w_d_s, int H, int I,
+                       uint16_t *act, uint16_t *y) {
+    no_ftz_daz();
+    for (int i = 0; i < I; ++i) {
+        double g = 0.0, u = 0.0;
+        for (int h = 0; h < H; ++h) {
+            double xv = (double)bf16_to_f32(x[h]);
+            g += xv * (double)weight_at(fmt, w_gu, w_gu_s, H, i, h);
+            u += xv * (double)weight_at(fmt, w_gu, w_gu_s, H, I + i, h);
+        }
+        float gf = (float)g, uf = (float)u;
+        double silu = (double)gf / (1.0 + exp(-(double)gf));
+        act[i] = f32_to_bf16((float)(silu * (double)uf));
+    }
+    for (int h = 0; h < H; ++h) {
+        double acc = 0.0;
+        for (int i = 0; i < I; ++i)
+            acc += (double)bf16_to_f32(act[i]) * (double)weight_at(fmt, w_d, w_d_s, I, h, i);
+        y[h] = f32_to_bf16((float)acc);
+    }
+}
+
+/* ---- step 6: finalize / unpermute ------------------------------------------
+ * out[t][h] = bf16(acc), acc = v_0 * w_0 (fp32 multiply), then
+ * acc = fma(v_j, w_j, acc) for j = 1..k-1 in slot order, round to nearest,
+ * no FTZ, v_j = y[inv_perm[t*k+j]][h]. FlashInfer PR #7196 analysis §1
+ * (moe_finalize.py: _mul_rn for slot 0, _fma_rn without .ftz afterwards).
+ */
+static float combine_slots(const float *v, const float *w, int k) {
+    float acc = v[0] * w[0];  /* one fp32 multiply; -ffp-contract=off keeps it unfused */
+    for (int j = 1; j < k; ++j) acc = fmaf(v[j], w[j], acc);
+    return acc;
+}
+
+void oracle_finalize(const uint16_t *y, const float *w, const int32_t *inv_perm, int T, int H, int k,
+                     uint16_t *out) {
+    no_ftz_daz();
+#pragma omp parallel
+    {
+        no_ftz_daz();
+        float *v = (float *)malloc(sizeof(float) * (size_t)(k > 0 ? k : 1));
+#pragma omp for schedule(static)
+        for (int t = 0; t < T; ++t) {
+            for (int h = 0; h < H; ++h) {
+                for (int j = 0; j < k; ++j)
+                    v[j] = bf16_to_f32(y[(size_t)inv_perm[(size_t)t * k + j] * H + h]);
+                out[(size_t)t * H + h] = f32_to_bf16(combine_slots(v, w + (size_t)t * k, k));
+            }
+        }
+        free(v);
+    }
+}
+
+/* ---- the whole layer --------------------------------------------------------
+ * route -> permute -> gather -> per-expert FFN over its rows -> finalize,
+ * the order of InfiniLM PR #500 §2.2. Intermediates are returned so that each
+ * step of the GPU path can be compared with its own stage. fmt 0: bf16
+ * weights [E,2I,H] and [E,H,I]; fmt 1: int4 [E,2I,H/2], [E,H,I/2] with bf16
+ * scales [E,2I,H/128], [E,H,I/128].
+ */
+int oracle_forward(int fmt, const uint16_t *hidden, const float *logits,
+                   const void *w_gu, const uint16_t *w_gu_s, const void *w_d, const uint16_t *w_d_s,
+                   int T, int H, int I, int E, int k,
+                   int32_t *ids, float *w, int32_t *counts, int32_t *offsets,
+                   int32_t *perm, int32_t *inv_perm, uint16_t *act, uint16_t *y, uint16_t *out) {
+    if (T < 0 || H < 1 || I < 1 || k < 1 || k > E) return -1;
+    if (fmt == 1 && (H % 128 || I % 128)) return -1;
+    int P = T * k;
+    if (oracle_route(logits, T, E, k, ids, w)) return -1;
+    if (oracle_permute(ids, P, E, counts, offsets, perm, inv_perm)) return -1;
+    size_t gu_elems = fmt == 0 ? (size_t)2 * I * H : (size_t)2 * I * (H / 2);
+    size_t d_elems = fmt == 0 ? (size_t)H * I : (size_t)H * (I / 2);
+    size_t esz = fmt == 0 ? 2 : 1;
+    for (int e = 0; e < E; ++e) {
+        const char *wgu_e = (const char *)w_gu + (size_t)e * gu_elems * esz;
+        const char *wd_e = (const char *)w_d + (size_t)e * d_elems * esz;
+        const uint16_t *sgu_e = fmt == 1 ? w_gu_s + (size_t)e * 2 * I * (H / 128) : NULL;
+        const uint16_t *sd_e = fmt == 1 ? w_d_s + (size_t)e * H * (I / 128) : NULL;
+#pragma omp parallel for schedule(dynamic, 1)
+        for (int r = offsets[e]; r < offsets[e + 1]; ++r) {
+            int t = perm[r] / k;
+            oracle_expert_ffn(fmt, hidden + (size_t)t * H, wgu_e, sgu_e, wd_e, sd_e, H, I,
+                              act + (size_t)r * I, y + (size_t)r * H);
+        }
+    }
+    oracle_finalize(y, w, inv_perm, T, H, k, out);
+    return 0;
+}
+
+/* The same layer for a subset of tokens only (used where the full layer is
+ * too slow for the oracle): routes the listed tokens, evaluates the FFN of
+ * each of their k pairs in slot order, and combines in slot order exactly as
+ * finalize does. out_rows[n] receives token tokens[n]; ids_out/w_out are
+ * [n_tokens, k].
+ */
+int oracle_forward_tokens(int fmt, const uint16_t *hidden, const float *logits,
+                          const void *w_gu, const uint16_t *w_gu_s, const void *w_d, const uint16_t *w_d_s,
+                          int T, int H, int I, int E, int k, const int32_t *tokens, int n_tokens,
+                          int32_t *ids_out, float *w_out, uint16_t *out_rows) {
+    if (T < 0 || H < 1 || I < 1 || k < 1 || k > E || n_tokens < 0) return -1;
+    if (fmt == 1 && (H % 128 || I % 128)) return -1;
+    for (int n = 0; n < n_tokens; ++n) {
+        if (tokens[n] < 0 || tokens[n] >= T) return -1;
+        if (oracle_route(logits + (size_t)tokens[n] * E, 1, E, k, ids_out + (size_t)n * k, w_out + (size_t)n * k))
+            return -1;
+    }
+    size_t gu_elems = fmt == 0 ? (size_t)2 * I * H : (size_t)2 * I * (H / 2);
+    size_t d_elems = fmt == 0 ? (size_t)H * I : (size_t)H * (I / 2);
+    size_t esz = fmt == 0 ? 2 : 1;
+    int npairs = n_tokens * k;
+    uint16_t *ybuf = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(npairs > 0 ? npairs : 1) * H);
+    if (!ybuf) return -1;
+    int bad = 0;
+#pragma omp parallel
+    {
+        uint16_t *abuf = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)I);
+        if (!abuf) bad = 1;
+#pragma omp for schedule(dynamic, 1)
+        for (int q = 0; q < npairs; ++q) {
+            if (!abuf) continue;
+            int n = q / k;
+            int e = ids_out[q];
+            const char *wgu_e = (const char *)w_gu + (size_t)e * gu_elems * esz;
+            const char *wd_e = (const char *)w_d + (size_t)e * d_elems * esz;
+            const uint16_t *sgu_e = fmt == 1 ? w_gu_s + (size_t)e * 2 * I * (H / 128) : NULL;
+            const uint16_t *sd_e = fmt == 1 ? w_d_s + (size_t)e * H * (I / 128) : NULL;
+            oracle_expert_ffn(fmt, hidden + (size_t)tokens[n] * H, wgu_e, sgu_e, wd_e, sd_e, H, I,
+                              abuf, ybuf + (size_t)q * H);
+        }
+        free(abuf);
+    }
+    if (!bad) {
+        /* the pairs of token n sit at rows n*k + j, so an identity inverse
+           permutation over ybuf gives the slot-ordered combine */
+        int32_t *ident = (int32_t *)malloc(sizeof(int32_t) * (size_t)(npairs > 0 ? npairs : 1));
+        if (!ident) { free(ybuf); return -1; }
+        for (int q = 0; q < npairs; ++q) ident[q] = q;
+        oracle_finalize(ybuf, w_out, ident, n_tokens, H, k, out_rows);
+        free(ident);
+    }
+    free(ybuf);
+    return bad ? -1 : 0;
+}

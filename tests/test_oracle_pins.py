@@ -1,0 +1,387 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test checks the oracle against a library routine, a closed form, an
+invariant, an exactly computed value or a dense brute-force evaluation,
+chosen so that a plausible slip in the oracle (a dropped term, a swapped
+gate/up, a wrong index or sign, an unstable sort, an FTZ, a fused slot-0
+multiply) fails at least one of them.
+
+Sources of what is pinned: InfiniLM PR #500 Qwen3-MoE report §2.1-§2.2
+(routing, bucketing, gather, grouped GEMMs with SwiGLU, weighted scatter) and
+the FlashInfer PR #7196 analysis §1 (finalize arithmetic) and §2-§3 (W4A16).
+"""
+
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import moe_synth
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bits_to_bf16(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.uint16).view(np.int16)).view(torch.bfloat16)
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+# ---------------------------------------------------------------- routing --
+
+@pytest.mark.parametrize("T,E,k", [(37, 8, 2), (64, 128, 8), (5, 256, 8), (9, 6, 6), (3, 1, 1)])
+def test_route_ids_are_a_stable_descending_sort(T, E, k):
+    g = torch.Generator().manual_seed(T * 1000 + E)
+    logits = torch.randn(T, E, generator=g)
+    # plant exact ties so that "ties go to the lower expert id" is exercised
+    logits[:, E // 2:] = torch.round(logits[:, E // 2:] * 2) / 2
+    logits[0, :] = 0.25
+    ids, _ = oracle.route(logits, k)
+    ref = torch.sort(logits, dim=1, descending=True, stable=True).indices[:, :k]
+    assert np.array_equal(ids, ref.numpy().astype(np.int32))
+
+
+@pytest.mark.parametrize("T,E,k", [(50, 8, 2), (64, 128, 8), (40, 64, 6), (7, 256, 8)])
+def test_route_weights_match_library_softmax(T, E, k):
+    g = torch.Generator().manual_seed(E + k)
+    logits = torch.randn(T, E, generator=g) * 2
+    ids, w = oracle.route(logits, k)
+    p = torch.softmax(logits.double(), dim=1)
+    sel = torch.gather(p, 1, torch.from_numpy(ids).long())
+    ref = (sel / sel.sum(dim=1, keepdim=True)).numpy()
+    assert np.all(np.abs(w.astype(np.float64) - ref) <= 2.0 ** -24 * ref + 1e-30)
+    # invariants: sum to one, non-increasing in slot order, in (0, 1]
+    assert np.all(np.abs(w.astype(np.float64).sum(1) - 1.0) <= 1e-6)
+    assert np.all(np.diff(w, axis=1) <= 0)
+    assert np.all((w > 0) & (w <= 1))
+
+
+def test_route_closed_forms():
+    g = torch.Generator().manual_seed(3)
+    logits = torch.randn(20, 16, generator=g)
+    # k = 1: the single weight is exactly 1
+    ids, w = oracle.route(logits, 1)
+    assert np.all(w == 1.0)
+    assert np.array_equal(ids[:, 0], logits.argmax(1).numpy())
+    # all-equal logits: experts 0..k-1, weights exactly 1/k (k a power of two)
+    for k in (2, 8):
+        ids, w = oracle.route(torch.full((4, 16), -1.5), k)
+        assert np.array_equal(ids, np.tile(np.arange(k, dtype=np.int32), (4, 1)))
+        assert np.all(w == np.float32(1.0 / k))
+    # k = E: the weights are the full softmax, in descending order
+    ids, w = oracle.route(logits, 16)
+    p = torch.softmax(logits.double(), 1).numpy()
+    ref = np.take_along_axis(p, ids.astype(np.int64), 1)
+    assert np.allclose(w, ref, rtol=2 ** -23, atol=0)
+
+
+def test_route_ignores_a_uniform_shift_of_the_logits():
+    g = torch.Generator().manual_seed(4)
+    logits = torch.randn(30, 64, generator=g)
+    ids0, w0 = oracle.route(logits, 6)
+    ids1, w1 = oracle.route(logits + 8.0, 6)     # exact in fp32 for |x| < 8
+    assert np.array_equal(ids0, ids1)
+    assert np.allclose(w0, w1, rtol=1e-6, atol=0)
+
+
+# ---------------------------------------------------------------- permute --
+
+@pytest.mark.parametrize("T,E,k", [(16, 8, 2), (64, 128, 8), (300, 64, 6), (1, 4, 4), (0, 8, 2)])
+def test_permute_matches_bincount_and_stable_argsort(T, E, k):
+    g = torch.Generator().manual_seed(T + E)
+    logits = torch.randn(T, E, generator=g)
+    ids, _ = oracle.route(logits, k) if T else (np.zeros((0, k), np.int32), None)
+    counts, offsets, perm, inv = oracle.permute(ids, E)
+    flat = torch.from_numpy(ids.reshape(-1).astype(np.int64))
+    assert np.array_equal(counts, torch.bincount(flat, minlength=E).numpy())
+    assert offsets[0] == 0 and offsets[-1] == T * k
+    assert np.array_equal(np.diff(offsets), counts)
+    assert np.array_equal(perm, torch.sort(flat, stable=True).indices.numpy())
+    assert np.array_equal(inv[perm], np.arange(T * k))
+    for e in range(E):
+        seg = perm[offsets[e]:offsets[e + 1]]
+        assert np.all(ids.reshape(-1)[seg] == e)
+        assert np.all(np.diff(seg) > 0)
+
+
+def test_permute_rejects_bad_ids():
+    with pytest.raises(ValueError):
+        oracle.permute(np.array([[0, 9]], np.int32), 8)
+    with pytest.raises(ValueError):
+        oracle.permute(np.array([[-1, 0]], np.int32), 8)
+
+
+def test_gather_rows():
+    h = torch.randn(5, 24).to(torch.bfloat16)
+    perm = np.array([3, 0, 9, 4, 1, 2, 8, 5, 6, 7], np.int32)     # k = 2
+    out = oracle.gather(h, perm, 2)
+    assert np.array_equal(out, bf16_bits(h)[perm // 2])
+
+
+# ---------------------------------------------------------- W4A16 decode --
+
+def test_dequant_int4_matches_torch_rne():
+    g = torch.Generator().manual_seed(5)
+    rows, K = 6, 384
+    q = torch.randint(0, 256, (rows, K // 2), generator=g, dtype=torch.uint8)
+    s = (torch.rand(rows, K // 128, generator=g) * 0.018 + 0.002).to(torch.bfloat16)
+    out = oracle.dequant_int4(q, s)
+    lo = (q & 15).to(torch.int32)
+    hi = (q >> 4).to(torch.int32)
+    nib = torch.stack([lo, hi], dim=2).reshape(rows, K)        # low nibble = even K index
+    val = torch.where(nib >= 8, nib - 16, nib)
+    ref = (val.float() * s.float().repeat_interleave(128, dim=1)).to(torch.bfloat16)
+    assert np.array_equal(out, bf16_bits(ref))
+
+
+def test_dequant_int4_special_values():
+    q = np.zeros((1, 64), np.uint8)
+    q[0, 0] = 0x80          # element 0 -> 0, element 1 -> -8
+    q[0, 1] = 0x7F          # element 2 -> -1, element 3 -> 7
+    s = bf16_bits(torch.tensor([[2.0 ** -7]], dtype=torch.bfloat16))
+    out = bits_to_bf16(oracle.dequant_int4(q, s)).float().numpy()[0]
+    assert out[0] == 0.0 and not np.signbit(out[0])
+    assert out[1] == -8 * 2.0 ** -7 and out[2] == -2.0 ** -7 and out[3] == 7 * 2.0 ** -7
+    assert np.all(out[4:] == 0.0)
+
+
+# ---------------------------------------------------------------- finalize --
+
+def _golden_finalize_cases():
+    cases = []
+    with open(os.path.join(GOLDEN, "finalize_special_cases.txt")) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            k, v, w, exp, why = [c.strip() for c in line.split("|")]
+            cases.append((int(k), [int(x, 16) for x in v.split()],
+                          [int(x, 16) for x in w.split()], int(exp, 16), why))
+    return cases
+
+
+@pytest.mark.parametrize("case", _golden_finalize_cases(), ids=lambda c: c[4])
+def test_finalize_golden_special_cases(case):
+    k, v, w, exp, _ = case
+    y = np.array(v, np.uint16).reshape(k, 1)
+    wf = np.array(w, np.uint32).view(np.float32).reshape(1, k)
+    out = oracle.finalize(y, wf, np.arange(k, dtype=np.int32), 1, 1, k)
+    assert int(out[0, 0]) == exp, f"got {out[0,0]:04x} want {exp:04x}"
+
+
+def _f32_rne(x: Fraction) -> float:
+    """Exact Fraction -> nearest-even fp32 (normal range), by integer arithmetic."""
+    if x == 0:
+        return 0.0
+    sign = -1 if x < 0 else 1
+    x = abs(x)
+    e = math.floor(math.log2(x.numerator) - math.log2(x.denominator))
+    while Fraction(2) ** e > x:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= x:
+        e += 1
+    scaled = x / Fraction(2) ** (e - 23)        # in [2^23, 2^24)
+    n = scaled.numerator // scaled.denominator
+    rem = scaled - n
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and n % 2 == 1):
+        n += 1
+    return sign * float(Fraction(n) * Fraction(2) ** (e - 23))
+
+
+def test_finalize_is_fused_after_slot_zero():
+    """Random slots checked against exact rational arithmetic: slot 0 is one
+    rounded multiply, later slots are single-rounding FMAs."""
+    rng = np.random.default_rng(7)
+    T, H, k = 40, 16, 6
+    y = bf16_bits(torch.from_numpy(rng.standard_normal((T * k, H)).astype(np.float32)).to(torch.bfloat16))
+    w = rng.random((T, k)).astype(np.float32)
+    inv = rng.permutation(T * k).astype(np.int32)
+    out = oracle.finalize(y, w, inv, T, H, k)
+    yf = bits_to_bf16(y).float().numpy()
+    n_unfused_differs = 0
+    for t in range(T):
+        for h in range(H):
+            acc = _f32_rne(Fraction(float(yf[inv[t * k], h])) * Fraction(float(w[t, 0])))
+            unf = acc
+            for j in range(1, k):
+                v = Fraction(float(yf[inv[t * k + j], h]))
+                acc = _f32_rne(v * Fraction(float(w[t, j])) + Fraction(acc))
+                unf = _f32_rne(Fraction(_f32_rne(v * Fraction(float(w[t, j])))) + Fraction(unf))
+            ref = bf16_bits(torch.tensor([acc], dtype=torch.float32).to(torch.bfloat16))[0]
+            n_unfused_differs += acc != unf
+            assert out[t, h] == ref, (t, h)
+    assert n_unfused_differs > 0    # the vectors do separate fused from unfused
+
+
+def test_finalize_metamorphic_scaling():
+    rng = np.random.default_rng(8)
+    T, H, k = 8, 32, 4
+    yt = torch.from_numpy(rng.standard_normal((T * k, H)).astype(np.float32)).to(torch.bfloat16)
+    w = rng.random((T, k)).astype(np.float32)
+    inv = np.arange(T * k, dtype=np.int32)
+    a = bits_to_bf16(oracle.finalize(bf16_bits(yt), w, inv, T, H, k)).float()
+    b = bits_to_bf16(oracle.finalize(bf16_bits(yt * 2), w, inv, T, H, k)).float()
+    assert torch.equal(b, a * 2)
+
+
+# ------------------------------------------------- FFN / the whole layer --
+
+def dense_brute_force(inp, k, fmt="bf16"):
+    """Every token through every expert in float64 (torch matmul), combined
+    with weight 0 for unselected experts; routing from torch softmax/sort.
+    Rounding points as in the layer: fp32 accumulators, bf16 act and y."""
+    x = inp["hidden"].double()
+    logits = inp["logits"]
+    T, H = x.shape
+    E = logits.shape[1]
+    if fmt == "bf16":
+        Wgu = inp["w_gu"].double()
+        Wd = inp["w_d"].double()
+    else:
+        Wgu = torch.stack([bits_to_bf16(oracle.dequant_int4(inp["w_gu"][e], inp["w_gu_scales"][e]))
+                           for e in range(E)]).double()
+        Wd = torch.stack([bits_to_bf16(oracle.dequant_int4(inp["w_d"][e], inp["w_d_scales"][e]))
+                          for e in range(E)]).double()
+    I = Wd.shape[2]
+    p = torch.softmax(logits.double(), 1)
+    order = torch.sort(logits, dim=1, descending=True, stable=True).indices[:, :k]
+    sel = torch.gather(p, 1, order)
+    wsel = sel / sel.sum(1, keepdim=True)
+    wfull = torch.zeros(T, E, dtype=torch.float64).scatter_(1, order, wsel)
+    out = torch.zeros(T, H, dtype=torch.float64)
+    for e in range(E):
+        g = (x @ Wgu[e, :I].T).float().double()
+        u = (x @ Wgu[e, I:].T).float().double()
+        act = (g / (1 + torch.exp(-g)) * u).float().to(torch.bfloat16).double()
+        y = (act @ Wd[e].T).float().to(torch.bfloat16).double()
+        out += wfull[:, e:e + 1] * y
+    return out
+
+
+SHAPES = [
+    moe_synth.get_config("tiny"),
+    moe_synth.get_config("tiny", T=1),
+    moe_synth.get_config("tiny", k=1),
+    moe_synth.get_config("tiny", k=8),                 # k = E
+    moe_synth.get_config("tiny", E=1, k=1),
+    moe_synth.get_config("tiny", T=33, H=72, I=40, E=5, k=3),
+    moe_synth.get_config("skewed", T=24, H=96, I=48, E=16, k=3),
+    moe_synth.get_config("qwen3_prefill", T=20, H=64, I=32, E=12, k=4),
+]
+
+
+@pytest.mark.parametrize("cfg", SHAPES, ids=lambda c: f"T{c.T}H{c.H}I{c.I}E{c.E}k{c.k}")
+def test_forward_matches_dense_brute_force(cfg):
+    inp = moe_synth.gen_inputs(cfg, seed=11)
+    r = oracle.forward(inp, cfg.k)
+    ref = dense_brute_force(inp, cfg.k)
+    out = bits_to_bf16(r["out"]).double()
+    err = (out - ref).abs()
+    # oracle: fp32 slot-ordered combine then bf16; brute force: float64 sum.
+    assert torch.all(err <= ref.abs() * 2.0 ** -8 + 1e-6), float(err.max())
+    assert np.array_equal(r["counts"].sum(), cfg.T * cfg.k)
+
+
+def test_forward_int4_matches_dense_brute_force():
+    cfg = moe_synth.MoeConfig("int4_small", T=12, H=256, I=128, E=6, k=2, fmt="int4_g128")
+    inp = moe_synth.gen_inputs(cfg, seed=12)
+    r = oracle.forward(inp, cfg.k, fmt=cfg.fmt)
+    ref = dense_brute_force(inp, cfg.k, fmt=cfg.fmt)
+    out = bits_to_bf16(r["out"]).double()
+    assert torch.all((out - ref).abs() <= ref.abs() * 2.0 ** -8 + 1e-6)
+
+
+def test_forward_closed_forms():
+    cfg = moe_synth.get_config("tiny")
+    inp = moe_synth.gen_inputs(cfg, seed=13)
+    # hidden = 0 -> g = u = 0 -> act = 0 -> out = 0
+    z = dict(inp, hidden=torch.zeros_like(inp["hidden"]))
+    assert np.all((oracle.forward(z, cfg.k)["out"] & 0x7FFF) == 0)
+    # W_down = 0 -> out = 0
+    z = dict(inp, w_d=torch.zeros_like(inp["w_d"]))
+    assert np.all((oracle.forward(z, cfg.k)["out"] & 0x7FFF) == 0)
+    base = bits_to_bf16(oracle.forward(inp, cfg.k)["out"]).float()
+    # doubling W_down doubles y exactly, hence the output
+    z = dict(inp, w_d=inp["w_d"] * 2)
+    assert torch.equal(bits_to_bf16(oracle.forward(z, cfg.k)["out"]).float(), base * 2)
+    # doubling the up rows doubles act exactly (linear in u) ...
+    I = cfg.I
+    wgu = inp["w_gu"].clone()
+    wgu[:, I:] *= 2
+    assert torch.equal(bits_to_bf16(oracle.forward(dict(inp, w_gu=wgu), cfg.k)["out"]).float(), base * 2)
+    # ... but doubling the gate rows does not (silu is not linear): gate/up not swapped
+    wgu = inp["w_gu"].clone()
+    wgu[:, :I] *= 2
+    other = bits_to_bf16(oracle.forward(dict(inp, w_gu=wgu), cfg.k)["out"]).float()
+    assert not torch.allclose(other, base * 2, rtol=1e-2, atol=1e-3)
+
+
+def test_forward_k1_is_the_single_expert_output():
+    cfg = moe_synth.get_config("tiny", k=1)
+    inp = moe_synth.gen_inputs(cfg, seed=14)
+    r = oracle.forward(inp, 1)
+    for t in range(cfg.T):
+        e = int(r["ids"][t, 0])
+        _, y = oracle.expert_ffn(inp["hidden"][t], inp["w_gu"][e], inp["w_d"][e], cfg.H, cfg.I)
+        assert np.array_equal(r["out"][t], y)
+
+
+def test_forward_tokens_agrees_with_forward():
+    cfg = moe_synth.get_config("tiny", T=40, E=8, k=3)
+    inp = moe_synth.gen_inputs(cfg, seed=15)
+    r = oracle.forward(inp, cfg.k)
+    toks = [0, 7, 39, 21]
+    ids, w, out = oracle.forward_tokens(inp, cfg.k, toks)
+    assert np.array_equal(ids, r["ids"][toks])
+    assert np.array_equal(w, r["w"][toks])
+    assert np.array_equal(out, r["out"][toks])
+
+
+def test_forward_intermediates_are_consistent():
+    cfg = moe_synth.get_config("tiny", T=21)
+    inp = moe_synth.gen_inputs(cfg, seed=16)
+    r = oracle.forward(inp, cfg.k)
+    hp = oracle.gather(inp["hidden"], r["perm"], cfg.k)
+    for row in (0, 5, cfg.P - 1):
+        p = int(r["perm"][row])
+        e = int(r["ids"].reshape(-1)[p])
+        act, y = oracle.expert_ffn(hp[row], inp["w_gu"][e], inp["w_d"][e], cfg.H, cfg.I)
+        assert np.array_equal(act, r["act"][row]) and np.array_equal(y, r["y"][row])
+
+
+# ------------------------------------------------------- input generator --
+
+def test_synthetic_inputs_are_deterministic_and_shaped():
+    cfg = moe_synth.get_config("tiny")
+    a = moe_synth.gen_inputs(cfg, seed=0)
+    b = moe_synth.gen_inputs(cfg, seed=0)
+    c = moe_synth.gen_inputs(cfg, seed=1)
+    for n in a:
+        assert torch.equal(a[n], b[n])
+    assert not torch.equal(a["hidden"], c["hidden"])
+    assert a["w_gu"].shape == (8, 128, 128) and a["w_d"].shape == (8, 128, 64)
+    # a single expert regenerates alone
+    one = moe_synth.gen_expert_weights(cfg, 5, seed=0)
+    assert torch.equal(one["w_gu"], a["w_gu"][5])
+
+
+def test_synthetic_distributions():
+    cfg = moe_synth.get_config("qwen3_decode")
+    w = moe_synth.gen_expert_weights(cfg, 0)["w_gu"].float()
+    assert abs(w.std().item() - 0.02) < 5e-4 and abs(w.mean().item()) < 5e-4
+    lg = moe_synth.gen_logits(moe_synth.get_config("skewed"))
+    col = lg.mean(0)
+    assert torch.all(col[1:] < col[:-1] + 0.2)       # Zipf popularity falls with rank
+    qcfg = moe_synth.MoeConfig("q", T=4, H=256, I=128, E=2, k=1, fmt="int4_g128")
+    q = moe_synth.gen_expert_weights(qcfg, 0)
+    nib = torch.cat([(q["w_gu"] & 15).flatten(), (q["w_gu"] >> 4).flatten()]).long()
+    hist = torch.bincount(nib, minlength=16).double()
+    assert hist.min() > 0.8 * hist.mean()
+    s = q["w_gu_scales"].float()
+    assert s.min() >= 0.0019 and s.max() <= 0.0201
