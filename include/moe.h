@@ -1,0 +1,184 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) MoE expert-FFN layer library,
+ * libmoe_b200.so.
+ *
+ * The layer (InfiniLM PR #500 Qwen3-MoE report, §2.2; FlashInfer PR #7196
+ * analysis, §1-§2):
+ *
+ *   route     top-k of a softmax over E router logits, renormalised over k
+ *   permute   bucket the T*k (token, expert) pairs by expert: counts, offsets,
+ *             a stable permutation, and optionally the gathered activations
+ *   gate/up   per expert, act = bf16(silu(x W_g^T) * (x W_u^T)), fp32 accumulate
+ *   down      per expert, y = bf16(act W_d^T), fp32 accumulate
+ *   finalize  out[t] = bf16(w_0 v_0 (+) w_1 v_1 (+) ...), slot order, fp32
+ *
+ * Conventions (all entry points):
+ *  - Every buffer argument is a DEVICE pointer unless its name ends in
+ *    "_host". The caller allocates and frees every buffer; the library never
+ *    allocates device or host memory on these paths.
+ *  - Row-major, contiguous. bf16 values are passed as their 16-bit patterns
+ *    (moe_bf16_t). Index arrays are int32.
+ *  - All work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream) and is asynchronous unless stated otherwise.
+ *  - Arguments are validated before anything is enqueued; a non-OK status
+ *    means nothing was launched. T = 0 is valid and enqueues nothing.
+ *  - Shape limits: 1 <= E <= 1024, 1 <= top_k <= min(E, 32), T*top_k < 2^31;
+ *    H and I multiples of 8 (multiples of 128 for MOE_W_INT4_G128).
+ *    Device pointers must be 16-byte aligned (4-byte for logits/topk_w and
+ *    the int32 arrays).
+ *  - Pair ids: p = t*top_k + j for token t and slot j. Slot order is
+ *    descending logit; equal logits go to the lower expert id.
+ *  - No C++ exception crosses this interface. Entry points are reentrant
+ *    given distinct workspaces and outputs.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,          /* null pointer, bad size, misalignment */
+    MOE_ERR_UNSUPPORTED = 2,          /* valid but outside this build's limits */
+    MOE_ERR_WORKSPACE_TOO_SMALL = 3,  /* ws_bytes below the matching *_workspace_size */
+    MOE_ERR_CUDA = 4,                 /* a CUDA runtime/driver call failed */
+    MOE_ERR_DEVICE_FLAG = 5           /* a kernel raised the device error flag */
+} moe_status_t;
+
+typedef enum {
+    MOE_W_BF16 = 0,        /* bf16 weights */
+    MOE_W_INT4_G128 = 1    /* W4A16: int4 weights, one bf16 scale per 128 K */
+} moe_weight_fmt_t;
+
+/* Layer shape. T tokens, hidden size H, expert intermediate size I, E experts,
+ * top_k experts per token, fmt a moe_weight_fmt_t. */
+typedef struct {
+    int32_t T, H, I, E, top_k, fmt;
+} moe_shape_t;
+
+typedef uint16_t moe_bf16_t;   /* bit pattern of a bfloat16 value */
+typedef void *moe_stream_t;    /* cudaStream_t */
+
+/* Bytes of device workspace moe_forward needs for this shape (0 if the shape
+ * is invalid). It holds the routing, the permutation, the gathered rows
+ * [T*k,H], act [T*k,I] and y [T*k,H]. */
+MOE_API size_t moe_workspace_size(const moe_shape_t *shape);
+
+/* Bytes of scratch moe_permute needs (may be 0). */
+MOE_API size_t moe_permute_workspace_size(const moe_shape_t *shape);
+
+/* Route. InfiniLM PR #500 report §2.1/§2.4 (top-k softmax routing) with
+ * renormalisation over the selected experts.
+ *   logits   [T,E] fp32 (finite values; NaN is treated as -inf)
+ *   topk_ids [T,top_k] int32 out: expert ids in slot order
+ *   topk_w   [T,top_k] fp32 out: w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0),
+ *            sums to one; one warp per token, expf, fp32 sum in slot order. */
+MOE_API moe_status_t moe_route(const float *logits, const moe_shape_t *shape,
+                       int32_t *topk_ids, float *topk_w, moe_stream_t stream);
+
+/* Permute (bucketing). InfiniLM PR #500 report §2.2 step 1 (per-expert counts
+ * and a permutation) and step 2 (gather by that permutation), done on the
+ * device with no host synchronisation.
+ *   topk_ids    [T*top_k] int32 expert ids (0 <= id < E)
+ *   counts      [E] out: pairs routed to each expert
+ *   offsets     [E+1] out: exclusive prefix sum of counts; offsets[E] = T*top_k
+ *   perm        [T*top_k] out: perm[r] = pair id of permuted row r; rows of one
+ *               expert are contiguous and in ascending pair id (stable)
+ *   inv_perm    [T*top_k] out: inv_perm[perm[r]] = r
+ *   hidden      [T,H] bf16, may be NULL (then hidden_perm must be NULL)
+ *   hidden_perm [T*top_k,H] bf16 out, may be NULL: hidden_perm[r] = hidden[perm[r]/top_k]
+ *   ws, ws_bytes scratch of at least moe_permute_workspace_size() bytes.
+ * Deterministic. An id outside [0,E) raises the device error flag; that pair
+ * is then dropped (inv_perm = -1) and the sums above no longer hold. */
+MOE_API moe_status_t moe_permute(const int32_t *topk_ids, const moe_shape_t *shape,
+                         int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv_perm,
+                         const moe_bf16_t *hidden, moe_bf16_t *hidden_perm,
+                         void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* Grouped GEMM gate/up with fused SwiGLU. InfiniLM PR #500 report §2.2 step 2
+ * (grouped GEMM over all experts in one call, then SwiGLU); FlashInfer PR
+ * #7196 analysis §2 (tokens on the MMA N side with a runtime N per tile).
+ *   a       [T*top_k,H] bf16 rows in permuted order (hidden_perm)
+ *   perm    must be NULL (a gather fused into the operand load is not offered)
+ *   offsets [E+1] from moe_permute
+ *   w_gu    MOE_W_BF16: [E,2I,H] bf16, rows [0,I) gate, rows [I,2I) up.
+ *           MOE_W_INT4_G128: [E,2I,H/2] bytes, low nibble = even K index,
+ *           two's complement int4; w_gu_scales [E,2I,H/128] bf16.
+ *           w = bf16(q * scale) is formed in shared memory before the MMA.
+ *   act     [T*top_k,I] bf16 out: act = bf16(silu(g) * u), g/u fp32 accumulated.
+ * Experts with no rows cost no tiles. */
+MOE_API moe_status_t moe_grouped_gemm_swiglu(const moe_bf16_t *a, const int32_t *perm, const int32_t *offsets,
+                                     const void *w_gu, const moe_bf16_t *w_gu_scales,
+                                     const moe_shape_t *shape, moe_bf16_t *act, moe_stream_t stream);
+
+/* Grouped GEMM down. InfiniLM PR #500 report §2.2 step 2 (third grouped GEMM).
+ *   act     [T*top_k,I] bf16, offsets [E+1]
+ *   w_d     MOE_W_BF16: [E,H,I] bf16. MOE_W_INT4_G128: [E,H,I/2] bytes with
+ *           w_d_scales [E,H,I/128] bf16.
+ *   y       [T*top_k,H] bf16 out: unscaled down projection, permuted row order. */
+MOE_API moe_status_t moe_grouped_gemm_down(const moe_bf16_t *act, const int32_t *offsets,
+                                   const void *w_d, const moe_bf16_t *w_d_scales,
+                                   const moe_shape_t *shape, moe_bf16_t *y, moe_stream_t stream);
+
+/* Finalize / unpermute. FlashInfer PR #7196 analysis §1 (moe_finalize):
+ *   out[t,h] = bf16_rne(acc), acc = v_0 * w_0 (fp32 multiply, round to
+ *   nearest), then acc = fma(v_j, w_j, acc) for j = 1..top_k-1 (round to
+ *   nearest, no flush-to-zero), v_j = y[inv_perm[t*top_k+j], h],
+ *   w_j = topk_w[t*top_k+j]. Signed zeros and subnormals are kept.
+ *   A row index outside [0, T*top_k) reads as 0. Bit-exact and deterministic. */
+MOE_API moe_status_t moe_finalize(const moe_bf16_t *y, const float *topk_w, const int32_t *inv_perm,
+                          const moe_shape_t *shape, moe_bf16_t *out, moe_stream_t stream);
+
+/* The whole layer: route, permute (with gather), gate/up + SwiGLU, down,
+ * finalize, enqueued on one stream with no host synchronisation.
+ *   hidden [T,H] bf16, logits [T,E] fp32, weights as above, out [T,H] bf16.
+ *   ws: at least moe_workspace_size(shape) bytes, 256-byte aligned. */
+MOE_API moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits,
+                         const void *w_gu, const moe_bf16_t *w_gu_scales,
+                         const void *w_d, const moe_bf16_t *w_d_scales,
+                         const moe_shape_t *shape, moe_bf16_t *out,
+                         void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* moe_forward with hidden, logits and out in HOST memory (page-locked memory
+ * gives asynchronous copies). Copies the inputs into the workspace, runs the
+ * layer and copies out back, all on `stream`, then waits for the stream:
+ * when it returns OK, out_host holds the result. Weights stay device-resident.
+ *   ws: at least moe_forward_host_workspace_size(shape) bytes. */
+MOE_API size_t moe_forward_host_workspace_size(const moe_shape_t *shape);
+MOE_API moe_status_t moe_forward_host(const moe_bf16_t *hidden_host, const float *logits_host,
+                              const void *w_gu, const moe_bf16_t *w_gu_scales,
+                              const void *w_d, const moe_bf16_t *w_d_scales,
+                              const moe_shape_t *shape, moe_bf16_t *out_host,
+                              void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* W4A16 weight decoding on its own (the step the int4 GEMMs run in shared
+ * memory). FlashInfer PR #7196 analysis §2-§3.
+ *   q [rows, K/2] bytes, scales [rows, K/128] bf16 -> out [rows, K] bf16,
+ *   out = bf16_rne(q * scale). K a multiple of 128. */
+MOE_API moe_status_t moe_dequant_int4(const uint8_t *q, const moe_bf16_t *scales, int32_t rows, int32_t K,
+                              moe_bf16_t *out, moe_stream_t stream);
+
+/* Device error flag of the current device: waits for all work on the device,
+ * stores the flag in *code (0 = none; 1 = bad expert id; 2 = a pipeline wait
+ * timed out) and clears it. */
+MOE_API moe_status_t moe_get_device_error(int32_t *code);
+
+/* Static description of a status code. */
+MOE_API const char *moe_status_string(moe_status_t status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

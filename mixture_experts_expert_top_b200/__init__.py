@@ -1,0 +1,216 @@
+"""Python binding of libmoe_b200, the B200 (sm_100a) MoE expert-FFN layer.
+
+Argument marshalling only: every function here passes torch tensors' device
+pointers and sizes to the C entry point of the same name (include/moe.h) and
+raises MoeError on a non-OK status. All computation runs in the library's
+CUDA kernels. If the library is missing this module raises on first use; it
+has no fallback of any kind.
+
+The layer: top-k softmax routing -> permute (bucket by expert, gather) ->
+grouped GEMM gate/up + SwiGLU -> grouped GEMM down -> weighted finalize
+(InfiniLM PR #500 Qwen3-MoE report §2.2; FlashInfer PR #7196 analysis §1-§2).
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+__all__ = [
+    "MoeError", "Shape", "lib", "library_path", "FMT_BF16", "FMT_INT4_G128",
+    "moe_workspace_size", "moe_permute_workspace_size", "moe_forward_host_workspace_size",
+    "moe_route", "moe_permute", "moe_grouped_gemm_swiglu", "moe_grouped_gemm_down",
+    "moe_finalize", "moe_forward", "moe_forward_host", "moe_dequant_int4",
+    "moe_get_device_error", "moe_status_string", "forward",
+]
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(HERE, "libmoe_b200.so")
+
+FMT_BF16 = 0
+FMT_INT4_G128 = 1
+
+STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
+          3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_FLAG"}
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
+                ("E", ctypes.c_int32), ("top_k", ctypes.c_int32), ("fmt", ctypes.c_int32)]
+
+    @classmethod
+    def of(cls, T, H, I, E, top_k, fmt=FMT_BF16) -> "Shape":
+        if isinstance(fmt, str):
+            fmt = {"bf16": FMT_BF16, "int4_g128": FMT_INT4_G128}[fmt]
+        return cls(int(T), int(H), int(I), int(E), int(top_k), int(fmt))
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise RuntimeError(f"{library_path} is missing: build it with "
+                               "`python -m mixture_experts_expert_top_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(library_path)
+        vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
+        sp = ctypes.POINTER(Shape)
+        sigs = {
+            "moe_workspace_size": ([sp], sz),
+            "moe_permute_workspace_size": ([sp], sz),
+            "moe_forward_host_workspace_size": ([sp], sz),
+            "moe_route": ([vp, sp, vp, vp, vp], ctypes.c_int),
+            "moe_permute": ([vp, sp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+            "moe_grouped_gemm_swiglu": ([vp, vp, vp, vp, vp, sp, vp, vp], ctypes.c_int),
+            "moe_grouped_gemm_down": ([vp, vp, vp, vp, sp, vp, vp], ctypes.c_int),
+            "moe_finalize": ([vp, vp, vp, sp, vp, vp], ctypes.c_int),
+            "moe_forward": ([vp, vp, vp, vp, vp, vp, sp, vp, vp, sz, vp], ctypes.c_int),
+            "moe_forward_host": ([vp, vp, vp, vp, vp, vp, sp, vp, vp, sz, vp], ctypes.c_int),
+            "moe_dequant_int4": ([vp, vp, i32, i32, vp, vp], ctypes.c_int),
+            "moe_get_device_error": ([ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
+            "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        }
+        for name, (args, res) in sigs.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+# ---- marshalling helpers ---------------------------------------------------
+
+def _p(t) -> Optional[int]:
+    """Device (or host) address of a tensor, None for None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libmoe_b200 must be contiguous")
+    return t.data_ptr()
+
+
+def _s(stream) -> Optional[int]:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _check(status: int, where: str) -> None:
+    if status != 0:
+        raise MoeError(status, where)
+
+
+def _shape(shape) -> Shape:
+    if isinstance(shape, Shape):
+        return shape
+    return Shape.of(*shape)
+
+
+# ---- entry points (same names as the C ABI) --------------------------------
+
+def moe_workspace_size(shape) -> int:
+    return int(lib().moe_workspace_size(ctypes.byref(_shape(shape))))
+
+
+def moe_permute_workspace_size(shape) -> int:
+    return int(lib().moe_permute_workspace_size(ctypes.byref(_shape(shape))))
+
+
+def moe_forward_host_workspace_size(shape) -> int:
+    return int(lib().moe_forward_host_workspace_size(ctypes.byref(_shape(shape))))
+
+
+def moe_route(logits, shape, topk_ids, topk_w, stream=None) -> None:
+    _check(lib().moe_route(_p(logits), ctypes.byref(_shape(shape)), _p(topk_ids), _p(topk_w), _s(stream)),
+           "moe_route")
+
+
+def moe_permute(topk_ids, shape, counts, offsets, perm, inv_perm, hidden=None, hidden_perm=None,
+                ws=None, stream=None) -> None:
+    nbytes = 0 if ws is None else ws.numel() * ws.element_size()
+    _check(lib().moe_permute(_p(topk_ids), ctypes.byref(_shape(shape)), _p(counts), _p(offsets), _p(perm),
+                             _p(inv_perm), _p(hidden), _p(hidden_perm), _p(ws), nbytes, _s(stream)),
+           "moe_permute")
+
+
+def moe_grouped_gemm_swiglu(a, perm, offsets, w_gu, w_gu_scales, shape, act, stream=None) -> None:
+    _check(lib().moe_grouped_gemm_swiglu(_p(a), _p(perm), _p(offsets), _p(w_gu), _p(w_gu_scales),
+                                         ctypes.byref(_shape(shape)), _p(act), _s(stream)),
+           "moe_grouped_gemm_swiglu")
+
+
+def moe_grouped_gemm_down(act, offsets, w_d, w_d_scales, shape, y, stream=None) -> None:
+    _check(lib().moe_grouped_gemm_down(_p(act), _p(offsets), _p(w_d), _p(w_d_scales),
+                                       ctypes.byref(_shape(shape)), _p(y), _s(stream)),
+           "moe_grouped_gemm_down")
+
+
+def moe_finalize(y, topk_w, inv_perm, shape, out, stream=None) -> None:
+    _check(lib().moe_finalize(_p(y), _p(topk_w), _p(inv_perm), ctypes.byref(_shape(shape)), _p(out), _s(stream)),
+           "moe_finalize")
+
+
+def moe_forward(hidden, logits, w_gu, w_gu_scales, w_d, w_d_scales, shape, out, ws, stream=None) -> None:
+    nbytes = ws.numel() * ws.element_size()
+    _check(lib().moe_forward(_p(hidden), _p(logits), _p(w_gu), _p(w_gu_scales), _p(w_d), _p(w_d_scales),
+                             ctypes.byref(_shape(shape)), _p(out), _p(ws), nbytes, _s(stream)),
+           "moe_forward")
+
+
+def moe_forward_host(hidden_host, logits_host, w_gu, w_gu_scales, w_d, w_d_scales, shape, out_host, ws,
+                     stream=None) -> None:
+    nbytes = ws.numel() * ws.element_size()
+    _check(lib().moe_forward_host(_p(hidden_host), _p(logits_host), _p(w_gu), _p(w_gu_scales), _p(w_d),
+                                  _p(w_d_scales), ctypes.byref(_shape(shape)), _p(out_host), _p(ws), nbytes,
+                                  _s(stream)),
+           "moe_forward_host")
+
+
+def moe_dequant_int4(q, scales, rows: int, K: int, out, stream=None) -> None:
+    _check(lib().moe_dequant_int4(_p(q), _p(scales), int(rows), int(K), _p(out), _s(stream)), "moe_dequant_int4")
+
+
+def moe_get_device_error() -> int:
+    code = ctypes.c_int32(0)
+    _check(lib().moe_get_device_error(ctypes.byref(code)), "moe_get_device_error")
+    return int(code.value)
+
+
+def moe_status_string(status: int) -> str:
+    return lib().moe_status_string(int(status)).decode()
+
+
+# ---- convenience -----------------------------------------------------------
+
+def forward(hidden: torch.Tensor, logits: torch.Tensor, w_gu: torch.Tensor, w_d: torch.Tensor, top_k: int,
+            w_gu_scales: Optional[torch.Tensor] = None, w_d_scales: Optional[torch.Tensor] = None,
+            out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """moe_forward on device tensors; allocates out and the workspace with
+    torch when they are not given. hidden [T,H] bf16, logits [T,E] fp32,
+    w_gu [E,2I,H] bf16 (or uint8 [E,2I,H/2] + scales), w_d [E,H,I] (or uint8)."""
+    T, H = hidden.shape
+    E = logits.shape[1]
+    fmt = FMT_INT4_G128 if w_gu.dtype == torch.uint8 else FMT_BF16
+    I = w_d.shape[2] * (2 if fmt == FMT_INT4_G128 else 1)
+    shape = Shape.of(T, H, I, E, top_k, fmt)
+    if out is None:
+        out = torch.empty(T, H, dtype=torch.bfloat16, device=hidden.device)
+    if ws is None:
+        ws = torch.empty(max(moe_workspace_size(shape), 1), dtype=torch.uint8, device=hidden.device)
+    moe_forward(hidden, logits, w_gu, w_gu_scales, w_d, w_d_scales, shape, out, ws, stream)
+    return out

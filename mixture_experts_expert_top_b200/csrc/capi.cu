@@ -1,0 +1,317 @@
+// capi.cu -- the extern "C" entry points of libmoe_b200 (declared and
+// documented in include/moe.h): argument validation, workspace layout and the
+// launch sequence of the whole layer. Compute lives in the kernel files.
+#include <stdint.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "launch.h"
+#include "moe.h"
+
+// Device error flag word (0 = none), one per device that loads the library.
+static __device__ int g_moe_error_flag;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+int *error_flag_ptr() {
+    static int *ptrs[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!ptrs[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_moe_error_flag) == cudaSuccess) ptrs[dev] = static_cast<int *>(p);
+    }
+    return ptrs[dev];
+}
+
+inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+moe_status_t check_shape(const moe_shape_t *s) {
+    if (!s) return MOE_ERR_INVALID_ARG;
+    if (s->T < 0 || s->H <= 0 || s->I <= 0 || s->E < 1 || s->top_k < 1 || s->top_k > s->E)
+        return MOE_ERR_INVALID_ARG;
+    if (s->fmt != MOE_W_BF16 && s->fmt != MOE_W_INT4_G128) return MOE_ERR_INVALID_ARG;
+    if (s->E > 1024 || s->top_k > 32) return MOE_ERR_UNSUPPORTED;
+    if (s->H % 8 || s->I % 8) return MOE_ERR_UNSUPPORTED;
+    if (s->fmt == MOE_W_INT4_G128 && (s->H % 128 || s->I % 128)) return MOE_ERR_UNSUPPORTED;
+    if (static_cast<long long>(s->T) * s->top_k >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
+    if (static_cast<long long>(s->E) * 2 * s->I >= (1LL << 31) || static_cast<long long>(s->E) * s->H >= (1LL << 31))
+        return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+moe_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Byte offsets of moe_forward's intermediates inside the workspace.
+struct Layout {
+    size_t ids, w, counts, offsets, perm, inv, scratch, hperm, act, y;
+    size_t hidden_in, logits_in, out_st;   // staging for moe_forward_host
+    size_t total;
+};
+
+Layout layout(const moe_shape_t *s, bool host) {
+    const size_t P = static_cast<size_t>(s->T) * s->top_k;
+    Layout L;
+    size_t o = 0;
+    auto take = [&](size_t bytes) {
+        const size_t at = o;
+        o = align256(o + bytes);
+        return at;
+    };
+    L.ids = take(P * 4);
+    L.w = take(P * 4);
+    L.counts = take(static_cast<size_t>(s->E) * 4);
+    L.offsets = take(static_cast<size_t>(s->E + 1) * 4);
+    L.perm = take(P * 4);
+    L.inv = take(P * 4);
+    L.scratch = take(moe::permute_scratch_bytes(static_cast<long long>(P), s->E));
+    L.hperm = take(P * s->H * 2);
+    L.act = take(P * s->I * 2);
+    L.y = take(P * s->H * 2);
+    L.hidden_in = L.logits_in = L.out_st = 0;
+    if (host) {
+        L.hidden_in = take(static_cast<size_t>(s->T) * s->H * 2);
+        L.logits_in = take(static_cast<size_t>(s->T) * s->E * 4);
+        L.out_st = take(static_cast<size_t>(s->T) * s->H * 2);
+    }
+    L.total = o;
+    return L;
+}
+
+moe::GemmArgs gemm_args(const moe_shape_t *s, const void *a, const int32_t *offsets, const void *w,
+                        const moe_bf16_t *scales, bool swiglu, moe_bf16_t *out) {
+    moe::GemmArgs g;
+    g.a = a;
+    g.offsets = offsets;
+    g.w = w;
+    g.w_scales = scales;
+    g.P = s->T * s->top_k;
+    g.E = s->E;
+    g.K = swiglu ? s->H : s->I;
+    g.m_out = swiglu ? s->I : s->H;
+    g.w_rows = swiglu ? 2 * s->I : s->H;
+    g.fmt = s->fmt;
+    g.swiglu = swiglu;
+    g.out = out;
+    g.err = error_flag_ptr();
+    return g;
+}
+
+moe_status_t check_weights(const moe_shape_t *s, const void *w, const moe_bf16_t *scales) {
+    if (!w || !aligned(w, 16)) return MOE_ERR_INVALID_ARG;
+    if (s->fmt == MOE_W_INT4_G128) {
+        if (!scales || !aligned(scales, 4)) return MOE_ERR_INVALID_ARG;
+    } else if (scales) {
+        return MOE_ERR_INVALID_ARG;
+    }
+    return MOE_OK;
+}
+
+moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const void *w_gu,
+                            const moe_bf16_t *w_gu_scales, const void *w_d, const moe_bf16_t *w_d_scales,
+                            const moe_shape_t *s, moe_bf16_t *out, uint8_t *ws, const Layout &L,
+                            cudaStream_t st) {
+    const int T = s->T, k = s->top_k, E = s->E, H = s->H;
+    const int P = T * k;
+    auto *ids = reinterpret_cast<int32_t *>(ws + L.ids);
+    auto *w = reinterpret_cast<float *>(ws + L.w);
+    auto *counts = reinterpret_cast<int32_t *>(ws + L.counts);
+    auto *offsets = reinterpret_cast<int32_t *>(ws + L.offsets);
+    auto *perm = reinterpret_cast<int32_t *>(ws + L.perm);
+    auto *inv = reinterpret_cast<int32_t *>(ws + L.inv);
+    auto *hperm = reinterpret_cast<uint16_t *>(ws + L.hperm);
+    auto *act = reinterpret_cast<uint16_t *>(ws + L.act);
+    auto *y = reinterpret_cast<uint16_t *>(ws + L.y);
+    cudaError_t e;
+    if ((e = moe::launch_route(logits, T, E, k, ids, w, st)) != cudaSuccess) return cuda_status(e);
+    if ((e = moe::launch_permute(ids, P, E, counts, offsets, perm, inv, ws + L.scratch, error_flag_ptr(), st)) !=
+        cudaSuccess)
+        return cuda_status(e);
+    if ((e = moe::launch_gather(hidden, perm, P, H, k, hperm, st)) != cudaSuccess) return cuda_status(e);
+    if ((e = moe::launch_grouped_gemm(gemm_args(s, hperm, offsets, w_gu, w_gu_scales, true, act), st)) !=
+        cudaSuccess)
+        return cuda_status(e);
+    if ((e = moe::launch_grouped_gemm(gemm_args(s, act, offsets, w_d, w_d_scales, false, y), st)) != cudaSuccess)
+        return cuda_status(e);
+    return cuda_status(moe::launch_finalize(y, w, inv, T, H, k, out, st));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t moe_workspace_size(const moe_shape_t *shape) {
+    if (check_shape(shape) != MOE_OK) return 0;
+    return layout(shape, false).total;
+}
+
+size_t moe_forward_host_workspace_size(const moe_shape_t *shape) {
+    if (check_shape(shape) != MOE_OK) return 0;
+    return layout(shape, true).total;
+}
+
+size_t moe_permute_workspace_size(const moe_shape_t *shape) {
+    if (check_shape(shape) != MOE_OK) return 0;
+    return moe::permute_scratch_bytes(static_cast<long long>(shape->T) * shape->top_k, shape->E);
+}
+
+moe_status_t moe_route(const float *logits, const moe_shape_t *shape, int32_t *topk_ids, float *topk_w,
+                       moe_stream_t stream) {
+    moe_status_t st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (shape->T == 0) return MOE_OK;
+    if (!logits || !topk_ids || !topk_w || !aligned(logits, 4) || !aligned(topk_ids, 4) || !aligned(topk_w, 4))
+        return MOE_ERR_INVALID_ARG;
+    return cuda_status(moe::launch_route(logits, shape->T, shape->E, shape->top_k, topk_ids, topk_w,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_permute(const int32_t *topk_ids, const moe_shape_t *shape, int32_t *counts, int32_t *offsets,
+                         int32_t *perm, int32_t *inv_perm, const moe_bf16_t *hidden, moe_bf16_t *hidden_perm,
+                         void *ws, size_t ws_bytes, moe_stream_t stream) {
+    moe_status_t st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (shape->T == 0) return MOE_OK;
+    const long long P = static_cast<long long>(shape->T) * shape->top_k;
+    if (!counts || !offsets || !aligned(counts, 4) || !aligned(offsets, 4)) return MOE_ERR_INVALID_ARG;
+    if (P > 0 && (!topk_ids || !perm || !inv_perm || !aligned(topk_ids, 4) || !aligned(perm, 4) ||
+                  !aligned(inv_perm, 4)))
+        return MOE_ERR_INVALID_ARG;
+    if ((hidden == nullptr) != (hidden_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+    if (hidden && (!aligned(hidden, 16) || !aligned(hidden_perm, 16))) return MOE_ERR_INVALID_ARG;
+    const size_t need = moe::permute_scratch_bytes(P, shape->E);
+    if (need > 0 && (!ws || ws_bytes < need)) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (ws && !aligned(ws, 16)) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    cudaError_t e = moe::launch_permute(topk_ids, static_cast<int>(P), shape->E, counts, offsets, perm, inv_perm, ws,
+                                        error_flag_ptr(), s);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    if (hidden) e = moe::launch_gather(hidden, perm, static_cast<int>(P), shape->H, shape->top_k, hidden_perm, s);
+    return cuda_status(e);
+}
+
+moe_status_t moe_grouped_gemm_swiglu(const moe_bf16_t *a, const int32_t *perm, const int32_t *offsets,
+                                     const void *w_gu, const moe_bf16_t *w_gu_scales, const moe_shape_t *shape,
+                                     moe_bf16_t *act, moe_stream_t stream) {
+    moe_status_t st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (perm) return MOE_ERR_UNSUPPORTED;
+    if (shape->T == 0) return MOE_OK;
+    if (!a || !offsets || !act || !aligned(a, 16) || !aligned(act, 16) || !aligned(offsets, 4))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_weights(shape, w_gu, w_gu_scales)) != MOE_OK) return st;
+    return cuda_status(moe::launch_grouped_gemm(gemm_args(shape, a, offsets, w_gu, w_gu_scales, true, act),
+                                                static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_grouped_gemm_down(const moe_bf16_t *act, const int32_t *offsets, const void *w_d,
+                                   const moe_bf16_t *w_d_scales, const moe_shape_t *shape, moe_bf16_t *y,
+                                   moe_stream_t stream) {
+    moe_status_t st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (shape->T == 0) return MOE_OK;
+    if (!act || !offsets || !y || !aligned(act, 16) || !aligned(y, 16) || !aligned(offsets, 4))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_weights(shape, w_d, w_d_scales)) != MOE_OK) return st;
+    return cuda_status(moe::launch_grouped_gemm(gemm_args(shape, act, offsets, w_d, w_d_scales, false, y),
+                                                static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_finalize(const moe_bf16_t *y, const float *topk_w, const int32_t *inv_perm,
+                          const moe_shape_t *shape, moe_bf16_t *out, moe_stream_t stream) {
+    moe_status_t st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (shape->T == 0) return MOE_OK;
+    if (!y || !topk_w || !inv_perm || !out || !aligned(y, 16) || !aligned(out, 16) || !aligned(topk_w, 4) ||
+        !aligned(inv_perm, 4))
+        return MOE_ERR_INVALID_ARG;
+    return cuda_status(moe::launch_finalize(y, topk_w, inv_perm, shape->T, shape->H, shape->top_k, out,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits, const void *w_gu,
+                         const moe_bf16_t *w_gu_scales, const void *w_d, const moe_bf16_t *w_d_scales,
+                         const moe_shape_t *shape, moe_bf16_t *out, void *ws, size_t ws_bytes,
+                         moe_stream_t stream) {
+    moe_status_t st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (shape->T == 0) return MOE_OK;
+    if (!hidden || !logits || !out || !aligned(hidden, 16) || !aligned(out, 16) || !aligned(logits, 4))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_weights(shape, w_gu, w_gu_scales)) != MOE_OK) return st;
+    if ((st = check_weights(shape, w_d, w_d_scales)) != MOE_OK) return st;
+    const Layout L = layout(shape, false);
+    if (!ws || ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+    return forward_device(hidden, logits, w_gu, w_gu_scales, w_d, w_d_scales, shape, out,
+                          static_cast<uint8_t *>(ws), L, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_forward_host(const moe_bf16_t *hidden_host, const float *logits_host, const void *w_gu,
+                              const moe_bf16_t *w_gu_scales, const void *w_d, const moe_bf16_t *w_d_scales,
+                              const moe_shape_t *shape, moe_bf16_t *out_host, void *ws, size_t ws_bytes,
+                              moe_stream_t stream) {
+    moe_status_t st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (shape->T == 0) return MOE_OK;
+    if (!hidden_host || !logits_host || !out_host) return MOE_ERR_INVALID_ARG;
+    if ((st = check_weights(shape, w_gu, w_gu_scales)) != MOE_OK) return st;
+    if ((st = check_weights(shape, w_d, w_d_scales)) != MOE_OK) return st;
+    const Layout L = layout(shape, true);
+    if (!ws || ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+    auto *base = static_cast<uint8_t *>(ws);
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const size_t hb = static_cast<size_t>(shape->T) * shape->H * 2;
+    const size_t lb = static_cast<size_t>(shape->T) * shape->E * 4;
+    if (cudaMemcpyAsync(base + L.hidden_in, hidden_host, hb, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaMemcpyAsync(base + L.logits_in, logits_host, lb, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    st = forward_device(reinterpret_cast<const moe_bf16_t *>(base + L.hidden_in),
+                        reinterpret_cast<const float *>(base + L.logits_in), w_gu, w_gu_scales, w_d, w_d_scales,
+                        shape, reinterpret_cast<moe_bf16_t *>(base + L.out_st), base, L, s);
+    if (st != MOE_OK) return st;
+    if (cudaMemcpyAsync(out_host, base + L.out_st, hb, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return cuda_status(cudaStreamSynchronize(s));
+}
+
+moe_status_t moe_dequant_int4(const uint8_t *q, const moe_bf16_t *scales, int32_t rows, int32_t K,
+                              moe_bf16_t *out, moe_stream_t stream) {
+    if (rows < 0 || K <= 0 || K % 128) return MOE_ERR_INVALID_ARG;
+    if (rows == 0) return MOE_OK;
+    if (!q || !scales || !out || !aligned(q, 16) || !aligned(out, 16) || !aligned(scales, 2))
+        return MOE_ERR_INVALID_ARG;
+    return cuda_status(moe::launch_dequant_int4(q, scales, rows, K, out, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_get_device_error(int32_t *code) {
+    if (!code) return MOE_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_moe_error_flag, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_moe_error_flag, &zero, sizeof(int)) != cudaSuccess) return MOE_ERR_CUDA;
+    *code = v;
+    return MOE_OK;
+}
+
+const char *moe_status_string(moe_status_t status) {
+    switch (status) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported shape or option";
+        case MOE_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case MOE_ERR_CUDA: return "CUDA error";
+        case MOE_ERR_DEVICE_FLAG: return "device error flag raised";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

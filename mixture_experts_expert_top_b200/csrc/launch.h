@@ -1,0 +1,47 @@
+// launch.h -- host-side launchers of the libmoe_b200 kernels. Internal to the
+// library: the C ABI in include/moe.h validates arguments and calls these.
+// Every launcher enqueues on `stream` and returns the cudaGetLastError() of
+// its launches.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+// ---- route.cu
+cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s);
+
+// ---- permute.cu
+// Scratch bytes the permute needs for P pairs over E experts (0 when a
+// single CTA handles all pairs).
+size_t permute_scratch_bytes(long long P, int E);
+cudaError_t launch_permute(const int32_t *ids, int P, int E, int32_t *counts, int32_t *offsets, int32_t *perm,
+                           int32_t *inv_perm, void *scratch, int *err, cudaStream_t s);
+cudaError_t launch_gather(const uint16_t *hidden, const int32_t *perm, int P, int H, int k, uint16_t *hidden_perm,
+                          cudaStream_t s);
+
+// ---- finalize.cu
+cudaError_t launch_finalize(const uint16_t *y, const float *w, const int32_t *inv_perm, int T, int H, int k,
+                            uint16_t *out, cudaStream_t s);
+
+// ---- gemm_sm100.cu
+struct GemmArgs {
+    const void *a;              // activations [P, K] bf16, permuted row order
+    const int32_t *offsets;     // [E+1]
+    const void *w;              // weights (bf16 [E, rows, K] or int4 [E, rows, K/2])
+    const uint16_t *w_scales;   // int4 only: [E, rows, K/128] bf16
+    int P, E, K;
+    int m_out;                  // output features: I (gate/up) or H (down)
+    int w_rows;                 // weight rows per expert: 2I or H
+    int fmt;                    // 0 bf16, 1 int4 g128
+    bool swiglu;
+    uint16_t *out;              // [P, m_out] bf16
+    int *err;
+};
+cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t s);
+cudaError_t launch_dequant_int4(const uint8_t *q, const uint16_t *scales, int rows, int K, uint16_t *out,
+                                cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,259 @@
+// permute.cu -- bucketing of the (token, expert) pairs by expert, on the GPU.
+//
+// InfiniLM PR #500 Qwen3-MoE report, §2.2 step 1 buckets the routing indices
+// into per-expert token counts and a permutation (on the host there, behind a
+// device-to-host copy, §2.3); step 2 gathers the activations by that
+// permutation. Here both stay on the device:
+//   counts[e]  = #{p : ids[p] = e}
+//   offsets    = exclusive prefix sum of counts, offsets[E] = P
+//   perm[r]    = pair id p of permuted row r; within an expert, ascending p
+//   inv_perm[p] = r
+// Deterministic: the rank of a pair inside its expert is computed from
+// per-warp histograms in pair order, never from the order of atomics.
+//
+// Layout of the work: a CTA of 1024 threads (32 warps) owns a chunk of up to
+// kChunk consecutive pairs; warp w owns a contiguous slice of the chunk and
+// walks it 32 pairs at a time, using __match_any_sync to rank equal experts
+// inside each step. One CTA does everything when P <= kChunk; otherwise
+// three kernels run: per-chunk histograms, one scan CTA, per-chunk scatter.
+#include "common.cuh"
+#include "launch.h"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 1024;
+constexpr int kWarps = kThreads / 32;
+constexpr int kChunk = 8192;          // pairs per CTA
+
+// Slice of the chunk owned by each warp: a multiple of 32 pairs.
+__device__ __forceinline__ int warp_slice(int chunk_pairs) {
+    return ((chunk_pairs + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+}
+
+// hist[w*E + e] = pairs of warp w's slice routed to expert e.
+__device__ void warp_histograms(const int32_t *__restrict__ ids, int begin, int n, int E, int *hist, int *err) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    for (int i = threadIdx.x; i < kWarps * E; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    const int slice = warp_slice(n);
+    for (int it = 0; it < slice; it += 32) {
+        const int local = w * slice + it + lane;
+        const bool in = local < n;
+        const int e = in ? __ldg(ids + begin + local) : -1;
+        const bool ok = in && e >= 0 && e < E;
+        if (in && !ok) raise_error(err, kErrBadExpertId);
+        const unsigned m = __match_any_sync(0xffffffffu, ok ? e : -1);
+        if (ok && lane == __ffs(m) - 1) hist[w * E + e] += __popc(m);
+        __syncwarp();
+    }
+    __syncthreads();
+}
+
+// In place: hist[w*E+e] <- base[e] + sum_{w'<w} hist[w'*E+e]; returns nothing.
+__device__ void warp_bases(int E, int *hist, const int *base) {
+    for (int e = threadIdx.x; e < E; e += kThreads) {
+        int run = base[e];
+        for (int w = 0; w < kWarps; ++w) {
+            const int c = hist[w * E + e];
+            hist[w * E + e] = run;
+            run += c;
+        }
+    }
+    __syncthreads();
+}
+
+// Writes perm / inv_perm for the chunk, given per-warp starting rows.
+__device__ void warp_scatter(const int32_t *__restrict__ ids, int begin, int n, int E, int *hist,
+                             int32_t *__restrict__ perm, int32_t *__restrict__ inv_perm) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int slice = warp_slice(n);
+    const unsigned lt = (1u << lane) - 1u;
+    for (int it = 0; it < slice; it += 32) {
+        const int local = w * slice + it + lane;
+        const bool in = local < n;
+        const int e = in ? __ldg(ids + begin + local) : -1;
+        const bool ok = in && e >= 0 && e < E;
+        const unsigned m = __match_any_sync(0xffffffffu, ok ? e : -1);
+        if (ok) {
+            const int r = hist[w * E + e] + __popc(m & lt);
+            perm[r] = begin + local;
+            inv_perm[begin + local] = r;
+        } else if (in) {
+            inv_perm[begin + local] = -1;
+        }
+        __syncwarp();
+        if (ok && lane == __ffs(m) - 1) hist[w * E + e] += __popc(m);
+        __syncwarp();
+    }
+}
+
+// Exclusive scan of counts[0..E) into offsets[0..E], offsets[E] = total.
+// Also leaves offsets in shared memory `base`. E <= kThreads.
+__device__ void block_exclusive_scan(const int *vals, int E, int *base, int32_t *__restrict__ offsets) {
+    __shared__ int warp_sums[kWarps];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int v = threadIdx.x < E ? vals[threadIdx.x] : 0;
+    int x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) warp_sums[w] = x;
+    __syncthreads();
+    if (w == 0) {
+        int s = warp_sums[lane];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, s, o);
+            if (lane >= o) s += y;
+        }
+        warp_sums[lane] = s;   // inclusive over warps
+    }
+    __syncthreads();
+    const int excl = x - v + (w > 0 ? warp_sums[w - 1] : 0);
+    if (threadIdx.x < E) {
+        base[threadIdx.x] = excl;
+        offsets[threadIdx.x] = excl;
+    }
+    if (threadIdx.x == E - 1) offsets[E] = excl + v;
+    __syncthreads();
+}
+
+// All pairs in one CTA.
+__global__ void __launch_bounds__(kThreads, 1)
+permute_single_kernel(const int32_t *__restrict__ ids, int P, int E, int32_t *__restrict__ counts,
+                      int32_t *__restrict__ offsets, int32_t *__restrict__ perm, int32_t *__restrict__ inv_perm,
+                      int *err) {
+    extern __shared__ int smem[];
+    int *hist = smem;                 // [kWarps * E]
+    int *tot = hist + kWarps * E;     // [E]
+    int *base = tot + E;              // [E]
+    warp_histograms(ids, 0, P, E, hist, err);
+    for (int e = threadIdx.x; e < E; e += kThreads) {
+        int s = 0;
+        for (int w = 0; w < kWarps; ++w) s += hist[w * E + e];
+        tot[e] = s;
+        counts[e] = s;
+    }
+    __syncthreads();
+    block_exclusive_scan(tot, E, base, offsets);
+    warp_bases(E, hist, base);
+    warp_scatter(ids, 0, P, E, hist, perm, inv_perm);
+}
+
+// Multi-CTA pass 1: chunk_hist[c*E + e].
+__global__ void __launch_bounds__(kThreads, 1)
+permute_count_kernel(const int32_t *__restrict__ ids, int P, int E, int32_t *__restrict__ chunk_hist, int *err) {
+    extern __shared__ int smem[];
+    const int begin = blockIdx.x * kChunk;
+    const int n = min(kChunk, P - begin);
+    warp_histograms(ids, begin, n, E, smem, err);
+    for (int e = threadIdx.x; e < E; e += kThreads) {
+        int s = 0;
+        for (int w = 0; w < kWarps; ++w) s += smem[w * E + e];
+        chunk_hist[static_cast<size_t>(blockIdx.x) * E + e] = s;
+    }
+}
+
+// Multi-CTA pass 2 (one CTA): counts, offsets, and chunk_hist turned into the
+// first row of each (chunk, expert).
+__global__ void __launch_bounds__(kThreads, 1)
+permute_scan_kernel(int nchunks, int E, int32_t *__restrict__ chunk_hist, int32_t *__restrict__ counts,
+                    int32_t *__restrict__ offsets) {
+    extern __shared__ int smem[];
+    int *tot = smem;        // [E]
+    int *base = tot + E;    // [E]
+    for (int e = threadIdx.x; e < E; e += kThreads) {
+        int run = 0;
+        for (int c = 0; c < nchunks; ++c) {
+            const int v = chunk_hist[static_cast<size_t>(c) * E + e];
+            chunk_hist[static_cast<size_t>(c) * E + e] = run;
+            run += v;
+        }
+        tot[e] = run;
+        counts[e] = run;
+    }
+    __syncthreads();
+    block_exclusive_scan(tot, E, base, offsets);
+    for (int e = threadIdx.x; e < E; e += kThreads)
+        for (int c = 0; c < nchunks; ++c) chunk_hist[static_cast<size_t>(c) * E + e] += base[e];
+}
+
+// Multi-CTA pass 3: scatter each chunk from its per-expert first rows.
+__global__ void __launch_bounds__(kThreads, 1)
+permute_scatter_kernel(const int32_t *__restrict__ ids, int P, int E, const int32_t *__restrict__ chunk_base,
+                       int32_t *__restrict__ perm, int32_t *__restrict__ inv_perm) {
+    extern __shared__ int smem[];
+    int *hist = smem;                 // [kWarps * E]
+    int *base = hist + kWarps * E;    // [E]
+    const int begin = blockIdx.x * kChunk;
+    const int n = min(kChunk, P - begin);
+    for (int e = threadIdx.x; e < E; e += kThreads) base[e] = chunk_base[static_cast<size_t>(blockIdx.x) * E + e];
+    warp_histograms(ids, begin, n, E, hist, nullptr);
+    warp_bases(E, hist, base);
+    warp_scatter(ids, begin, n, E, hist, perm, inv_perm);
+}
+
+// hidden_perm[r] = hidden[perm[r] / k]: one warp per row, 16-byte vectors.
+__global__ void __launch_bounds__(256)
+gather_rows_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ perm, int P, int vecs_per_row,
+                   int k, uint4 *__restrict__ out) {
+    const int lane = threadIdx.x & 31;
+    const int warps = gridDim.x * (blockDim.x >> 5);
+    for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < P; r += warps) {
+        const int p = __ldg(perm + r);
+        const uint4 *src = hidden + static_cast<size_t>(p / k) * vecs_per_row;
+        uint4 *dst = out + static_cast<size_t>(r) * vecs_per_row;
+        for (int v = lane; v < vecs_per_row; v += 32) dst[v] = __ldg(src + v);
+    }
+}
+
+}  // namespace
+
+size_t permute_scratch_bytes(long long P, int E) {
+    if (P <= kChunk) return 0;
+    const long long nchunks = (P + kChunk - 1) / kChunk;
+    return static_cast<size_t>(nchunks) * E * sizeof(int32_t);
+}
+
+cudaError_t launch_permute(const int32_t *ids, int P, int E, int32_t *counts, int32_t *offsets, int32_t *perm,
+                           int32_t *inv_perm, void *scratch, int *err, cudaStream_t s) {
+    cudaError_t st;
+    if (P <= kChunk) {
+        const size_t sm = (static_cast<size_t>(kWarps) * E + 2 * E) * sizeof(int);
+        st = cudaFuncSetAttribute(permute_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  static_cast<int>(sm));
+        if (st != cudaSuccess) return st;
+        permute_single_kernel<<<1, kThreads, sm, s>>>(ids, P, E, counts, offsets, perm, inv_perm, err);
+        return cudaGetLastError();
+    }
+    const int nchunks = (P + kChunk - 1) / kChunk;
+    int32_t *chunk_hist = static_cast<int32_t *>(scratch);
+    const size_t sm_hist = static_cast<size_t>(kWarps) * E * sizeof(int);
+    const size_t sm_scatter = (static_cast<size_t>(kWarps) * E + E) * sizeof(int);
+    st = cudaFuncSetAttribute(permute_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(sm_hist));
+    if (st != cudaSuccess) return st;
+    st = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(sm_scatter));
+    if (st != cudaSuccess) return st;
+    permute_count_kernel<<<nchunks, kThreads, sm_hist, s>>>(ids, P, E, chunk_hist, err);
+    permute_scan_kernel<<<1, kThreads, 2 * E * sizeof(int), s>>>(nchunks, E, chunk_hist, counts, offsets);
+    permute_scatter_kernel<<<nchunks, kThreads, sm_scatter, s>>>(ids, P, E, chunk_hist, perm, inv_perm);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_gather(const uint16_t *hidden, const int32_t *perm, int P, int H, int k, uint16_t *hidden_perm,
+                          cudaStream_t s) {
+    if (P == 0) return cudaSuccess;
+    const int rows_per_block = 8;
+    int blocks = (P + rows_per_block - 1) / rows_per_block;
+    if (blocks > 148 * 16) blocks = 148 * 16;
+    gather_rows_kernel<<<blocks, 32 * rows_per_block, 0, s>>>(reinterpret_cast<const uint4 *>(hidden), perm, P,
+                                                              H / 8, k, reinterpret_cast<uint4 *>(hidden_perm));
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -8,8 +8,8 @@ patterns.
 
 Functions follow the layer's steps (InfiniLM PR #500 Qwen3-MoE report §2.2;
 FlashInfer PR #7196 analysis §1 for finalize, §2-§3 for W4A16):
-  route, permute, gather, dequant_int4, expert_ffn, finalize, forward,
-  forward_tokens.
+  route, permute, gather, dequant_int4, expert_ffn, expert_down, finalize,
+  forward, forward_tokens.
 """
 
 from __future__ import annotations
@@ -37,6 +37,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_gather.argtypes = [vp, vp, i32, i32, i32, vp]
         L.oracle_dequant_int4.argtypes = [vp, vp, i32, i32, vp]
         L.oracle_expert_ffn.argtypes = [i32, vp, vp, vp, vp, vp, i32, i32, vp, vp]
+        L.oracle_expert_gate_up.argtypes = [i32, vp, vp, vp, i32, i32, vp]
+        L.oracle_expert_down.argtypes = [i32, vp, vp, vp, i32, i32, vp]
         L.oracle_finalize.argtypes = [vp, vp, vp, i32, i32, i32, vp]
         L.oracle_forward.argtypes = [i32, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                      vp, vp, vp, vp, vp, vp, vp, vp, vp]
@@ -151,6 +153,18 @@ def expert_ffn(x, w_gu, w_d, H: int, I: int, fmt: str = "bf16", w_gu_scales=None
     y = np.zeros(H, np.uint16)
     lib().oracle_expert_ffn(f, _p(xa), _p(gu), _p(sg), _p(d), _p(sd), H, I, _p(act), _p(y))
     return act, y
+
+
+def expert_down(act, w_d, H: int, I: int, fmt: str = "bf16", w_d_scales=None):
+    """The down projection of one act row [I] by expert weights: y [H] bf16 bits."""
+    f = _fmt_code(fmt)
+    wdt = np.uint16 if f == 0 else np.uint8
+    aa = _np(act, np.uint16).reshape(-1)
+    d = _np(w_d, wdt)
+    sd = None if f == 0 else _np(w_d_scales, np.uint16)
+    y = np.zeros(H, np.uint16)
+    lib().oracle_expert_down(f, _p(aa), _p(d), _p(sd), H, I, _p(y))
+    return y
 
 
 def finalize(y, w, inv_perm, T: int, H: int, k: int) -> np.ndarray:

@@ -209,9 +209,8 @@ static float weight_at(int fmt, const void *w, const uint16_t *s, int K, int row
     return bf16_to_f32(dequant_one((const uint8_t *)w + (size_t)row * (K / 2), s + (size_t)row * (K / 128), col));
 }
 
-void oracle_expert_ffn(int fmt, const uint16_t *x, const void *w_gu, const uint16_t *w_gu_s,
-                       const void *w_d, const uint16_t *w_d_s, int H, int I,
-                       uint16_t *act, uint16_t *y) {
+void oracle_expert_gate_up(int fmt, const uint16_t *x, const void *w_gu, const uint16_t *w_gu_s, int H, int I,
+                           uint16_t *act) {
     no_ftz_daz();
     for (int i = 0; i < I; ++i) {
         double g = 0.0, u = 0.0;
@@ -224,12 +223,24 @@ void oracle_expert_ffn(int fmt, const uint16_t *x, const void *w_gu, const uint1
         double silu = (double)gf / (1.0 + exp(-(double)gf));
         act[i] = f32_to_bf16((float)(silu * (double)uf));
     }
+}
+
+void oracle_expert_down(int fmt, const uint16_t *act, const void *w_d, const uint16_t *w_d_s, int H, int I,
+                        uint16_t *y) {
+    no_ftz_daz();
     for (int h = 0; h < H; ++h) {
         double acc = 0.0;
         for (int i = 0; i < I; ++i)
             acc += (double)bf16_to_f32(act[i]) * (double)weight_at(fmt, w_d, w_d_s, I, h, i);
         y[h] = f32_to_bf16((float)acc);
     }
+}
+
+void oracle_expert_ffn(int fmt, const uint16_t *x, const void *w_gu, const uint16_t *w_gu_s,
+                       const void *w_d, const uint16_t *w_d_s, int H, int I,
+                       uint16_t *act, uint16_t *y) {
+    oracle_expert_gate_up(fmt, x, w_gu, w_gu_s, H, I, act);
+    oracle_expert_down(fmt, act, w_d, w_d_s, H, I, y);
 }
 
 /* ---- step 6: finalize / unpermute ------------------------------------------

@@ -1,0 +1,116 @@
+"""The C-ABI library without a GPU: it loads, exports every entry point that
+include/moe.h declares, and rejects bad arguments before touching CUDA."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixture_experts_expert_top_b200 as moe
+from mixture_experts_expert_top_b200 import build as moe_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    moe_build.build()
+
+
+def declared_entry_points():
+    names = []
+    for f in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            names += re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text)
+    return names
+
+
+def test_header_declares_the_layer_entry_points():
+    names = declared_entry_points()
+    for n in ("moe_route", "moe_permute", "moe_grouped_gemm_swiglu", "moe_grouped_gemm_down",
+              "moe_finalize", "moe_forward", "moe_workspace_size", "moe_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(moe.library_path)
+    for n in declared_entry_points():
+        assert hasattr(lib, n), n
+
+
+def test_binding_names_match_the_header():
+    for n in declared_entry_points():
+        assert callable(getattr(moe, n)), n
+
+
+def test_status_strings():
+    assert moe.moe_status_string(0) == "ok"
+    assert "workspace" in moe.moe_status_string(3)
+    assert moe.moe_status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("shape,ok", [
+    ((16, 128, 64, 8, 2, 0), True),
+    ((0, 128, 64, 8, 2, 0), True),
+    ((16, 128, 64, 8, 9, 0), False),       # k > E
+    ((16, 128, 64, 0, 1, 0), False),       # E = 0
+    ((16, 130, 64, 8, 2, 0), False),       # H not a multiple of 8
+    ((16, 128, 64, 2048, 2, 0), False),    # E > 1024
+    ((16, 128, 64, 64, 33, 0), False),     # k > 32
+    ((16, 192, 128, 8, 2, 1), False),      # int4 needs H % 128 == 0
+    ((16, 256, 128, 8, 2, 1), True),
+    ((-1, 128, 64, 8, 2, 0), False),
+    ((16, 128, 64, 8, 2, 7), False),       # unknown format
+])
+def test_workspace_size_validates_the_shape(shape, ok):
+    n = moe.moe_workspace_size(moe.Shape.of(*shape))
+    assert (n > 0) == ok or (shape[0] == 0 and n >= 0)
+
+
+def test_workspace_grows_with_tokens():
+    a = moe.moe_workspace_size(moe.Shape.of(64, 2048, 768, 128, 8))
+    b = moe.moe_workspace_size(moe.Shape.of(128, 2048, 768, 128, 8))
+    assert b > a > 64 * 8 * (2048 * 2 * 2 + 768 * 2)
+    assert moe.moe_forward_host_workspace_size(moe.Shape.of(64, 2048, 768, 128, 8)) > a
+    assert moe.moe_permute_workspace_size(moe.Shape.of(64, 2048, 768, 128, 8)) == 0
+    assert moe.moe_permute_workspace_size(moe.Shape.of(8192, 2048, 768, 128, 8)) == 8 * 128 * 4
+
+
+def test_bad_arguments_are_rejected_before_any_launch():
+    L = moe.lib()
+    sh = moe.Shape.of(16, 128, 64, 8, 2)
+    byref = ctypes.byref
+    # null pointers
+    assert L.moe_route(None, byref(sh), None, None, None) == 1
+    assert L.moe_finalize(None, None, None, byref(sh), None, None) == 1
+    assert L.moe_forward(None, None, None, None, None, None, byref(sh), None, None, 0, None) == 1
+    # a fused gather in the gate/up GEMM is not offered
+    assert L.moe_grouped_gemm_swiglu(16, 16, 16, 16, None, byref(sh), 16, None) == 2
+    # misaligned hidden
+    assert L.moe_forward(17, 16, 16, None, 16, None, byref(sh), 16, 256, 1 << 30, None) == 1
+    # scales given for bf16 weights
+    assert L.moe_grouped_gemm_down(16, 16, 16, 16, byref(sh), 16, None) == 1
+    # int4 without scales
+    sh4 = moe.Shape.of(16, 256, 128, 8, 2, moe.FMT_INT4_G128)
+    assert L.moe_grouped_gemm_down(16, 16, 16, None, byref(sh4), 16, None) == 1
+    # workspace too small
+    assert L.moe_forward(16, 16, 16, None, 16, None, byref(sh), 16, 256, 1024, None) == 3
+    # k > E
+    bad = moe.Shape.of(16, 128, 64, 8, 9)
+    assert L.moe_route(16, byref(bad), 16, 16, None) == 1
+    # permute: hidden without hidden_perm
+    assert L.moe_permute(16, byref(sh), 16, 16, 16, 16, 16, None, None, 0, None) == 1
+    # dequant: K not a multiple of 128
+    assert L.moe_dequant_int4(16, 16, 4, 100, 16, None) == 1
+
+
+def test_empty_batch_is_a_no_op():
+    L = moe.lib()
+    sh = moe.Shape.of(0, 128, 64, 8, 2)
+    byref = ctypes.byref
+    assert L.moe_route(None, byref(sh), None, None, None) == 0
+    assert L.moe_permute(None, byref(sh), None, None, None, None, None, None, None, 0, None) == 0
+    assert L.moe_forward(None, None, None, None, None, None, byref(sh), None, None, 0, None) == 0
+    assert L.moe_finalize(None, None, None, byref(sh), None, None) == 0

@@ -1,0 +1,231 @@
+"""Per-kernel parity of the CUDA path with the CPU oracle, through the C ABI.
+
+Bit-exact: routing ids, counts, offsets, perm, inv_perm, the gather, the
+W4A16 decode and finalize (fed the same y and weights). Within tolerance:
+routing weights (expf vs exp in double) and the GEMM outputs (fp32
+accumulation order; see _util.gemm_rows_close).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import moe_synth
+import oracle
+import mixture_experts_expert_top_b200 as moe
+from mixture_experts_expert_top_b200 import build as moe_build
+from _util import bf16_bits, bits_to_bf16, gemm_rows_close
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_device):
+    moe_build.build()
+    moe.lib()
+    yield
+    assert moe.moe_get_device_error() == 0
+
+
+def dev(x, dtype=None):
+    t = torch.as_tensor(x)
+    if dtype is not None:
+        t = t.to(dtype)
+    return t.contiguous().to(DEV)
+
+
+def run_route(logits, k):
+    T, E = logits.shape
+    ids = torch.empty(T, k, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k, dtype=torch.float32, device=DEV)
+    moe.moe_route(dev(logits), moe.Shape.of(T, 8, 8, E, k), ids, w)
+    torch.cuda.synchronize()
+    return ids.cpu().numpy(), w.cpu().numpy()
+
+
+def run_permute(ids, E, H=8, hidden=None):
+    T, k = ids.shape
+    P = T * k
+    sh = moe.Shape.of(T, H, 8, E, k)
+    counts = torch.empty(E, dtype=torch.int32, device=DEV)
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=DEV)
+    perm = torch.empty(P, dtype=torch.int32, device=DEV)
+    inv = torch.empty(P, dtype=torch.int32, device=DEV)
+    ws = torch.empty(max(1, moe.moe_permute_workspace_size(sh)), dtype=torch.uint8, device=DEV)
+    hp = None
+    if hidden is not None:
+        hp = torch.empty(P, H, dtype=torch.bfloat16, device=DEV)
+    moe.moe_permute(dev(ids, torch.int32), sh, counts, offsets, perm, inv,
+                    None if hidden is None else dev(hidden), hp, ws)
+    torch.cuda.synchronize()
+    out = [x.cpu().numpy() for x in (counts, offsets, perm, inv)]
+    return out + ([bf16_bits(hp)] if hidden is not None else [])
+
+
+# ---------------------------------------------------------------- routing --
+
+ROUTE_CASES = [(c.T, c.E, c.k, c.name) for c in moe_synth.CONFIGS.values()] + [
+    (100, 8, 8, "k=E"), (33, 64, 1, "k=1"), (5, 1, 1, "E=1"), (40, 1024, 32, "E=1024,k=32"), (3, 33, 4, "E=33"),
+]
+
+
+@pytest.mark.parametrize("T,E,k,name", ROUTE_CASES, ids=[c[3] for c in ROUTE_CASES])
+def test_route_matches_oracle(T, E, k, name):
+    cfg = moe_synth.CONFIGS.get(name)
+    logits = moe_synth.gen_logits(cfg) if cfg else torch.randn(T, E, generator=torch.Generator().manual_seed(T + E))
+    gi, gw = run_route(logits, k)
+    oi, ow = oracle.route(logits, k)
+    assert np.array_equal(gi, oi)
+    # The GPU forms x = l_j - l_0 in fp32 (rounding error up to |x| 2^-24,
+    # which exp turns into the same relative error), then expf (<= 2 ulp), an
+    # fp32 sum of k terms and one division; the oracle works in double.
+    # Bound: 2^-24 (8 + 2 max_j |l_j - l_0|) relative, per token.
+    lsel = np.take_along_axis(logits.numpy().astype(np.float64), oi.astype(np.int64), 1)
+    spread = np.abs(lsel - lsel[:, :1]).max(1, keepdims=True)
+    rel = np.abs(gw.astype(np.float64) - ow) / np.abs(ow)
+    bound = 2.0 ** -24 * (8 + 2 * spread)
+    assert np.all(rel <= bound), f"max relative error {rel.max():.3g}, worst ratio {(rel / bound).max():.3g}"
+    assert np.all(np.abs(gw.astype(np.float64).sum(1) - 1) <= 1e-6)
+
+
+def test_route_ties_go_to_the_lower_expert():
+    logits = torch.zeros(6, 16)
+    logits[1, 3] = logits[1, 9] = 1.0
+    logits[2] = torch.arange(16) % 4 * 0.5
+    logits[3, :] = -3.0
+    logits[4, 15] = 5.0
+    gi, gw = run_route(logits, 4)
+    oi, ow = oracle.route(logits, 4)
+    assert np.array_equal(gi, oi)
+    assert np.array_equal(gi[3], [0, 1, 2, 3]) and np.all(gw[3] == 0.25)
+
+
+# ---------------------------------------------------------------- permute --
+
+PERMUTE_CASES = [(16, 8, 2), (64, 128, 8), (256, 256, 8), (1024, 8, 8), (1025, 64, 8), (8192, 128, 8),
+                 (4096, 64, 6), (1, 4, 4), (3000, 1024, 3), (20000, 2, 1)]
+
+
+@pytest.mark.parametrize("T,E,k", PERMUTE_CASES)
+def test_permute_matches_oracle(T, E, k):
+    g = torch.Generator().manual_seed(T * 7 + E)
+    logits = torch.randn(T, E, generator=g)
+    if E >= 16:     # skew the load so that some experts stay empty
+        logits += torch.linspace(3, -3, E)[None, :]
+    ids, _ = oracle.route(logits, k)
+    counts, offsets, perm, inv = run_permute(ids, E)
+    oc, oo, op, oinv = oracle.permute(ids, E)
+    assert np.array_equal(counts, oc)
+    assert np.array_equal(offsets, oo)
+    assert np.array_equal(perm, op)
+    assert np.array_equal(inv, oinv)
+
+
+def test_permute_with_gather():
+    cfg = moe_synth.get_config("qwen3_decode")
+    hidden = moe_synth.gen_hidden(cfg)
+    ids, _ = oracle.route(moe_synth.gen_logits(cfg), cfg.k)
+    *_, perm, inv, hp = run_permute(ids, cfg.E, H=cfg.H, hidden=hidden)
+    assert np.array_equal(hp, oracle.gather(hidden, perm, cfg.k))
+
+
+def test_permute_flags_bad_expert_ids():
+    ids = np.array([[0, 1], [2, 7], [1, 9]], np.int32)     # 9 is out of range for E = 8
+    counts, offsets, perm, inv = run_permute(ids, 8)
+    assert moe.moe_get_device_error() == 1
+    assert counts.sum() == 5 and offsets[-1] == 5 and inv[5] == -1
+    assert moe.moe_get_device_error() == 0                  # reading clears it
+
+
+# -------------------------------------------------------------- finalize --
+
+def run_finalize(y_bits, w, inv, T, H, k):
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=DEV)
+    moe.moe_finalize(dev(bits_to_bf16(y_bits)), dev(w, torch.float32), dev(inv, torch.int32),
+                     moe.Shape.of(T, H, 8, max(k, 1), k), out)
+    torch.cuda.synchronize()
+    return bf16_bits(out)
+
+
+@pytest.mark.parametrize("T,H,k", [(16, 128, 2), (64, 2048, 8), (333, 72, 6), (7, 7168, 8), (1, 8, 1), (50, 64, 32)])
+def test_finalize_bit_exact(T, H, k):
+    rng = np.random.default_rng(T * H + k)
+    y = rng.standard_normal((T * k, H)).astype(np.float32)
+    y[rng.random(y.shape) < 0.05] = 0.0
+    y[rng.random(y.shape) < 0.02] *= 2.0 ** -130           # subnormal rows of values
+    y_bits = bf16_bits(torch.from_numpy(y).to(torch.bfloat16))
+    w = rng.random((T, k)).astype(np.float32)
+    w[rng.random(w.shape) < 0.05] = 0.0
+    inv = rng.permutation(T * k).astype(np.int32)
+    assert np.array_equal(run_finalize(y_bits, w, inv, T, H, k), oracle.finalize(y_bits, w, inv, T, H, k))
+
+
+def test_finalize_special_cases_from_the_golden_file():
+    import test_oracle_pins as pins
+    for k, v, w, exp, why in pins._golden_finalize_cases():
+        # replicate the one-element case across 8 lanes (one 16-byte vector)
+        y = np.repeat(np.array(v, np.uint16).reshape(k, 1), 8, axis=1)
+        wf = np.array(w, np.uint32).view(np.float32).reshape(1, k)
+        out = run_finalize(y, wf, np.arange(k, dtype=np.int32), 1, 8, k)
+        assert np.all(out == exp), why
+
+
+# ---------------------------------------------------------- W4A16 decode --
+
+@pytest.mark.parametrize("rows,K", [(4, 128), (300, 7168), (129, 2048)])
+def test_dequant_int4_bit_exact(rows, K):
+    g = torch.Generator().manual_seed(rows + K)
+    q = torch.randint(0, 256, (rows, K // 2), generator=g, dtype=torch.uint8)
+    s = (torch.rand(rows, K // 128, generator=g) * 0.018 + 0.002).to(torch.bfloat16)
+    s[0, 0] = 2.0 ** -130 if rows > 1 else s[0, 0]      # subnormal-range scale
+    out = torch.empty(rows, K, dtype=torch.bfloat16, device=DEV)
+    moe.moe_dequant_int4(dev(q), dev(s), rows, K, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(bf16_bits(out), oracle.dequant_int4(q, s))
+
+
+# ----------------------------------------------------------- grouped GEMMs --
+
+GEMM_CFGS = [
+    moe_synth.get_config("tiny"),
+    moe_synth.get_config("qwen3_decode"),
+    moe_synth.get_config("qwen3_decode", T=200, E=16),                 # many rows per expert: several N blocks
+    moe_synth.get_config("tiny", T=33, H=72, I=40, E=5, k=3),           # ragged H, I < 128
+    moe_synth.get_config("skewed", T=96, H=256, I=192, E=16, k=3),      # uneven, empty experts
+    moe_synth.get_config("qwen3_prefill", T=700, H=512, I=256, E=8, k=2),  # BN = 128 path, ragged tail
+]
+
+
+def gemm_case(cfg, seed=21):
+    inp = moe_synth.gen_inputs(cfg, seed=seed)
+    r = oracle.forward(inp, cfg.k, fmt=cfg.fmt)
+    hp = oracle.gather(inp["hidden"], r["perm"], cfg.k)
+    return inp, r, hp
+
+
+def wdev(inp, name):
+    return dev(inp[name]) if name in inp else None
+
+
+@pytest.mark.parametrize("cfg", GEMM_CFGS, ids=lambda c: f"T{c.T}H{c.H}I{c.I}E{c.E}k{c.k}")
+def test_grouped_gemm_swiglu_and_down_match_oracle(cfg):
+    inp, r, hp = gemm_case(cfg)
+    P = cfg.P
+    sh = moe.Shape.of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.fmt)
+    offsets = dev(r["offsets"], torch.int32)
+    act = torch.empty(P, cfg.I, dtype=torch.bfloat16, device=DEV)
+    moe.moe_grouped_gemm_swiglu(dev(bits_to_bf16(hp)), None, offsets, wdev(inp, "w_gu"), wdev(inp, "w_gu_scales"),
+                                sh, act)
+    # the down GEMM is fed the oracle's act so that each GEMM is checked alone
+    y = torch.empty(P, cfg.H, dtype=torch.bfloat16, device=DEV)
+    moe.moe_grouped_gemm_down(dev(bits_to_bf16(r["act"])), offsets, wdev(inp, "w_d"), wdev(inp, "w_d_scales"), sh, y)
+    torch.cuda.synchronize()
+    gemm_rows_close(bf16_bits(act), r["act"], "act")
+    gemm_rows_close(bf16_bits(y), r["y"], "y")
+
+
+def test_grouped_gemm_int4_matches_oracle():
+    cfg = moe_synth.MoeConfig("int4_mid", T=48, H=1024, I=384, E=12, k=4, fmt="int4_g128")
+    test_grouped_gemm_swiglu_and_down_match_oracle(cfg)

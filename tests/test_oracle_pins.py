@@ -385,3 +385,10 @@ def test_synthetic_distributions():
     assert hist.min() > 0.8 * hist.mean()
     s = q["w_gu_scales"].float()
     assert s.min() >= 0.0019 and s.max() <= 0.0201
+
+
+def test_expert_ffn_is_gate_up_then_down():
+    cfg = moe_synth.get_config("tiny")
+    inp = moe_synth.gen_inputs(cfg, seed=17)
+    act, y = oracle.expert_ffn(inp["hidden"][3], inp["w_gu"][2], inp["w_d"][2], cfg.H, cfg.I)
+    assert np.array_equal(oracle.expert_down(act, inp["w_d"][2], cfg.H, cfg.I), y)
