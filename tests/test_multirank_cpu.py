@@ -1,0 +1,97 @@
+"""The N > 1 host logic of bench.py on CPU with two gloo ranks: the
+max-over-ranks timing reduction, and the reference arm's rank gating
+(rank 0 alone runs and prints; other ranks exit 0 without work)."""
+
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    import bench
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        local_ms = [3.5, 7.25][rank]
+        q.put((rank, bench.max_over_ranks(local_ms)))
+        bench.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_with_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    got = dict(q.get(timeout=10) for _ in range(2))
+    assert got == {0: 7.25, 1: 7.25}
+
+
+def test_max_over_ranks_without_a_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(2.5) == 2.5
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    port = _free_port()
+    procs = []
+    for rank in range(2):
+        env = dict(os.environ, RANK=str(rank), WORLD_SIZE="2", LOCAL_RANK=str(rank),
+                   MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+        procs.append(subprocess.Popen(
+            [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+             "--workload", "tiny", "--steps", "3", "--warmup", "3", "--ref-budget-s", "2"],
+            env=env, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True))
+    outs = [p.communicate(timeout=300) for p in procs]
+    assert [p.returncode for p in procs] == [0, 0], [o[1][-2000:] for o in outs]
+    line = json.loads(outs[0][0].strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["n_gpus"] == 2
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0
+    assert outs[1][0].strip() == ""
+
+
+def test_bench_work_accounting():
+    sys.path.insert(0, ROOT)
+    import bench
+    import moe_synth
+    cfg = moe_synth.get_config("qwen3_decode")
+    counts = [4] * 120 + [0] * 8
+    w = bench.work_per_step(cfg, counts)
+    assert w["active_experts"] == 120
+    assert w["weight_bytes"] == 120 * 3 * 2048 * 768 * 2
+    assert w["layer_flops"] == 2 * 64 * 8 * 3 * 2048 * 768
+    assert bench.launches_per_step(cfg) == 6
+    assert bench.launches_per_step(moe_synth.get_config("qwen3_prefill")) == 8
+    q = moe_synth.get_config("w4a16_decode")
+    wq = bench.work_per_step(q, [8] * 256)
+    assert wq["weight_bytes"] == 256 * (2 * 2048 * (7168 // 2 + 56 * 2) + 7168 * (2048 // 2 + 16 * 2))
+
+
+def test_bench_rejects_too_few_warmup_steps():
+    sys.path.insert(0, ROOT)
+    import bench
+    with pytest.raises(SystemExit):
+        bench.parse_args(["--warmup", "2"])
