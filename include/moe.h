@@ -174,6 +174,32 @@ MOE_API moe_status_t moe_dequant_int4(const uint8_t *q, const moe_bf16_t *scales
  * timed out) and clears it. */
 MOE_API moe_status_t moe_get_device_error(int32_t *code);
 
+/* moe_permute for callers that cannot allocate device memory: the same
+ * outputs, bit for bit, with the scratch taken from a fixed 256 KiB array
+ * built into the library instead of a caller workspace. It is meant for code
+ * that runs inside a host framework which owns every device allocation and
+ * passes no workspace, and for hot loops that must not call cudaMalloc,
+ * because that call can synchronise the device. The pages have no
+ * counterpart to this entry point.
+ *   Arguments as moe_permute, without ws/ws_bytes. It allocates nothing and
+ *   calls no allocating routine.
+ *   Limit: the per-chunk histogram, ceil(T*top_k / 8192) * E int32 entries,
+ *   must fit 65536 entries. For example, E = 128 allows up to 4,194,304
+ *   pairs. Larger calls return MOE_ERR_UNSUPPORTED before anything is
+ *   enqueued. Calls with T*top_k <= 8192 use no scratch at all.
+ *   The array exists once per GPU that loads the library and is held until
+ *   the process exits. Its device address is looked up on the first call
+ *   made with a given device current, so make that first call before any
+ *   stream capture.
+ *   Every call on a device shares the one array. Calls whose work overlaps
+ *   on the GPU (different streams, no ordering between them) race on it, so
+ *   order such calls. Each call overwrites every entry it reads, so the
+ *   previous call's contents need no clearing. */
+MOE_API moe_status_t moe_permute_noalloc(const int32_t *topk_ids, const moe_shape_t *shape,
+                                         int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv_perm,
+                                         const moe_bf16_t *hidden, moe_bf16_t *hidden_perm,
+                                         moe_stream_t stream);
+
 /* Static description of a status code. */
 MOE_API const char *moe_status_string(moe_status_t status);
 

@@ -24,7 +24,7 @@ __all__ = [
     "moe_workspace_size", "moe_permute_workspace_size", "moe_forward_host_workspace_size",
     "moe_route", "moe_permute", "moe_grouped_gemm_swiglu", "moe_grouped_gemm_down",
     "moe_finalize", "moe_forward", "moe_forward_host", "moe_dequant_int4",
-    "moe_get_device_error", "moe_status_string", "forward",
+    "moe_get_device_error", "moe_status_string", "moe_permute_noalloc", "forward",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -78,6 +78,7 @@ def lib() -> ctypes.CDLL:
             "moe_forward": ([vp, vp, vp, vp, vp, vp, sp, vp, vp, sz, vp], ctypes.c_int),
             "moe_forward_host": ([vp, vp, vp, vp, vp, vp, sp, vp, vp, sz, vp], ctypes.c_int),
             "moe_dequant_int4": ([vp, vp, i32, i32, vp, vp], ctypes.c_int),
+            "moe_permute_noalloc": ([vp, sp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
             "moe_get_device_error": ([ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
             "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
         }
@@ -146,6 +147,15 @@ def moe_permute(topk_ids, shape, counts, offsets, perm, inv_perm, hidden=None, h
     _check(lib().moe_permute(_p(topk_ids), ctypes.byref(_shape(shape)), _p(counts), _p(offsets), _p(perm),
                              _p(inv_perm), _p(hidden), _p(hidden_perm), _p(ws), nbytes, _s(stream)),
            "moe_permute")
+
+
+def moe_permute_noalloc(topk_ids, shape, counts, offsets, perm, inv_perm, hidden=None, hidden_perm=None,
+                        stream=None) -> None:
+    """moe_permute without a workspace: its scratch is a fixed array inside the
+    library (for callers that cannot allocate device memory)."""
+    _check(lib().moe_permute_noalloc(_p(topk_ids), ctypes.byref(_shape(shape)), _p(counts), _p(offsets), _p(perm),
+                                     _p(inv_perm), _p(hidden), _p(hidden_perm), _s(stream)),
+           "moe_permute_noalloc")
 
 
 def moe_grouped_gemm_swiglu(a, perm, offsets, w_gu, w_gu_scales, shape, act, stream=None) -> None:

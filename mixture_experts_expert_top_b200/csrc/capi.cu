@@ -143,6 +143,11 @@ moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const
 
 }  // namespace
 
+namespace moe {
+moe_status_t validate_shape(const moe_shape_t *shape) { return check_shape(shape); }
+int *device_error_flag() { return error_flag_ptr(); }
+}  // namespace moe
+
 extern "C" {
 
 size_t moe_workspace_size(const moe_shape_t *shape) {

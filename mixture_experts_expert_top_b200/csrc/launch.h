@@ -8,7 +8,15 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include "moe.h"
+
 namespace moe {
+
+// ---- capi.cu
+// The shape rules every entry point applies (MOE_OK or the status to return).
+moe_status_t validate_shape(const moe_shape_t *shape);
+// Device address of the library's error flag word on the current device.
+int *device_error_flag();
 
 // ---- route.cu
 cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s);
