@@ -54,6 +54,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="qwen3_decode")
+    ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
+                    help="override a workload field (T, H, I, E, k), e.g. for a smaller profiling case")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -228,6 +230,20 @@ def launches_per_step(cfg) -> int:
 
 # ------------------------------------------------------------------ our arm --
 
+def workload(args):
+    import moe_synth
+    cfg = moe_synth.get_config(args.workload)
+    over = {}
+    for kv in args.set:
+        k, v = kv.split("=", 1)
+        if k not in ("T", "H", "I", "E", "k"):
+            raise SystemExit(f"--set: unknown field {k}")
+        over[k] = int(v)
+    if over:
+        cfg = cfg.with_(**over, name=cfg.name + "+" + ",".join(f"{k}={v}" for k, v in sorted(over.items())))
+    return cfg
+
+
 def run_ours(args, rank, world, local):
     import numpy as np
     import torch
@@ -244,7 +260,7 @@ def run_ours(args, rank, world, local):
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
     moe.lib()
-    cfg = moe_synth.get_config(args.workload)
+    cfg = workload(args)
     # weights are the same on every rank (replicas); each rank draws its own tokens
     inp = moe_synth.gen_inputs(cfg, seed=args.seed)
     if rank:
@@ -433,7 +449,7 @@ def run_reference(args, rank, world):
         return None
     import moe_synth
     import oracle
-    cfg = moe_synth.get_config(args.workload)
+    cfg = workload(args)
     inp = moe_synth.gen_inputs(cfg, seed=args.seed)
     # size each step so that warmup + steps fit the budget
     t0 = time.perf_counter()

@@ -65,12 +65,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // Waits for the phase with the given parity to complete. Returns false (and
 // raises kErrTimeout, and sets *abort so that the CTA's other roles stop too)
 // if it does not complete within kWaitLimitNs, or if *abort is already set.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int *err) {
+// After a few immediate polls the waiting warp sleeps between polls, doubling
+// the sleep up to max_sleep_ns, so that waiters leave issue slots to the warps
+// doing work (a long cap for waits that span whole tiles; 0 = never sleep, for
+// waits on the critical path).
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int *err,
+                                          uint32_t max_sleep_ns = 64) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
-    uint32_t n = 0;
+    uint32_t n = 0, sleep_ns = 8;
     while (!mbar_try_wait(bar, parity)) {
-        if ((++n & 255u) == 0u) {
+        if (++n > 4 && max_sleep_ns) {
+            __nanosleep(sleep_ns);
+            if (sleep_ns < max_sleep_ns) sleep_ns <<= 1;
+        }
+        if ((n & 63u) == 0u) {
             if (*abort) return false;
             if (globaltimer_ns() - t0 > kWaitLimitNs) {
                 raise_error(err, kErrTimeout);
@@ -151,6 +160,37 @@ __device__ __forceinline__ void umma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, u
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
+}
+
+// D[tmem] (+)= A[tmem] * B[smem]^T, bf16 inputs, fp32 accumulator, one CTA.
+// A (M = 128 rows x K = 16) sits in TMEM lanes 0-127, two bf16 per 32-bit
+// column: row m in lane m, K elements 2c and 2c+1 in column a_tmem + c.
+__device__ __forceinline__ void umma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 registers per thread -> 32 consecutive TMEM columns of this thread's
+// lane (thread i of the warp writes lane (lane base + i)).
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+        "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+        "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+        "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // Arrives once on `bar` when all previously issued tcgen05.mma of this thread

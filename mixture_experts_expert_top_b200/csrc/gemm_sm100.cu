@@ -7,12 +7,12 @@
 //   down:     y[r, h]  = bf16( act[r] . W_d[e, h] )
 // for every permuted row r of expert e (offsets[e] <= r < offsets[e+1]).
 //
-// Design (sm_100a; the FlashInfer PR #7196 analysis §2 describes the same
-// operand roles for its W4A16 kernel):
+// Design (sm_100a; the FlashInfer PR #7196 analysis §2 and the GC-MoE
+// abstract describe the same operand roles):
 //  - Weights are the MMA's A operand (M = 128 weight rows per tile), tokens
 //    are the B operand (N = tokens). The MMA's N is chosen per tile at run
 //    time as the routed-token count rounded up to 16, so a decode tile with 5
-//    tokens issues N = 16 instructions and reads only 16 token rows.
+//    tokens issues N = 16 instructions and loads only 16 token rows.
 //  - gate/up tiles hold 128 gate rows and the matching 128 up rows: two MMAs
 //    per K step into two TMEM accumulators, so each epilogue thread finds g
 //    and u of the same (feature, token) in the same TMEM lane.
@@ -22,10 +22,13 @@
 //    ring, warp 1 issues tcgen05.mma (one thread) and owns the TMEM
 //    allocation, warps 2-5 drain the double-buffered TMEM accumulators
 //    (tcgen05.ld), apply SwiGLU and store bf16 rows.
-//  - W4A16 (INT4 = true): the TMA brings packed int4 weight tiles; warps 2-5
-//    first turn each stage into a swizzled bf16 tile in shared memory
-//    (w = bf16(q * scale)), then the MMA reads it like a bf16 tile; the same
-//    warps run the epilogue once a tile's K loop is converted.
+//  - W4A16 has a kernel of its own (grouped_gemm_int4_kernel): one ring stage
+//    covers K = 256, so each packed weight row arrives as one 128-byte TMA
+//    row; four groups of decode warps each turn one 64-K quarter of the stage
+//    into bf16 (w = bf16(q * scale)) and store it straight into a TMEM ring,
+//    from which the MMA reads its A operand. Shared memory carries 0.5 byte
+//    per weight instead of the 4.5 bytes a decode through shared memory would
+//    move (packed in, bf16 out, bf16 read again by the MMA).
 //  - Every wait is bounded (see mbar_wait); a timeout raises the device flag
 //    and unwinds the CTA.
 #include <cudaTypedefs.h>
@@ -40,32 +43,19 @@ namespace moe {
 namespace {
 
 constexpr int kBM = 128;          // weight rows per tile (MMA M)
-constexpr int kBK = 64;           // K elements per stage (one 128-byte swizzle row)
+constexpr int kBK = 64;           // K elements per bf16 stage / per int4 quarter (one 128-byte bf16 row)
 constexpr int kBoxN = 16;         // token rows per TMA box
-constexpr int kThreads = 192;     // 6 warps
-constexpr int kTileBytesA = kBM * kBK * 2;          // 16 KB bf16 tile
-constexpr int kPackedBytesA = kBM * kBK / 2;        // 4 KB int4 tile
+constexpr int kTileBytesA = kBM * kBK * 2;          // 16 KB bf16 tile (128 x 64)
+constexpr int kBoxBytesB = kBoxN * kBK * 2;         // 2 KB token box (16 x 64)
 constexpr int kMaxExperts = 1024;
+constexpr int kSmemLimit = 232448;                  // 227 KB per CTA
+constexpr int kEpiThreads = 128;                    // warps 2-5
 
-template <int BN, int STAGES, bool SWIGLU, bool INT4>
-struct Cfg {
-    static constexpr int kNumA = SWIGLU ? 2 : 1;
-    static constexpr int kBBytes = BN * kBK * 2;
-    static constexpr int kStageBytes = kNumA * kTileBytesA + kBBytes;
-    static constexpr int kPackedStage = INT4 ? kNumA * kPackedBytesA : 0;
-    static constexpr int kAccCols = SWIGLU ? 2 * BN : BN;
-    static constexpr int kTmemCols = (2 * kAccCols <= 32) ? 32 : (2 * kAccCols <= 64) ? 64
-                                   : (2 * kAccCols <= 128) ? 128 : (2 * kAccCols <= 256) ? 256 : 512;
-    // ring, then packed ring (int4), then barriers and bookkeeping
-    static constexpr int kRingBytes = STAGES * kStageBytes;
-    static constexpr int kPackedRingBytes = STAGES * kPackedStage;
-    static constexpr int kBarBytes = 8 * (4 * STAGES + 4 + 1);
-    static constexpr int kMiscBytes = 64 + 2 * (kMaxExperts + 1) * 4;
-    static constexpr int kSmemBytes = 1024 /*align slack*/ + kRingBytes + kPackedRingBytes + kBarBytes + kMiscBytes;
-    static_assert(kStageBytes % 1024 == 0, "stage must keep 1024-byte alignment");
-    static_assert(2 * kAccCols <= 512, "TMEM holds 512 fp32 columns");
-    static_assert(BN % kBoxN == 0 && BN <= 256, "BN");
-};
+// int4 kernel
+constexpr int kQuarters = 4;                        // 64-K quarters per int4 stage (K = 256)
+constexpr int kPackedTile = kBM * 128;              // 16 KB: 128 rows x 128 packed bytes
+constexpr int kConvGroups = kQuarters;              // decode group g handles quarter g of every stage
+constexpr int kMaxTmemA = 8;
 
 struct Params {
     const int32_t *offsets;
@@ -76,7 +66,7 @@ struct Params {
     int evict_first_weights;
 };
 
-// Tile bookkeeping shared by the three roles.
+// Tile bookkeeping shared by the roles.
 struct TileInfo {
     int e, mb, row0, valid, n_mma;
 };
@@ -99,45 +89,152 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int *pre, const 
     return t;
 }
 
-// W4A16 decoding of one 16-byte packed chunk (32 int4 values of one row) into
-// four 16-byte bf16 chunks: w = bf16_rne(q * scale). The fp32 product is exact
-// (q has at most 4 significant bits, the bf16 scale 8), so converting it with
-// round-to-nearest-even is the only rounding.
-__device__ __forceinline__ void dequant32(const uint4 &packed, float scale, uint4 (&o)[4]) {
-    const uint32_t words[4] = {packed.x, packed.y, packed.z, packed.w};
-#pragma unroll
-    for (int wi = 0; wi < 4; ++wi) {
-        const uint32_t x = words[wi];
-        uint32_t r[4];
-#pragma unroll
-        for (int b = 0; b < 4; ++b) {
-            const uint32_t byte = (x >> (8 * b)) & 0xFFu;
-            const int lo = static_cast<int>((byte & 0xFu) ^ 8u) - 8;     // sign-extended low nibble
-            const int hi = static_cast<int>((byte >> 4) ^ 8u) - 8;
-            const __nv_bfloat162 v = __floats2bfloat162_rn(static_cast<float>(lo) * scale,
-                                                           static_cast<float>(hi) * scale);
-            r[b] = *reinterpret_cast<const uint32_t *>(&v);
+// Copies offsets into shared memory and builds pre[e] = number of tiles of
+// experts 0..e-1 (a block-wide scan). All threads of the CTA call it.
+template <int NT>
+__device__ __forceinline__ void build_tile_prefix(const int32_t *offsets, int E, int MB, int BN, int *off_s,
+                                                  int *pre_s) {
+    __shared__ int wsum[NT / 32];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int i = threadIdx.x; i <= E; i += NT) off_s[i] = __ldg(offsets + i);
+    __syncthreads();
+    const int seg = (E + NT - 1) / NT;
+    const int b0 = threadIdx.x * seg;
+    int local = 0;
+    for (int i = 0; i < seg; ++i) {
+        const int e = b0 + i;
+        if (e < E) {
+            const int cnt = off_s[e + 1] - off_s[e];
+            local += ((cnt + BN - 1) / BN) * MB;
+            pre_s[e + 1] = local;        // segment-local inclusive
         }
-        o[wi] = make_uint4(r[0], r[1], r[2], r[3]);
+    }
+    int x = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    int before = x - local;
+    for (int w = 0; w < warp; ++w) before += wsum[w];
+    for (int i = 0; i < seg; ++i) {
+        const int e = b0 + i;
+        if (e < E) pre_s[e + 1] += before;
+    }
+    if (threadIdx.x == 0) pre_s[0] = 0;
+}
+
+// Epilogue of warps 2-5: per tile, wait for the accumulator buffer, read it
+// with tcgen05.ld (warp w reads TMEM lanes 32*(w%4)...), apply SwiGLU for
+// gate/up, round to bf16 and store; then hand the buffer back.
+template <int BN, bool SWIGLU, int ACC_COLS>
+__device__ __forceinline__ void run_epilogue(const Params &p, const int *pre_s, const int *off_s, int total_tiles,
+                                             int MB, uint32_t tmem_base, uint64_t *tfull_bar, uint64_t *tempty_bar,
+                                             volatile int *abort_flag) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q = warp & 3;
+    int buf = 0;
+    uint32_t bphase = 0;
+    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+        const TileInfo ti = decode_tile(tile, pre_s, off_s, p.E, MB, BN);
+        if (!mbar_wait(&tfull_bar[buf], bphase, abort_flag, p.err, 512)) break;
+        tc_fence_after_sync();
+        const int f = ti.mb * kBM + q * 32 + lane;         // output feature of this thread
+        const bool f_ok = f < p.m_out;
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * ACC_COLS;
+        for (int c0 = 0; c0 < ti.n_mma; c0 += 16) {
+            uint32_t g[16], u[16];
+            tmem_ld_32x32b_x16(tb + c0, g);
+            if (SWIGLU) tmem_ld_32x32b_x16(tb + BN + c0, u);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                const int n = c0 + j;
+                if (f_ok && n < ti.valid) {
+                    float v = __uint_as_float(g[j]);
+                    if (SWIGLU) {
+                        const float uu = __uint_as_float(u[j]);
+                        v = v / (1.0f + expf(-v)) * uu;
+                    }
+                    const __nv_bfloat16 bv = __float2bfloat16_rn(v);
+                    p.out[static_cast<size_t>(ti.row0 + n) * p.m_out + f] = __bfloat16_as_ushort(bv);
+                }
+            }
+        }
+        tc_fence_before_sync();
+        mbar_arrive(&tempty_bar[buf]);
+        if (++buf == 2) { buf = 0; bphase ^= 1; }
     }
 }
 
-template <int BN, int STAGES, bool SWIGLU, bool INT4>
-__global__ void __launch_bounds__(kThreads, 1)
+// W4A16 decoding of one 32-bit word of packed int4 (K elements 8i..8i+7 of a
+// row; byte b holds element 2b in its low nibble, 2b+1 in its high nibble,
+// two's complement) into four bf16x2 words (elements 2j, 2j+1 in word j):
+//   w = bf16_rne(q * scale)
+// Each nibble pair is placed in the mantissas of a bf16x2 with exponent 2^7
+// and biased to n = q + 8 (the bias is the flip of the nibble's sign bit,
+// folded into the same three-input logic op), giving bf16 (128 + n) exactly;
+// subtracting 136 gives q exactly, and one bf16 multiply by the scale rounds
+// the exact product once, to nearest even.
+__device__ __forceinline__ void dequant_word(uint32_t packed, __nv_bfloat162 scale2, uint32_t *out4) {
+    const uint32_t hi = packed >> 4;                       // odd elements move to the low nibble of each byte
+    const __nv_bfloat162 bias = __floats2bfloat162_rn(136.0f, 136.0f);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        // byte 0 <- element 2j (low nibble of byte j), byte 2 <- element 2j+1
+        const uint32_t r = __byte_perm(packed, hi, static_cast<uint32_t>(j | ((4 + j) << 8)));
+        // bits of 0x000F000F: r ^ 0x00080008 (n = q + 8); other bits: 0x43004300
+        const uint32_t v = (r & 0x000F000Fu) ^ 0x43084308u;
+        const __nv_bfloat162 q = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&v), bias);
+        const __nv_bfloat162 w = __hmul2(q, scale2);
+        out4[j] = *reinterpret_cast<const uint32_t *>(&w);
+    }
+}
+
+__device__ __forceinline__ __nv_bfloat162 bf16_pair(uint16_t bits) {
+    const __nv_bfloat16 b = __ushort_as_bfloat16(bits);
+    return __halves2bfloat162(b, b);
+}
+
+// =============================================================================
+// bf16 weights
+// =============================================================================
+
+template <int BN, int STAGES, bool SWIGLU>
+struct Bf16Cfg {
+    static constexpr int kNumA = SWIGLU ? 2 : 1;
+    static constexpr int kThreads = 192;
+    static constexpr int kABytes = kNumA * kTileBytesA;
+    static constexpr int kStageBytes = kABytes + BN * kBK * 2;
+    static constexpr int kAccCols = SWIGLU ? 2 * BN : BN;
+    static constexpr int kTmemUsed = 2 * kAccCols;
+    static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
+                                   : kTmemUsed <= 256 ? 256 : 512;
+    static constexpr int kRingBytes = STAGES * kStageBytes;
+    static constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1;
+    static constexpr int kSmemBytes = 1024 + kRingBytes + 8 * kNumBars + 64 + 2 * (kMaxExperts + 1) * 4;
+    static_assert(kStageBytes % 1024 == 0, "tiles must keep 1024-byte alignment");
+    static_assert(kTmemUsed <= 512, "TMEM holds 512 32-bit columns");
+    static_assert(BN % kBoxN == 0 && BN <= 256, "BN");
+    static_assert(kSmemBytes + 64 <= kSmemLimit, "shared memory");
+};
+
+template <int BN, int STAGES, bool SWIGLU>
+__global__ void __launch_bounds__(192, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const Params p) {
-    using C = Cfg<BN, STAGES, SWIGLU, INT4>;
+    using C = Bf16Cfg<BN, STAGES, SWIGLU>;
     extern __shared__ uint8_t smem_raw[];
     // operand tiles need 1024-byte alignment in the shared window (swizzle atoms)
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *ring = smem;                                    // STAGES x [A0 | A1 | B]
-    uint8_t *pring = smem + C::kRingBytes;                   // int4: STAGES x [Aq0 | Aq1]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(pring + C::kPackedRingBytes);
-    uint64_t *full_bar = bars;                 // TMA -> (converter | MMA)
-    uint64_t *empty_bar = bars + STAGES;       // MMA -> TMA
-    uint64_t *conv_bar = bars + 2 * STAGES;    // converter -> MMA (int4)
-    uint64_t *tfull_bar = bars + 3 * STAGES;   // MMA -> epilogue, 2 buffers
-    uint64_t *tempty_bar = tfull_bar + 2;      // epilogue -> MMA, 2 buffers
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + C::kRingBytes);
+    uint64_t *full_bar = bars;                               // TMA -> MMA
+    uint64_t *empty_bar = full_bar + STAGES;                 // MMA -> TMA
+    uint64_t *tfull_bar = empty_bar + STAGES;                // MMA -> epilogue, 2 buffers
+    uint64_t *tempty_bar = tfull_bar + 2;                    // epilogue -> MMA, 2 buffers
     uint64_t *drain_bar = tempty_bar + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
@@ -150,16 +247,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const int MB = (p.m_out + kBM - 1) / kBM;
     const int KB = (p.K + kBK - 1) / kBK;
 
-    // ---- prologue: barriers, TMEM, tile prefix --------------------------------
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full_bar[s], 1);
             mbar_init(&empty_bar[s], 1);
-            mbar_init(&conv_bar[s], 128);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull_bar[b], 1);
-            mbar_init(&tempty_bar[b], 128);
+            mbar_init(&tempty_bar[b], kEpiThreads);
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -173,39 +268,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         tmem_alloc(tmem_holder, C::kTmemCols);
         tmem_relinquish();
     }
-    for (int i = threadIdx.x; i <= E; i += kThreads) off_s[i] = __ldg(p.offsets + i);
-    __syncthreads();
-    // tiles per expert, then an inclusive scan by segments of ceil((E)/192)
-    {
-        const int seg = (E + kThreads - 1) / kThreads;
-        const int b0 = threadIdx.x * seg;
-        int local = 0;
-        for (int i = 0; i < seg; ++i) {
-            const int e = b0 + i;
-            if (e < E) {
-                const int cnt = off_s[e + 1] - off_s[e];
-                local += ((cnt + BN - 1) / BN) * MB;
-                pre_s[e + 1] = local;        // segment-local inclusive
-            }
-        }
-        // exclusive scan of segment totals over the 192 threads
-        __shared__ int wsum[kThreads / 32];
-        int x = local;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-        }
-        if (lane == 31) wsum[warp] = x;
-        __syncthreads();
-        int before = x - local;
-        for (int w = 0; w < warp; ++w) before += wsum[w];
-        for (int i = 0; i < seg; ++i) {
-            const int e = b0 + i;
-            if (e < E) pre_s[e + 1] += before;
-        }
-        if (threadIdx.x == 0) pre_s[0] = 0;
-    }
+    build_tile_prefix<C::kThreads>(p.offsets, E, MB, BN, off_s, pre_s);
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
@@ -219,36 +282,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const uint64_t pol_x = l2_policy_evict_last();
             int stage = 0;
             uint32_t phase = 0;
-            for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
                 const TileInfo ti = decode_tile(tile, pre_s, off_s, E, MB, BN);
                 const int nbox = ti.n_mma / kBoxN;
                 const int a_row = ti.e * p.w_rows + ti.mb * kBM;
-                const uint32_t a_bytes = INT4 ? C::kNumA * kPackedBytesA : C::kNumA * kTileBytesA;
-                const uint32_t tx = a_bytes + nbox * kBoxN * kBK * 2;
-                bool ok = true;
-                for (int kb = 0; kb < KB && ok; ++kb) {
-                    ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.err);
+                const uint32_t tx = C::kABytes + nbox * kBoxBytesB;
+                for (int kb = 0; kb < KB; ++kb) {
+                    ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.err, 256);
                     if (!ok) break;
                     mbar_arrive_expect_tx(&full_bar[stage], tx);
                     uint8_t *st = ring + stage * C::kStageBytes;
-                    if (INT4) {
-                        uint8_t *pq = pring + stage * C::kPackedStage;
-                        tma_load_2d(pq, &tmA, &full_bar[stage], kb * (kBK / 2), a_row, pol_w);
-                        if (SWIGLU)
-                            tma_load_2d(pq + kPackedBytesA, &tmA, &full_bar[stage], kb * (kBK / 2), a_row + p.m_out,
-                                        pol_w);
-                    } else {
-                        tma_load_2d(st, &tmA, &full_bar[stage], kb * kBK, a_row, pol_w);
-                        if (SWIGLU)
-                            tma_load_2d(st + kTileBytesA, &tmA, &full_bar[stage], kb * kBK, a_row + p.m_out, pol_w);
-                    }
-                    uint8_t *sb = st + C::kNumA * kTileBytesA;
+                    tma_load_2d(st, &tmA, &full_bar[stage], kb * kBK, a_row, pol_w);
+                    if (SWIGLU) tma_load_2d(st + kTileBytesA, &tmA, &full_bar[stage], kb * kBK, a_row + p.m_out, pol_w);
+                    uint8_t *sb = st + C::kABytes;
                     for (int b = 0; b < nbox; ++b)
-                        tma_load_2d(sb + b * kBoxN * kBK * 2, &tmB, &full_bar[stage], kb * kBK, ti.row0 + b * kBoxN,
-                                    pol_x);
+                        tma_load_2d(sb + b * kBoxBytesB, &tmB, &full_bar[stage], kb * kBK, ti.row0 + b * kBoxN, pol_x);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
                 }
-                if (!ok) break;
             }
         }
     } else if (warp == 1) {
@@ -267,13 +318,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 tc_fence_after_sync();
                 const uint32_t d0 = tmem_base + buf * C::kAccCols;
                 for (int kb = 0; kb < KB; ++kb) {
-                    ok = mbar_wait(INT4 ? &conv_bar[stage] : &full_bar[stage], phase, abort_flag, p.err);
+                    ok = mbar_wait(&full_bar[stage], phase, abort_flag, p.err, 0);
                     if (!ok) break;
                     tc_fence_after_sync();
                     const uint32_t st = smem_u32(ring + stage * C::kStageBytes);
                     const uint64_t da0 = sw128_kmajor_desc(st);
                     const uint64_t da1 = sw128_kmajor_desc(st + kTileBytesA);
-                    const uint64_t db = sw128_kmajor_desc(st + C::kNumA * kTileBytesA);
+                    const uint64_t db = sw128_kmajor_desc(st + C::kABytes);
 #pragma unroll
                     for (int k = 0; k < kBK / 16; ++k) {
                         const uint32_t acc = (kb | k) != 0;
@@ -294,85 +345,275 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             mbar_wait(drain_bar, 0, &never, p.err);
         }
     } else {
-        // ============ warps 2-5: int4 converters, then the epilogue =============
-        const int q = warp & 3;                 // TMEM lane quarter of this warp
-        const int et = threadIdx.x - 64;        // 0..127
-        int stage = 0;
-        uint32_t phase = 0;
-        int buf = 0;
-        uint32_t bphase = 0;
-        bool ok = true;
-        for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-            const TileInfo ti = decode_tile(tile, pre_s, off_s, E, MB, BN);
-            if (INT4) {
-                const int a_row = ti.e * p.w_rows + ti.mb * kBM + et;
-                const int srows = p.E * p.w_rows;
-                const int kgroups = p.K / 128;
-                for (int kb = 0; kb < KB; ++kb) {
-                    ok = mbar_wait(&full_bar[stage], phase, abort_flag, p.err);
-                    if (!ok) break;
-                    const uint8_t *pq = pring + stage * C::kPackedStage;
-                    uint8_t *st = ring + stage * C::kStageBytes;
-#pragma unroll
-                    for (int a = 0; a < C::kNumA; ++a) {
-                        const int row = a_row + a * p.m_out;
-                        const float scale =
-                            row < srows ? bf16_bits_to_float(__ldg(p.w_scales + static_cast<size_t>(row) * kgroups +
-                                                                    (kb * kBK) / 128))
-                                        : 0.f;
-                        const uint4 *src = reinterpret_cast<const uint4 *>(pq + a * kPackedBytesA + et * (kBK / 2));
-                        uint8_t *dst_row = st + a * kTileBytesA + et * 128;
-#pragma unroll
-                        for (int half = 0; half < 2; ++half) {
-                            uint4 o[4];
-                            dequant32(src[half], scale, o);
-#pragma unroll
-                            for (int c = 0; c < 4; ++c) {
-                                const int chunk = half * 4 + c;
-                                *reinterpret_cast<uint4 *>(dst_row + ((chunk ^ (et & 7)) << 4)) = o[c];
-                            }
-                        }
-                    }
-                    fence_proxy_async_smem();
-                    mbar_arrive(&conv_bar[stage]);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                }
-                if (!ok) break;
-            }
-            ok = mbar_wait(&tfull_bar[buf], bphase, abort_flag, p.err);
-            if (!ok) break;
-            tc_fence_after_sync();
-            const int f = ti.mb * kBM + q * 32 + lane;         // output feature of this thread
-            const bool f_ok = f < p.m_out;
-            const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * C::kAccCols;
-            for (int c0 = 0; c0 < ti.n_mma; c0 += 16) {
-                uint32_t g[16], u[16];
-                tmem_ld_32x32b_x16(tb + c0, g);
-                if (SWIGLU) tmem_ld_32x32b_x16(tb + BN + c0, u);
-                tmem_wait_ld();
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int n = c0 + j;
-                    if (f_ok && n < ti.valid) {
-                        float v = __uint_as_float(g[j]);
-                        if (SWIGLU) {
-                            const float uu = __uint_as_float(u[j]);
-                            v = v / (1.0f + expf(-v)) * uu;
-                        }
-                        const __nv_bfloat16 bv = __float2bfloat16_rn(v);
-                        p.out[static_cast<size_t>(ti.row0 + n) * p.m_out + f] = __bfloat16_as_ushort(bv);
-                    }
-                }
-            }
-            tc_fence_before_sync();
-            mbar_arrive(&tempty_bar[buf]);
-            if (++buf == 2) { buf = 0; bphase ^= 1; }
-        }
+        run_epilogue<BN, SWIGLU, C::kAccCols>(p, pre_s, off_s, total_tiles, MB, tmem_base, tfull_bar, tempty_bar,
+                                              abort_flag);
     }
 
     __syncthreads();
     if (*abort_flag) {
         // let copies already in flight land before the CTA's memory is reused
+        for (int i = 0; i < 1000; ++i) __nanosleep(1000);
+    }
+    if (warp == 1) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// =============================================================================
+// W4A16: int4 weights (one bf16 scale per 128 K), bf16 tokens
+// =============================================================================
+
+template <int BN, int STAGES, bool SWIGLU>
+struct Int4Cfg {
+    static constexpr int kNumA = SWIGLU ? 2 : 1;
+    static constexpr int kThreads = 192 + 128 * kConvGroups;
+    static constexpr int kABytes = kNumA * kPackedTile;                 // packed A per stage (K = 256)
+    static constexpr int kBQuarter = BN * kBK * 2;                      // token rows for one 64-K quarter
+    static constexpr int kStageBytes = kABytes + kQuarters * kBQuarter;
+    static constexpr int kAccCols = SWIGLU ? 2 * BN : BN;
+    static constexpr int kACols = kNumA * (kBK / 2);                    // TMEM columns per decoded quarter
+    static constexpr int kTmemAStages = (512 - 2 * kAccCols) / kACols < kMaxTmemA ? (512 - 2 * kAccCols) / kACols
+                                                                                 : kMaxTmemA;
+    static constexpr int kTmemUsed = 2 * kAccCols + kTmemAStages * kACols;
+    static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
+                                   : kTmemUsed <= 256 ? 256 : 512;
+    static constexpr int kRingBytes = STAGES * kStageBytes;
+    static constexpr int kNumBars = 2 * STAGES + 2 * kMaxTmemA + 2 + 2 + 1;
+    static constexpr int kSmemBytes = 1024 + kRingBytes + 8 * kNumBars + 64 + 2 * (kMaxExperts + 1) * 4;
+    static_assert(kStageBytes % 1024 == 0 && kBQuarter % 1024 == 0, "tiles must keep 1024-byte alignment");
+    static_assert(kTmemUsed <= 512, "TMEM holds 512 32-bit columns");
+    static_assert(kTmemAStages >= kConvGroups, "every decode group needs a TMEM slot in flight");
+    static_assert(BN % kBoxN == 0 && BN <= 256, "BN");
+    static_assert(kSmemBytes + 64 <= kSmemLimit, "shared memory");
+};
+
+template <int BN, int STAGES, bool SWIGLU>
+__global__ void __launch_bounds__(Int4Cfg<BN, STAGES, SWIGLU>::kThreads, 1)
+grouped_gemm_int4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                         const Params p) {
+    using C = Int4Cfg<BN, STAGES, SWIGLU>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+    uint8_t *ring = smem;                                    // STAGES x [Aq0 | Aq1 | B quarter 0..3]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + C::kRingBytes);
+    uint64_t *full_bar = bars;                               // TMA -> decode groups
+    uint64_t *empty_bar = full_bar + STAGES;                 // MMA -> TMA
+    uint64_t *tready_bar = empty_bar + STAGES;               // decode group -> MMA (TMEM ring slot)
+    uint64_t *tfree_bar = tready_bar + kMaxTmemA;            // MMA -> decode groups
+    uint64_t *tfull_bar = tfree_bar + kMaxTmemA;             // MMA -> epilogue, 2 buffers
+    uint64_t *tempty_bar = tfull_bar + 2;                    // epilogue -> MMA, 2 buffers
+    uint64_t *drain_bar = tempty_bar + 2;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain_bar + 1);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
+    int *off_s = reinterpret_cast<int *>(tmem_holder + 16);  // [E+1]
+    int *pre_s = off_s + (kMaxExperts + 1);                  // [E+1] tile prefix
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int E = p.E;
+    const int MB = (p.m_out + kBM - 1) / kBM;
+    const int KS = (p.K + 4 * kBK - 1) / (4 * kBK);          // stages of K = 256 per tile
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full_bar[s], 1);
+            mbar_init(&empty_bar[s], 1);
+        }
+        for (int t = 0; t < C::kTmemAStages; ++t) {
+            mbar_init(&tready_bar[t], 128);   // the 4 warps of one decode group
+            mbar_init(&tfree_bar[t], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&tfull_bar[b], 1);
+            mbar_init(&tempty_bar[b], kEpiThreads);
+        }
+        mbar_init(drain_bar, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, C::kTmemCols);
+        tmem_relinquish();
+    }
+    build_tile_prefix<C::kThreads>(p.offsets, E, MB, BN, off_s, pre_s);
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem_base = *tmem_holder;
+    const uint32_t tmem_a0 = tmem_base + 2 * C::kAccCols;   // first decoded-A column
+    const int total_tiles = pre_s[E];
+
+    if (warp == 0) {
+        // ================================ TMA producer ==========================
+        if (lane == 0) {
+            const uint64_t pol_w = p.evict_first_weights ? l2_policy_evict_first() : l2_policy_evict_last();
+            const uint64_t pol_x = l2_policy_evict_last();
+            int stage = 0;
+            uint32_t phase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+                const TileInfo ti = decode_tile(tile, pre_s, off_s, E, MB, BN);
+                const int nbox = ti.n_mma / kBoxN;
+                const int a_row = ti.e * p.w_rows + ti.mb * kBM;
+                const uint32_t tx = C::kABytes + kQuarters * nbox * kBoxBytesB;
+                for (int ks = 0; ks < KS; ++ks) {
+                    ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.err, 256);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(&full_bar[stage], tx);
+                    uint8_t *st = ring + stage * C::kStageBytes;
+                    tma_load_2d(st, &tmA, &full_bar[stage], ks * 128, a_row, pol_w);
+                    if (SWIGLU) tma_load_2d(st + kPackedTile, &tmA, &full_bar[stage], ks * 128, a_row + p.m_out, pol_w);
+                    uint8_t *sb = st + C::kABytes;
+                    for (int j = 0; j < kQuarters; ++j)
+                        for (int b = 0; b < nbox; ++b)
+                            tma_load_2d(sb + j * C::kBQuarter + b * kBoxBytesB, &tmB, &full_bar[stage],
+                                        (ks * kQuarters + j) * kBK, ti.row0 + b * kBoxN, pol_x);
+                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ================================ MMA issuer ============================
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase_unused = 0;
+            (void)phase_unused;
+            int t = 0;                  // TMEM ring slot of the next quarter
+            uint32_t tphase = 0;
+            int buf = 0;
+            uint32_t bphase = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+                const TileInfo ti = decode_tile(tile, pre_s, off_s, E, MB, BN);
+                const uint32_t idesc = idesc_bf16_f32(kBM, ti.n_mma);
+                ok = mbar_wait(&tempty_bar[buf], bphase ^ 1, abort_flag, p.err);
+                if (!ok) break;
+                tc_fence_after_sync();
+                const uint32_t d0 = tmem_base + buf * C::kAccCols;
+                for (int ks = 0; ks < KS && ok; ++ks) {
+                    const uint32_t sb = smem_u32(ring + stage * C::kStageBytes + C::kABytes);
+                    for (int j = 0; j < kQuarters; ++j) {
+                        // tready implies the stage's TMA data landed (the decode group waited for it)
+                        ok = mbar_wait(&tready_bar[t], tphase, abort_flag, p.err, 0);
+                        if (!ok) break;
+                        tc_fence_after_sync();
+                        const uint32_t a0 = tmem_a0 + t * C::kACols;
+                        const uint64_t db = sw128_kmajor_desc(sb + j * C::kBQuarter);
+#pragma unroll
+                        for (int k = 0; k < kBK / 16; ++k) {
+                            const uint32_t acc = (ks | j | k) != 0;
+                            // 16 K elements = 8 TMEM columns of A; +32 bytes of B per K step
+                            umma_bf16_ts(d0, a0 + 8 * k, db + 2 * k, idesc, acc);
+                            if (SWIGLU) umma_bf16_ts(d0 + BN, a0 + 32 + 8 * k, db + 2 * k, idesc, acc);
+                        }
+                        umma_commit(&tfree_bar[t]);
+                        if (++t == C::kTmemAStages) { t = 0; tphase ^= 1; }
+                    }
+                    if (!ok) break;
+                    umma_commit(&empty_bar[stage]);
+                    if (++stage == STAGES) stage = 0;
+                }
+                if (!ok) break;
+                umma_commit(&tfull_bar[buf]);
+                if (++buf == 2) { buf = 0; bphase ^= 1; }
+            }
+            umma_commit(drain_bar);
+            volatile int never = 0;
+            mbar_wait(drain_bar, 0, &never, p.err);
+        }
+    } else if (warp < 6) {
+        run_epilogue<BN, SWIGLU, C::kAccCols>(p, pre_s, off_s, total_tiles, MB, tmem_base, tfull_bar, tempty_bar,
+                                              abort_flag);
+    } else {
+        // ====== warps 6-21: decode group g = quarter g of every ring stage =======
+        // Row r of the tile, packed bytes [32g, 32g+32) of the stage's 128-byte
+        // row (stored with the 128-byte swizzle: 16-byte chunk c of row r sits
+        // at chunk c ^ (r % 8)), K elements 64g .. 64g+63 of the stage.
+        const int g = (warp - 6) >> 2;
+        const int q = warp & 3;                 // TMEM lane quarter = rows q*32 .. q*32+31
+        const int r = q * 32 + lane;
+        const int kgroups = p.K / 128;
+        const size_t srows = static_cast<size_t>(p.E) * p.w_rows;
+        // position of the next stage to decode: tile n_tile, stage ks n_ks
+        int n_tile = blockIdx.x, n_ks = 0;
+        const uint16_t *n_srow[2] = {nullptr, nullptr};   // scale rows of n_tile
+        auto set_rows = [&]() {
+            n_srow[0] = n_srow[1] = nullptr;
+            if (n_tile >= total_tiles) return;
+            const TileInfo ti = decode_tile(n_tile, pre_s, off_s, E, MB, BN);
+            const size_t row_g = static_cast<size_t>(ti.e) * p.w_rows + ti.mb * kBM + r;
+#pragma unroll
+            for (int a = 0; a < C::kNumA; ++a) {
+                const size_t row = row_g + static_cast<size_t>(a) * p.m_out;
+                if (row < srows) n_srow[a] = p.w_scales + row * kgroups;
+            }
+        };
+        auto fetch = [&](uint16_t (&sb)[2]) {
+            const int grp = n_ks * 2 + (g >> 1);           // the 128-K scale group of quarter g
+#pragma unroll
+            for (int a = 0; a < 2; ++a)
+                sb[a] = (a < C::kNumA && n_srow[a] && grp < kgroups) ? __ldg(n_srow[a] + grp) : 0;
+        };
+        // scales of the stage being decoded (sb_cur), and of the next one
+        // (sb_next): fetches run two stages ahead of their use
+        set_rows();
+        uint16_t sb_cur[2], sb_next[2];
+        fetch(sb_cur);
+        auto step = [&]() {
+            if (++n_ks == KS) {
+                n_ks = 0;
+                n_tile += gridDim.x;
+                set_rows();
+            }
+        };
+        int c_tile = n_tile;          // tile of the stage being decoded
+        step();
+        fetch(sb_next);
+        int stage = 0;
+        uint32_t sphase = 0;
+        int t = g % C::kTmemAStages;
+        uint32_t tphase = (g / C::kTmemAStages) & 1;
+        const int ch0 = ((2 * g) ^ (r & 7)) << 4, ch1 = ((2 * g + 1) ^ (r & 7)) << 4;
+        while (c_tile < total_tiles) {
+            const uint16_t sb0 = sb_cur[0], sb1 = sb_cur[1];
+            sb_cur[0] = sb_next[0];
+            sb_cur[1] = sb_next[1];
+            c_tile = n_tile;
+            step();
+            fetch(sb_next);
+            bool ok = mbar_wait(&full_bar[stage], sphase, abort_flag, p.err, 0);
+            if (ok) ok = mbar_wait(&tfree_bar[t], tphase ^ 1, abort_flag, p.err, 0);
+            if (!ok) break;
+            tc_fence_after_sync();
+            const uint8_t *st = ring + stage * C::kStageBytes + r * 128;
+#pragma unroll
+            for (int a = 0; a < C::kNumA; ++a) {
+                const uint4 p0 = *reinterpret_cast<const uint4 *>(st + a * kPackedTile + ch0);
+                const uint4 p1 = *reinterpret_cast<const uint4 *>(st + a * kPackedTile + ch1);
+                const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+                const __nv_bfloat162 s2 = bf16_pair(a == 0 ? sb0 : sb1);
+                uint32_t out[32];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) dequant_word(words[i], s2, out + 4 * i);
+                tmem_st_32x32b_x32(tmem_a0 + (static_cast<uint32_t>(q * 32) << 16) + t * C::kACols + a * 32, out);
+            }
+            tmem_wait_st();
+            tc_fence_before_sync();
+            mbar_arrive(&tready_bar[t]);
+            if (++stage == STAGES) { stage = 0; sphase ^= 1; }
+            // this group's next quarter is kQuarters ring slots further on
+            t += kConvGroups;
+            while (t >= C::kTmemAStages) { t -= C::kTmemAStages; tphase ^= 1; }
+        }
+    }
+
+    __syncthreads();
+    if (*abort_flag) {
         for (int i = 0; i < 1000; ++i) __nanosleep(1000);
     }
     if (warp == 1) {
@@ -415,21 +656,7 @@ int num_sms() {
     return n;
 }
 
-template <int BN, int STAGES, bool SWIGLU, bool INT4>
-cudaError_t run(const GemmArgs &g, cudaStream_t s) {
-    using C = Cfg<BN, STAGES, SWIGLU, INT4>;
-    CUtensorMap ta, tb;
-    const uint64_t a_rows = static_cast<uint64_t>(g.E) * g.w_rows;
-    bool ok;
-    if (INT4)
-        ok = make_map(&ta, g.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.K / 2, a_rows, kBK / 2, kBM,
-                      CU_TENSOR_MAP_SWIZZLE_NONE);
-    else
-        ok = make_map(&ta, g.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.K, a_rows, kBK, kBM,
-                      CU_TENSOR_MAP_SWIZZLE_128B);
-    ok = ok && make_map(&tb, g.a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.K, g.P, kBK, kBoxN,
-                        CU_TENSOR_MAP_SWIZZLE_128B);
-    if (!ok) return cudaErrorInvalidValue;
+Params make_params(const GemmArgs &g, int BN) {
     Params p;
     p.offsets = g.offsets;
     p.E = g.E;
@@ -441,32 +668,81 @@ cudaError_t run(const GemmArgs &g, cudaStream_t s) {
     p.err = g.err;
     p.w_scales = g.w_scales;
     p.evict_first_weights = BN <= 32;
-    auto kern = grouped_gemm_kernel<BN, STAGES, SWIGLU, INT4>;
-    cudaError_t st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
-    if (st != cudaSuccess) return st;
+    return p;
+}
+
+int grid_for(const GemmArgs &g, int BN) {
     const long long MB = (g.m_out + kBM - 1) / kBM;
     const long long max_tiles = ((static_cast<long long>(g.P) + BN - 1) / BN + std::min(g.E, g.P)) * MB;
-    const int grid = static_cast<int>(std::min<long long>(num_sms(), max_tiles));
+    return static_cast<int>(std::min<long long>(num_sms(), max_tiles));
+}
+
+template <int BN, int STAGES, bool SWIGLU>
+cudaError_t run_bf16(const GemmArgs &g, cudaStream_t s) {
+    using C = Bf16Cfg<BN, STAGES, SWIGLU>;
+    CUtensorMap ta, tb;
+    const uint64_t a_rows = static_cast<uint64_t>(g.E) * g.w_rows;
+    bool ok = make_map(&ta, g.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.K, a_rows, kBK, kBM,
+                       CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&tb, g.a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.K, g.P, kBK, kBoxN,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return cudaErrorInvalidValue;
+    auto kern = grouped_gemm_kernel<BN, STAGES, SWIGLU>;
+    cudaError_t st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (st != cudaSuccess) return st;
+    const int grid = grid_for(g, BN);
     if (grid <= 0) return cudaSuccess;
-    kern<<<grid, kThreads, C::kSmemBytes, s>>>(ta, tb, p);
+    kern<<<grid, C::kThreads, C::kSmemBytes, s>>>(ta, tb, make_params(g, BN));
     return cudaGetLastError();
 }
 
-template <bool SWIGLU, bool INT4>
-cudaError_t dispatch_bn(const GemmArgs &g, cudaStream_t s) {
+template <int BN, int STAGES, bool SWIGLU>
+cudaError_t run_int4(const GemmArgs &g, cudaStream_t s) {
+    using C = Int4Cfg<BN, STAGES, SWIGLU>;
+    CUtensorMap ta, tb;
+    const uint64_t a_rows = static_cast<uint64_t>(g.E) * g.w_rows;
+    // packed weights: 128 bytes (K = 256) per row and stage, 128-byte swizzle
+    bool ok = make_map(&ta, g.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.K / 2, a_rows, 128, kBM,
+                       CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&tb, g.a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.K, g.P, kBK, kBoxN,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!ok) return cudaErrorInvalidValue;
+    auto kern = grouped_gemm_int4_kernel<BN, STAGES, SWIGLU>;
+    cudaError_t st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (st != cudaSuccess) return st;
+    const int grid = grid_for(g, BN);
+    if (grid <= 0) return cudaSuccess;
+    kern<<<grid, C::kThreads, C::kSmemBytes, s>>>(ta, tb, make_params(g, BN));
+    return cudaGetLastError();
+}
+
+template <bool SWIGLU>
+cudaError_t dispatch_bf16(const GemmArgs &g, cudaStream_t s) {
     const double avg = static_cast<double>(g.P) / g.E;   // pairs per expert if the load were even
-    if (SWIGLU) {
-        if (avg <= 24) return run<32, INT4 ? 4 : 6, SWIGLU, INT4>(g, s);
-        if (avg <= 48) return run<64, INT4 ? 4 : 5, SWIGLU, INT4>(g, s);
-        return run<128, INT4 ? 3 : 4, SWIGLU, INT4>(g, s);
+    if constexpr (SWIGLU) {
+        if (avg <= 24) return run_bf16<32, 6, SWIGLU>(g, s);
+        if (avg <= 48) return run_bf16<64, 5, SWIGLU>(g, s);
+        return run_bf16<128, 4, SWIGLU>(g, s);
     } else {
-        if (avg <= 24) return run<32, INT4 ? 8 : 10, SWIGLU, INT4>(g, s);
-        if (avg <= 48) return run<64, INT4 ? 6 : 8, SWIGLU, INT4>(g, s);
-        return run<128, INT4 ? 5 : 6, SWIGLU, INT4>(g, s);
+        if (avg <= 24) return run_bf16<32, 10, SWIGLU>(g, s);
+        if (avg <= 48) return run_bf16<64, 8, SWIGLU>(g, s);
+        return run_bf16<128, 6, SWIGLU>(g, s);
     }
 }
 
-// Standalone W4A16 decoding (same arithmetic as the GEMMs' converter warps).
+template <bool SWIGLU>
+cudaError_t dispatch_int4(const GemmArgs &g, cudaStream_t s) {
+    const double avg = static_cast<double>(g.P) / g.E;
+    if constexpr (SWIGLU) {
+        if (avg <= 24) return run_int4<32, 4, SWIGLU>(g, s);    // 48 KB stages
+        return run_int4<64, 3, SWIGLU>(g, s);                   // 64 KB stages
+    } else {
+        if (avg <= 24) return run_int4<32, 6, SWIGLU>(g, s);    // 32 KB stages
+        return run_int4<64, 4, SWIGLU>(g, s);                   // 48 KB stages
+    }
+}
+
+// Standalone W4A16 decoding: the same dequant_word as the GEMMs' decode warps.
 __global__ void dequant_int4_kernel(const uint4 *__restrict__ q, const uint16_t *__restrict__ scales, int rows,
                                     int K, uint4 *__restrict__ out) {
     const long long chunks_per_row = K / 32;   // 16 packed bytes = 32 values
@@ -475,11 +751,14 @@ __global__ void dequant_int4_kernel(const uint4 *__restrict__ q, const uint16_t 
          i += static_cast<long long>(gridDim.x) * blockDim.x) {
         const long long r = i / chunks_per_row;
         const int c = static_cast<int>(i - r * chunks_per_row);
-        const float scale = bf16_bits_to_float(__ldg(scales + r * (K / 128) + (c * 32) / 128));
-        uint4 o[4];
-        dequant32(__ldg(q + i), scale, o);
+        const __nv_bfloat162 s2 = bf16_pair(__ldg(scales + r * (K / 128) + (c * 32) / 128));
+        const uint4 pk = __ldg(q + i);
+        const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
+        uint32_t o[16];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) out[i * 4 + j] = o[j];
+        for (int w = 0; w < 4; ++w) dequant_word(words[w], s2, o + 4 * w);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) out[i * 4 + j] = make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
     }
 }
 
@@ -487,8 +766,8 @@ __global__ void dequant_int4_kernel(const uint4 *__restrict__ q, const uint16_t 
 
 cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t s) {
     if (g.P == 0) return cudaSuccess;
-    if (g.fmt == 0) return g.swiglu ? dispatch_bn<true, false>(g, s) : dispatch_bn<false, false>(g, s);
-    return g.swiglu ? dispatch_bn<true, true>(g, s) : dispatch_bn<false, true>(g, s);
+    if (g.fmt == 0) return g.swiglu ? dispatch_bf16<true>(g, s) : dispatch_bf16<false>(g, s);
+    return g.swiglu ? dispatch_int4<true>(g, s) : dispatch_int4<false>(g, s);
 }
 
 cudaError_t launch_dequant_int4(const uint8_t *q, const uint16_t *scales, int rows, int K, uint16_t *out,
