@@ -71,8 +71,8 @@ typedef uint16_t moe_bf16_t;   /* bit pattern of a bfloat16 value */
 typedef void *moe_stream_t;    /* cudaStream_t */
 
 /* Bytes of device workspace moe_forward needs for this shape (0 if the shape
- * is invalid). It holds the routing, the permutation, the gathered rows
- * [T*k,H], act [T*k,I] and y [T*k,H]. */
+ * is invalid). It holds the routing, the permutation, act [T*k,I], y [T*k,H]
+ * and, when many tokens share each expert, the gathered rows [T*k,H]. */
 MOE_API size_t moe_workspace_size(const moe_shape_t *shape);
 
 /* Bytes of scratch moe_permute needs (may be 0). */
@@ -109,8 +109,11 @@ MOE_API moe_status_t moe_permute(const int32_t *topk_ids, const moe_shape_t *sha
 /* Grouped GEMM gate/up with fused SwiGLU. InfiniLM PR #500 report §2.2 step 2
  * (grouped GEMM over all experts in one call, then SwiGLU); FlashInfer PR
  * #7196 analysis §2 (tokens on the MMA N side with a runtime N per tile).
- *   a       [T*top_k,H] bf16 rows in permuted order (hidden_perm)
- *   perm    must be NULL (a gather fused into the operand load is not offered)
+ *   a       perm == NULL: [T*top_k,H] bf16 rows in permuted order (hidden_perm).
+ *           perm != NULL: hidden [T,H] bf16; row r of the operand is
+ *           a[perm[r] / top_k], gathered inside the GEMM (TMA gather4), so
+ *           the permuted copy is never written.
+ *   perm    NULL, or [T*top_k] from moe_permute
  *   offsets [E+1] from moe_permute
  *   w_gu    MOE_W_BF16: [E,2I,H] bf16, rows [0,I) gate, rows [I,2I) up.
  *           MOE_W_INT4_G128: [E,2I,H/2] bytes, low nibble = even K index,
@@ -140,8 +143,10 @@ MOE_API moe_status_t moe_grouped_gemm_down(const moe_bf16_t *act, const int32_t 
 MOE_API moe_status_t moe_finalize(const moe_bf16_t *y, const float *topk_w, const int32_t *inv_perm,
                           const moe_shape_t *shape, moe_bf16_t *out, moe_stream_t stream);
 
-/* The whole layer: route, permute (with gather), gate/up + SwiGLU, down,
- * finalize, enqueued on one stream with no host synchronisation.
+/* The whole layer: route, permute (with the gather when many tokens share
+ * each expert; otherwise the gate/up GEMM gathers through perm itself),
+ * gate/up + SwiGLU, down, finalize, enqueued on one stream with no host
+ * synchronisation.
  *   hidden [T,H] bf16, logits [T,E] fp32, weights as above, out [T,H] bf16.
  *   ws: at least moe_workspace_size(shape) bytes, 256-byte aligned. */
 MOE_API moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits,
@@ -183,8 +188,8 @@ MOE_API moe_status_t moe_get_device_error(int32_t *code);
  * counterpart to this entry point.
  *   Arguments as moe_permute, without ws/ws_bytes. It allocates nothing and
  *   calls no allocating routine.
- *   Limit: the per-chunk histogram, ceil(T*top_k / 8192) * E int32 entries,
- *   must fit 65536 entries. For example, E = 128 allows up to 4,194,304
+ *   Limit: the per-chunk histogram, ceil(T*top_k / 2048) * E int32 entries,
+ *   must fit 65536 entries. For example, E = 128 allows up to 1,048,576
  *   pairs. Larger calls return MOE_ERR_UNSUPPORTED before anything is
  *   enqueued. Calls with T*top_k <= 8192 use no scratch at all.
  *   The array exists once per GPU that loads the library and is held until

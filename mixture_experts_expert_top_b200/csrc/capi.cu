@@ -70,7 +70,7 @@ Layout layout(const moe_shape_t *s, bool host) {
     L.perm = take(P * 4);
     L.inv = take(P * 4);
     L.scratch = take(moe::permute_scratch_bytes(static_cast<long long>(P), s->E));
-    L.hperm = take(P * s->H * 2);
+    L.hperm = moe::gemm_gathers_in_kernel(static_cast<int>(P), s->E, s->fmt) ? o : take(P * s->H * 2);
     L.act = take(P * s->I * 2);
     L.y = take(P * s->H * 2);
     L.hidden_in = L.logits_in = L.out_st = 0;
@@ -83,10 +83,13 @@ Layout layout(const moe_shape_t *s, bool host) {
     return L;
 }
 
-moe::GemmArgs gemm_args(const moe_shape_t *s, const void *a, const int32_t *offsets, const void *w,
-                        const moe_bf16_t *scales, bool swiglu, moe_bf16_t *out) {
+moe::GemmArgs gemm_args(const moe_shape_t *s, const void *a, const int32_t *perm, const int32_t *offsets,
+                        const void *w, const moe_bf16_t *scales, bool swiglu, moe_bf16_t *out) {
     moe::GemmArgs g;
     g.a = a;
+    g.perm = perm;
+    g.T = s->T;
+    g.top_k = s->top_k;
     g.offsets = offsets;
     g.w = w;
     g.w_scales = scales;
@@ -124,7 +127,6 @@ moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const
     auto *offsets = reinterpret_cast<int32_t *>(ws + L.offsets);
     auto *perm = reinterpret_cast<int32_t *>(ws + L.perm);
     auto *inv = reinterpret_cast<int32_t *>(ws + L.inv);
-    auto *hperm = reinterpret_cast<uint16_t *>(ws + L.hperm);
     auto *act = reinterpret_cast<uint16_t *>(ws + L.act);
     auto *y = reinterpret_cast<uint16_t *>(ws + L.y);
     cudaError_t e;
@@ -132,11 +134,20 @@ moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const
     if ((e = moe::launch_permute(ids, P, E, counts, offsets, perm, inv, ws + L.scratch, error_flag_ptr(), st)) !=
         cudaSuccess)
         return cuda_status(e);
-    if ((e = moe::launch_gather(hidden, perm, P, H, k, hperm, st)) != cudaSuccess) return cuda_status(e);
-    if ((e = moe::launch_grouped_gemm(gemm_args(s, hperm, offsets, w_gu, w_gu_scales, true, act), st)) !=
+    // Few rows per expert: the gate/up GEMM gathers the token rows itself (TMA
+    // gather4 through perm). Many rows per expert: one gather kernel writes the
+    // permuted rows and the GEMM reads them as whole 128-row tiles, which keeps
+    // its TMA unit from turning into the bottleneck.
+    if (moe::gemm_gathers_in_kernel(P, E, s->fmt)) {
+        e = moe::launch_grouped_gemm(gemm_args(s, hidden, perm, offsets, w_gu, w_gu_scales, true, act), st);
+    } else {
+        auto *hperm = reinterpret_cast<uint16_t *>(ws + L.hperm);
+        if ((e = moe::launch_gather(hidden, perm, P, H, k, hperm, st)) != cudaSuccess) return cuda_status(e);
+        e = moe::launch_grouped_gemm(gemm_args(s, hperm, nullptr, offsets, w_gu, w_gu_scales, true, act), st);
+    }
+    if (e != cudaSuccess) return cuda_status(e);
+    if ((e = moe::launch_grouped_gemm(gemm_args(s, act, nullptr, offsets, w_d, w_d_scales, false, y), st)) !=
         cudaSuccess)
-        return cuda_status(e);
-    if ((e = moe::launch_grouped_gemm(gemm_args(s, act, offsets, w_d, w_d_scales, false, y), st)) != cudaSuccess)
         return cuda_status(e);
     return cuda_status(moe::launch_finalize(y, w, inv, T, H, k, out, st));
 }
@@ -205,12 +216,12 @@ moe_status_t moe_grouped_gemm_swiglu(const moe_bf16_t *a, const int32_t *perm, c
                                      moe_bf16_t *act, moe_stream_t stream) {
     moe_status_t st = check_shape(shape);
     if (st != MOE_OK) return st;
-    if (perm) return MOE_ERR_UNSUPPORTED;
     if (shape->T == 0) return MOE_OK;
     if (!a || !offsets || !act || !aligned(a, 16) || !aligned(act, 16) || !aligned(offsets, 4))
         return MOE_ERR_INVALID_ARG;
+    if (perm && !aligned(perm, 4)) return MOE_ERR_INVALID_ARG;
     if ((st = check_weights(shape, w_gu, w_gu_scales)) != MOE_OK) return st;
-    return cuda_status(moe::launch_grouped_gemm(gemm_args(shape, a, offsets, w_gu, w_gu_scales, true, act),
+    return cuda_status(moe::launch_grouped_gemm(gemm_args(shape, a, perm, offsets, w_gu, w_gu_scales, true, act),
                                                 static_cast<cudaStream_t>(stream)));
 }
 
@@ -223,7 +234,7 @@ moe_status_t moe_grouped_gemm_down(const moe_bf16_t *act, const int32_t *offsets
     if (!act || !offsets || !y || !aligned(act, 16) || !aligned(y, 16) || !aligned(offsets, 4))
         return MOE_ERR_INVALID_ARG;
     if ((st = check_weights(shape, w_d, w_d_scales)) != MOE_OK) return st;
-    return cuda_status(moe::launch_grouped_gemm(gemm_args(shape, act, offsets, w_d, w_d_scales, false, y),
+    return cuda_status(moe::launch_grouped_gemm(gemm_args(shape, act, nullptr, offsets, w_d, w_d_scales, false, y),
                                                 static_cast<cudaStream_t>(stream)));
 }
 

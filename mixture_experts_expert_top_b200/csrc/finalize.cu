@@ -24,25 +24,53 @@ __device__ __forceinline__ uint32_t pack_bf16x2_rne(float lo, float hi) {
     return static_cast<uint32_t>(__bfloat16_as_ushort(a)) | (static_cast<uint32_t>(__bfloat16_as_ushort(b)) << 16);
 }
 
+// KT > 0: top_k known at compile time, so the k row indices, weights and
+// 16-byte row loads of a thread are all issued before the combine.
+template <int KT>
 __global__ void __launch_bounds__(256)
 finalize_kernel(const uint4 *__restrict__ y, const float *__restrict__ w, const int32_t *__restrict__ inv_perm,
-                int T, int vecs_per_row, int k, int P, uint4 *__restrict__ out) {
+                int T, int vecs_per_row, int k_rt, int P, uint4 *__restrict__ out) {
+    const int k = KT > 0 ? KT : k_rt;
     const long long total = static_cast<long long>(T) * vecs_per_row;
     for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
          i += static_cast<long long>(gridDim.x) * blockDim.x) {
         const int t = static_cast<int>(i / vecs_per_row);
         const int v = static_cast<int>(i - static_cast<long long>(t) * vecs_per_row);
         float acc[8];
-        for (int j = 0; j < k; ++j) {
-            const int r = __ldg(inv_perm + static_cast<size_t>(t) * k + j);
-            const float wj = __ldg(w + static_cast<size_t>(t) * k + j);
-            uint4 q = make_uint4(0u, 0u, 0u, 0u);
-            if (r >= 0 && r < P) q = __ldg(y + static_cast<size_t>(r) * vecs_per_row + v);
-            const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
+        if constexpr (KT > 0) {
+            int r[KT];
+            float wj[KT];
+            uint4 q[KT];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                const float x = bf16_bits_to_float((qs[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu);
-                acc[e] = (j == 0) ? __fmul_rn(x, wj) : __fmaf_rn(x, wj, acc[e]);
+            for (int j = 0; j < KT; ++j) {
+                r[j] = __ldg(inv_perm + static_cast<size_t>(t) * KT + j);
+                wj[j] = __ldg(w + static_cast<size_t>(t) * KT + j);
+            }
+#pragma unroll
+            for (int j = 0; j < KT; ++j)
+                q[j] = (r[j] >= 0 && r[j] < P) ? __ldcs(y + static_cast<size_t>(r[j]) * vecs_per_row + v)
+                                               : make_uint4(0u, 0u, 0u, 0u);   // y is read once
+#pragma unroll
+            for (int j = 0; j < KT; ++j) {
+                const uint32_t qs[4] = {q[j].x, q[j].y, q[j].z, q[j].w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float x = bf16_bits_to_float((qs[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu);
+                    acc[e] = (j == 0) ? __fmul_rn(x, wj[j]) : __fmaf_rn(x, wj[j], acc[e]);
+                }
+            }
+        } else {
+            for (int j = 0; j < k; ++j) {
+                const int r = __ldg(inv_perm + static_cast<size_t>(t) * k + j);
+                const float wj = __ldg(w + static_cast<size_t>(t) * k + j);
+                uint4 q = make_uint4(0u, 0u, 0u, 0u);
+                if (r >= 0 && r < P) q = __ldg(y + static_cast<size_t>(r) * vecs_per_row + v);
+                const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const float x = bf16_bits_to_float((qs[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu);
+                    acc[e] = (j == 0) ? __fmul_rn(x, wj) : __fmaf_rn(x, wj, acc[e]);
+                }
             }
         }
         uint4 o;
@@ -50,8 +78,15 @@ finalize_kernel(const uint4 *__restrict__ y, const float *__restrict__ w, const 
         o.y = pack_bf16x2_rne(acc[2], acc[3]);
         o.z = pack_bf16x2_rne(acc[4], acc[5]);
         o.w = pack_bf16x2_rne(acc[6], acc[7]);
-        out[i] = o;
+        __stcs(out + i, o);
     }
+}
+
+template <int KT>
+void launch_finalize_t(int blocks, cudaStream_t s, const uint16_t *y, const float *w, const int32_t *inv_perm, int T,
+                       int vpr, int k, int P, uint16_t *out) {
+    finalize_kernel<KT><<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4 *>(y), w, inv_perm, T, vpr, k, P,
+                                               reinterpret_cast<uint4 *>(out));
 }
 
 }  // namespace
@@ -63,8 +98,15 @@ cudaError_t launch_finalize(const uint16_t *y, const float *w, const int32_t *in
     const long long total = static_cast<long long>(T) * vpr;
     long long blocks = (total + 255) / 256;
     if (blocks > 148LL * 32) blocks = 148LL * 32;
-    finalize_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(reinterpret_cast<const uint4 *>(y), w, inv_perm, T,
-                                                             vpr, k, T * k, reinterpret_cast<uint4 *>(out));
+    const int b = static_cast<int>(blocks);
+    switch (k) {
+        case 1: launch_finalize_t<1>(b, s, y, w, inv_perm, T, vpr, k, T * k, out); break;
+        case 2: launch_finalize_t<2>(b, s, y, w, inv_perm, T, vpr, k, T * k, out); break;
+        case 4: launch_finalize_t<4>(b, s, y, w, inv_perm, T, vpr, k, T * k, out); break;
+        case 6: launch_finalize_t<6>(b, s, y, w, inv_perm, T, vpr, k, T * k, out); break;
+        case 8: launch_finalize_t<8>(b, s, y, w, inv_perm, T, vpr, k, T * k, out); break;
+        default: launch_finalize_t<0>(b, s, y, w, inv_perm, T, vpr, k, T * k, out); break;
+    }
     return cudaGetLastError();
 }
 

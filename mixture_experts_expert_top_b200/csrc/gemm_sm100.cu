@@ -31,143 +31,12 @@
 //    move (packed in, bf16 out, bf16 read again by the MMA).
 //  - Every wait is bounded (see mbar_wait); a timeout raises the device flag
 //    and unwinds the CTA.
-#include <cudaTypedefs.h>
-#include <math.h>
-
-#include <algorithm>
-
-#include "common.cuh"
-#include "launch.h"
+#include "gemm_common.cuh"
 
 namespace moe {
 namespace {
 
-constexpr int kBM = 128;          // weight rows per tile (MMA M)
-constexpr int kBK = 64;           // K elements per bf16 stage / per int4 quarter (one 128-byte bf16 row)
-constexpr int kBoxN = 16;         // token rows per TMA box
-constexpr int kTileBytesA = kBM * kBK * 2;          // 16 KB bf16 tile (128 x 64)
-constexpr int kBoxBytesB = kBoxN * kBK * 2;         // 2 KB token box (16 x 64)
-constexpr int kMaxExperts = 1024;
-constexpr int kSmemLimit = 232448;                  // 227 KB per CTA
-constexpr int kEpiThreads = 128;                    // warps 2-5
-
-// int4 kernel
-constexpr int kQuarters = 4;                        // 64-K quarters per int4 stage (K = 256)
-constexpr int kPackedTile = kBM * 128;              // 16 KB: 128 rows x 128 packed bytes
-constexpr int kConvGroups = kQuarters;              // decode group g handles quarter g of every stage
-constexpr int kMaxTmemA = 8;
-
-struct Params {
-    const int32_t *offsets;
-    int E, K, m_out, w_rows, P;
-    uint16_t *out;
-    int *err;
-    const uint16_t *w_scales;   // int4: [E * w_rows, K/128]
-    int evict_first_weights;
-};
-
-// Tile bookkeeping shared by the roles.
-struct TileInfo {
-    int e, mb, row0, valid, n_mma;
-};
-
-__device__ __forceinline__ TileInfo decode_tile(int tile, const int *pre, const int *off, int E, int MB, int BN) {
-    int lo = 0, hi = E - 1;             // largest e with pre[e] <= tile (never an empty expert)
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (pre[mid] <= tile) lo = mid; else hi = mid - 1;
-    }
-    TileInfo t;
-    t.e = lo;
-    const int local = tile - pre[lo];
-    t.mb = local % MB;
-    const int nb = local / MB;
-    t.row0 = off[lo] + nb * BN;
-    const int cnt = off[lo + 1] - off[lo];
-    t.valid = min(BN, cnt - nb * BN);
-    t.n_mma = (t.valid + 15) & ~15;
-    return t;
-}
-
-// Copies offsets into shared memory and builds pre[e] = number of tiles of
-// experts 0..e-1 (a block-wide scan). All threads of the CTA call it.
-template <int NT>
-__device__ __forceinline__ void build_tile_prefix(const int32_t *offsets, int E, int MB, int BN, int *off_s,
-                                                  int *pre_s) {
-    __shared__ int wsum[NT / 32];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int i = threadIdx.x; i <= E; i += NT) off_s[i] = __ldg(offsets + i);
-    __syncthreads();
-    const int seg = (E + NT - 1) / NT;
-    const int b0 = threadIdx.x * seg;
-    int local = 0;
-    for (int i = 0; i < seg; ++i) {
-        const int e = b0 + i;
-        if (e < E) {
-            const int cnt = off_s[e + 1] - off_s[e];
-            local += ((cnt + BN - 1) / BN) * MB;
-            pre_s[e + 1] = local;        // segment-local inclusive
-        }
-    }
-    int x = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) wsum[warp] = x;
-    __syncthreads();
-    int before = x - local;
-    for (int w = 0; w < warp; ++w) before += wsum[w];
-    for (int i = 0; i < seg; ++i) {
-        const int e = b0 + i;
-        if (e < E) pre_s[e + 1] += before;
-    }
-    if (threadIdx.x == 0) pre_s[0] = 0;
-}
-
-// Epilogue of warps 2-5: per tile, wait for the accumulator buffer, read it
-// with tcgen05.ld (warp w reads TMEM lanes 32*(w%4)...), apply SwiGLU for
-// gate/up, round to bf16 and store; then hand the buffer back.
-template <int BN, bool SWIGLU, int ACC_COLS>
-__device__ __forceinline__ void run_epilogue(const Params &p, const int *pre_s, const int *off_s, int total_tiles,
-                                             int MB, uint32_t tmem_base, uint64_t *tfull_bar, uint64_t *tempty_bar,
-                                             volatile int *abort_flag) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int q = warp & 3;
-    int buf = 0;
-    uint32_t bphase = 0;
-    for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-        const TileInfo ti = decode_tile(tile, pre_s, off_s, p.E, MB, BN);
-        if (!mbar_wait(&tfull_bar[buf], bphase, abort_flag, p.err, 512)) break;
-        tc_fence_after_sync();
-        const int f = ti.mb * kBM + q * 32 + lane;         // output feature of this thread
-        const bool f_ok = f < p.m_out;
-        const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * ACC_COLS;
-        for (int c0 = 0; c0 < ti.n_mma; c0 += 16) {
-            uint32_t g[16], u[16];
-            tmem_ld_32x32b_x16(tb + c0, g);
-            if (SWIGLU) tmem_ld_32x32b_x16(tb + BN + c0, u);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-                const int n = c0 + j;
-                if (f_ok && n < ti.valid) {
-                    float v = __uint_as_float(g[j]);
-                    if (SWIGLU) {
-                        const float uu = __uint_as_float(u[j]);
-                        v = v / (1.0f + expf(-v)) * uu;
-                    }
-                    const __nv_bfloat16 bv = __float2bfloat16_rn(v);
-                    p.out[static_cast<size_t>(ti.row0 + n) * p.m_out + f] = __bfloat16_as_ushort(bv);
-                }
-            }
-        }
-        tc_fence_before_sync();
-        mbar_arrive(&tempty_bar[buf]);
-        if (++buf == 2) { buf = 0; bphase ^= 1; }
-    }
-}
+using namespace gemm;
 
 // W4A16 decoding of one 32-bit word of packed int4 (K elements 8i..8i+7 of a
 // row; byte b holds element 2b in its low nibble, 2b+1 in its high nibble,
@@ -277,29 +146,44 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
     if (warp == 0) {
         // ================================ TMA producer ==========================
-        if (lane == 0) {
-            const uint64_t pol_w = p.evict_first_weights ? l2_policy_evict_first() : l2_policy_evict_last();
-            const uint64_t pol_x = l2_policy_evict_last();
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-                const TileInfo ti = decode_tile(tile, pre_s, off_s, E, MB, BN);
-                const int nbox = ti.n_mma / kBoxN;
-                const int a_row = ti.e * p.w_rows + ti.mb * kBM;
-                const uint32_t tx = C::kABytes + nbox * kBoxBytesB;
-                for (int kb = 0; kb < KB; ++kb) {
-                    ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.err, 256);
-                    if (!ok) break;
+        // Lane 0 runs the ring; with perm, lanes i < n_mma/4 issue the token
+        // rows as gather4 loads (tile rows 4i .. 4i+3) straight from hidden.
+        const uint64_t pol_w = p.evict_first_weights ? l2_policy_evict_first() : l2_policy_evict_last();
+        const uint64_t pol_x = l2_policy_evict_last();
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+            const TileInfo ti = decode_tile(tile, pre_s, off_s, E, MB, BN);
+            const int nbox = ti.n_mma / kBoxN;
+            const int a_row = ti.e * p.w_rows + ti.mb * kBM;
+            const uint32_t tx = C::kABytes + nbox * kBoxBytesB;
+            const bool gather_lane = p.perm && 4 * lane < ti.n_mma;
+            int tr[4] = {0, 0, 0, 0};
+            if (gather_lane) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) tr[j] = token_row(p, ti.row0 + 4 * lane + j);
+            }
+            for (int kb = 0; kb < KB; ++kb) {
+                if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.err, 0);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                uint8_t *st = ring + stage * C::kStageBytes;
+                uint8_t *sb = st + C::kABytes;
+                if (lane == 0) {
                     mbar_arrive_expect_tx(&full_bar[stage], tx);
-                    uint8_t *st = ring + stage * C::kStageBytes;
                     tma_load_2d(st, &tmA, &full_bar[stage], kb * kBK, a_row, pol_w);
                     if (SWIGLU) tma_load_2d(st + kTileBytesA, &tmA, &full_bar[stage], kb * kBK, a_row + p.m_out, pol_w);
-                    uint8_t *sb = st + C::kABytes;
-                    for (int b = 0; b < nbox; ++b)
-                        tma_load_2d(sb + b * kBoxBytesB, &tmB, &full_bar[stage], kb * kBK, ti.row0 + b * kBoxN, pol_x);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    if (!p.perm)
+                        for (int b = 0; b < nbox; ++b)
+                            tma_load_2d(sb + b * kBoxBytesB, &tmB, &full_bar[stage], kb * kBK, ti.row0 + b * kBoxN,
+                                        pol_x);
                 }
+                __syncwarp();
+                if (gather_lane)
+                    tma_gather4(sb + lane * 4 * kBK * 2, &tmB, &full_bar[stage], kb * kBK, tr[0], tr[1], tr[2], tr[3],
+                                pol_x);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
         }
     } else if (warp == 1) {
@@ -346,7 +230,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
     } else {
         run_epilogue<BN, SWIGLU, C::kAccCols>(p, pre_s, off_s, total_tiles, MB, tmem_base, tfull_bar, tempty_bar,
-                                              abort_flag);
+                                              abort_flag, 128);
     }
 
     __syncthreads();
@@ -450,31 +334,44 @@ grouped_gemm_int4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
 
     if (warp == 0) {
         // ================================ TMA producer ==========================
-        if (lane == 0) {
-            const uint64_t pol_w = p.evict_first_weights ? l2_policy_evict_first() : l2_policy_evict_last();
-            const uint64_t pol_x = l2_policy_evict_last();
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-                const TileInfo ti = decode_tile(tile, pre_s, off_s, E, MB, BN);
-                const int nbox = ti.n_mma / kBoxN;
-                const int a_row = ti.e * p.w_rows + ti.mb * kBM;
-                const uint32_t tx = C::kABytes + kQuarters * nbox * kBoxBytesB;
-                for (int ks = 0; ks < KS; ++ks) {
-                    ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.err, 256);
-                    if (!ok) break;
+        const uint64_t pol_w = p.evict_first_weights ? l2_policy_evict_first() : l2_policy_evict_last();
+        const uint64_t pol_x = l2_policy_evict_last();
+        int stage = 0;
+        uint32_t phase = 0;
+        bool ok = true;
+        for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+            const TileInfo ti = decode_tile(tile, pre_s, off_s, E, MB, BN);
+            const int nbox = ti.n_mma / kBoxN;
+            const int a_row = ti.e * p.w_rows + ti.mb * kBM;
+            const uint32_t tx = C::kABytes + kQuarters * nbox * kBoxBytesB;
+            const bool gather_lane = p.perm && 4 * lane < ti.n_mma;
+            int tr[4] = {0, 0, 0, 0};
+            if (gather_lane) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) tr[j] = token_row(p, ti.row0 + 4 * lane + j);
+            }
+            for (int ks = 0; ks < KS; ++ks) {
+                if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.err, 256);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                uint8_t *st = ring + stage * C::kStageBytes;
+                uint8_t *sb = st + C::kABytes;
+                if (lane == 0) {
                     mbar_arrive_expect_tx(&full_bar[stage], tx);
-                    uint8_t *st = ring + stage * C::kStageBytes;
                     tma_load_2d(st, &tmA, &full_bar[stage], ks * 128, a_row, pol_w);
                     if (SWIGLU) tma_load_2d(st + kPackedTile, &tmA, &full_bar[stage], ks * 128, a_row + p.m_out, pol_w);
-                    uint8_t *sb = st + C::kABytes;
-                    for (int j = 0; j < kQuarters; ++j)
-                        for (int b = 0; b < nbox; ++b)
-                            tma_load_2d(sb + j * C::kBQuarter + b * kBoxBytesB, &tmB, &full_bar[stage],
-                                        (ks * kQuarters + j) * kBK, ti.row0 + b * kBoxN, pol_x);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
+                    if (!p.perm)
+                        for (int j = 0; j < kQuarters; ++j)
+                            for (int b = 0; b < nbox; ++b)
+                                tma_load_2d(sb + j * C::kBQuarter + b * kBoxBytesB, &tmB, &full_bar[stage],
+                                            (ks * kQuarters + j) * kBK, ti.row0 + b * kBoxN, pol_x);
                 }
+                __syncwarp();
+                if (gather_lane)
+                    for (int j = 0; j < kQuarters; ++j)
+                        tma_gather4(sb + j * C::kBQuarter + lane * 4 * kBK * 2, &tmB, &full_bar[stage],
+                                    (ks * kQuarters + j) * kBK, tr[0], tr[1], tr[2], tr[3], pol_x);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
         }
     } else if (warp == 1) {
@@ -624,59 +521,6 @@ grouped_gemm_int4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
 
 // ------------------------------------------------------------------ host side
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
-// 2-D row-major map: `cols` contiguous elements per row, `rows` rows.
-bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem_bytes, uint64_t cols,
-              uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {cols, rows};
-    cuuint64_t strides[1] = {cols * static_cast<uint64_t>(elem_bytes)};
-    cuuint32_t box[2] = {box_cols, box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
-              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-int num_sms() {
-    int dev = 0, n = 148;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    return n;
-}
-
-Params make_params(const GemmArgs &g, int BN) {
-    Params p;
-    p.offsets = g.offsets;
-    p.E = g.E;
-    p.K = g.K;
-    p.m_out = g.m_out;
-    p.w_rows = g.w_rows;
-    p.P = g.P;
-    p.out = g.out;
-    p.err = g.err;
-    p.w_scales = g.w_scales;
-    p.evict_first_weights = BN <= 32;
-    return p;
-}
-
-int grid_for(const GemmArgs &g, int BN) {
-    const long long MB = (g.m_out + kBM - 1) / kBM;
-    const long long max_tiles = ((static_cast<long long>(g.P) + BN - 1) / BN + std::min(g.E, g.P)) * MB;
-    return static_cast<int>(std::min<long long>(num_sms(), max_tiles));
-}
-
 template <int BN, int STAGES, bool SWIGLU>
 cudaError_t run_bf16(const GemmArgs &g, cudaStream_t s) {
     using C = Bf16Cfg<BN, STAGES, SWIGLU>;
@@ -684,8 +528,7 @@ cudaError_t run_bf16(const GemmArgs &g, cudaStream_t s) {
     const uint64_t a_rows = static_cast<uint64_t>(g.E) * g.w_rows;
     bool ok = make_map(&ta, g.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.K, a_rows, kBK, kBM,
                        CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_map(&tb, g.a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.K, g.P, kBK, kBoxN,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
+              make_token_map(&tb, g, kBoxN);
     if (!ok) return cudaErrorInvalidValue;
     auto kern = grouped_gemm_kernel<BN, STAGES, SWIGLU>;
     cudaError_t st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -704,8 +547,7 @@ cudaError_t run_int4(const GemmArgs &g, cudaStream_t s) {
     // packed weights: 128 bytes (K = 256) per row and stage, 128-byte swizzle
     bool ok = make_map(&ta, g.w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, g.K / 2, a_rows, 128, kBM,
                        CU_TENSOR_MAP_SWIZZLE_128B) &&
-              make_map(&tb, g.a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.K, g.P, kBK, kBoxN,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
+              make_token_map(&tb, g, kBoxN);
     if (!ok) return cudaErrorInvalidValue;
     auto kern = grouped_gemm_int4_kernel<BN, STAGES, SWIGLU>;
     cudaError_t st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
@@ -762,11 +604,20 @@ __global__ void dequant_int4_kernel(const uint4 *__restrict__ q, const uint16_t 
     }
 }
 
+// Many rows per expert: bf16 weights go to the tokens-on-M kernel.
+bool uses_prefill_kernel(long long P, int E, int fmt) { return fmt == 0 && P >= 64LL * E; }
+
 }  // namespace
+
+bool gemm_gathers_in_kernel(int P, int E, int fmt) { return !uses_prefill_kernel(P, E, fmt); }
 
 cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t s) {
     if (g.P == 0) return cudaSuccess;
-    if (g.fmt == 0) return g.swiglu ? dispatch_bf16<true>(g, s) : dispatch_bf16<false>(g, s);
+    if (g.fmt == 0) {
+        // many tokens per expert: tokens on M, 128 x 256 tiles (gemm_prefill_sm100.cu)
+        if (uses_prefill_kernel(g.P, g.E, g.fmt)) return launch_grouped_gemm_prefill(g, s);
+        return g.swiglu ? dispatch_bf16<true>(g, s) : dispatch_bf16<false>(g, s);
+    }
     return g.swiglu ? dispatch_int4<true>(g, s) : dispatch_int4<false>(g, s);
 }
 

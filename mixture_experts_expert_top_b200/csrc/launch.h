@@ -36,7 +36,10 @@ cudaError_t launch_finalize(const uint16_t *y, const float *w, const int32_t *in
 
 // ---- gemm_sm100.cu
 struct GemmArgs {
-    const void *a;              // activations [P, K] bf16, permuted row order
+    const void *a;              // activations [P, K] bf16 in permuted row order, or, when perm is
+                                // given, hidden [T, K] with row r of the operand = a[perm[r] / top_k]
+    const int32_t *perm;        // optional [P]: gather the token operand through it
+    int T, top_k;               // rows of `a` and pairs per token (used with perm)
     const int32_t *offsets;     // [E+1]
     const void *w;              // weights (bf16 [E, rows, K] or int4 [E, rows, K/2])
     const uint16_t *w_scales;   // int4 only: [E, rows, K/128] bf16
@@ -49,6 +52,11 @@ struct GemmArgs {
     int *err;
 };
 cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t s);
+// True when the gate/up GEMM for this shape should read the token rows through
+// perm itself (few rows per expert) rather than from a gathered copy.
+bool gemm_gathers_in_kernel(int P, int E, int fmt);
+// ---- gemm_prefill_sm100.cu: bf16, tokens on the MMA's M side (many tokens per expert)
+cudaError_t launch_grouped_gemm_prefill(const GemmArgs &g, cudaStream_t s);
 cudaError_t launch_dequant_int4(const uint8_t *q, const uint16_t *scales, int rows, int K, uint16_t *out,
                                 cudaStream_t s);
 

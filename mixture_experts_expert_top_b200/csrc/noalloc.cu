@@ -20,7 +20,7 @@
 namespace {
 
 // Largest chunk histogram the array holds: nchunks * E int32 entries, where
-// nchunks = ceil(T*top_k / 8192). 65536 entries = 256 KiB.
+// nchunks = ceil(T*top_k / 2048) once T*top_k > 8192. 65536 entries = 256 KiB.
 constexpr int kScratchInts = 65536;
 constexpr int kMaxDevices = 64;
 

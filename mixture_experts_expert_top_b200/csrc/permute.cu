@@ -11,32 +11,36 @@
 // Deterministic: the rank of a pair inside its expert is computed from
 // per-warp histograms in pair order, never from the order of atomics.
 //
-// Layout of the work: a CTA of 1024 threads (32 warps) owns a chunk of up to
-// kChunk consecutive pairs; warp w owns a contiguous slice of the chunk and
-// walks it 32 pairs at a time, using __match_any_sync to rank equal experts
-// inside each step. One CTA does everything when P <= kChunk; otherwise
-// three kernels run: per-chunk histograms, one scan CTA, per-chunk scatter.
+// Layout of the work: a CTA owns a chunk of consecutive pairs; warp w owns a
+// contiguous slice of the chunk and walks it 32 pairs at a time, using
+// __match_any_sync to rank equal experts inside each step. One CTA of 1024
+// threads does everything when P <= kSingleMax; otherwise three kernels run:
+// per-chunk histograms (CTAs of 256 threads, kChunk pairs each), one scan CTA,
+// per-chunk scatter.
 #include "common.cuh"
 #include "launch.h"
 
 namespace moe {
 namespace {
 
-constexpr int kThreads = 1024;
-constexpr int kWarps = kThreads / 32;
-constexpr int kChunk = 8192;          // pairs per CTA
+constexpr int kThreads = 1024;        // single-CTA path and the scan CTA
+constexpr int kSingleMax = 8192;      // pairs handled by the single-CTA path
+constexpr int kChunkThreads = 256;    // multi-CTA path
+constexpr int kChunk = 2048;          // pairs per CTA on the multi-CTA path
 
-// Slice of the chunk owned by each warp: a multiple of 32 pairs.
+// Slice of the chunk owned by each of NW warps: a multiple of 32 pairs.
+template <int NW>
 __device__ __forceinline__ int warp_slice(int chunk_pairs) {
-    return ((chunk_pairs + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+    return ((chunk_pairs + NW * 32 - 1) / (NW * 32)) * 32;
 }
 
 // hist[w*E + e] = pairs of warp w's slice routed to expert e.
+template <int NW>
 __device__ void warp_histograms(const int32_t *__restrict__ ids, int begin, int n, int E, int *hist, int *err) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    for (int i = threadIdx.x; i < kWarps * E; i += kThreads) hist[i] = 0;
+    for (int i = threadIdx.x; i < NW * E; i += NW * 32) hist[i] = 0;
     __syncthreads();
-    const int slice = warp_slice(n);
+    const int slice = warp_slice<NW>(n);
     for (int it = 0; it < slice; it += 32) {
         const int local = w * slice + it + lane;
         const bool in = local < n;
@@ -50,11 +54,12 @@ __device__ void warp_histograms(const int32_t *__restrict__ ids, int begin, int 
     __syncthreads();
 }
 
-// In place: hist[w*E+e] <- base[e] + sum_{w'<w} hist[w'*E+e]; returns nothing.
+// In place: hist[w*E+e] <- base[e] + sum_{w'<w} hist[w'*E+e].
+template <int NW>
 __device__ void warp_bases(int E, int *hist, const int *base) {
-    for (int e = threadIdx.x; e < E; e += kThreads) {
+    for (int e = threadIdx.x; e < E; e += NW * 32) {
         int run = base[e];
-        for (int w = 0; w < kWarps; ++w) {
+        for (int w = 0; w < NW; ++w) {
             const int c = hist[w * E + e];
             hist[w * E + e] = run;
             run += c;
@@ -64,10 +69,11 @@ __device__ void warp_bases(int E, int *hist, const int *base) {
 }
 
 // Writes perm / inv_perm for the chunk, given per-warp starting rows.
+template <int NW>
 __device__ void warp_scatter(const int32_t *__restrict__ ids, int begin, int n, int E, int *hist,
                              int32_t *__restrict__ perm, int32_t *__restrict__ inv_perm) {
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const int slice = warp_slice(n);
+    const int slice = warp_slice<NW>(n);
     const unsigned lt = (1u << lane) - 1u;
     for (int it = 0; it < slice; it += 32) {
         const int local = w * slice + it + lane;
@@ -91,7 +97,7 @@ __device__ void warp_scatter(const int32_t *__restrict__ ids, int begin, int n, 
 // Exclusive scan of counts[0..E) into offsets[0..E], offsets[E] = total.
 // Also leaves offsets in shared memory `base`. E <= kThreads.
 __device__ void block_exclusive_scan(const int *vals, int E, int *base, int32_t *__restrict__ offsets) {
-    __shared__ int warp_sums[kWarps];
+    __shared__ int warp_sums[kThreads / 32];
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
     const int v = threadIdx.x < E ? vals[threadIdx.x] : 0;
     int x = v;
@@ -127,32 +133,34 @@ permute_single_kernel(const int32_t *__restrict__ ids, int P, int E, int32_t *__
                       int32_t *__restrict__ offsets, int32_t *__restrict__ perm, int32_t *__restrict__ inv_perm,
                       int *err) {
     extern __shared__ int smem[];
-    int *hist = smem;                 // [kWarps * E]
-    int *tot = hist + kWarps * E;     // [E]
+    constexpr int NW = kThreads / 32;
+    int *hist = smem;                 // [NW * E]
+    int *tot = hist + NW * E;         // [E]
     int *base = tot + E;              // [E]
-    warp_histograms(ids, 0, P, E, hist, err);
+    warp_histograms<NW>(ids, 0, P, E, hist, err);
     for (int e = threadIdx.x; e < E; e += kThreads) {
         int s = 0;
-        for (int w = 0; w < kWarps; ++w) s += hist[w * E + e];
+        for (int w = 0; w < NW; ++w) s += hist[w * E + e];
         tot[e] = s;
         counts[e] = s;
     }
     __syncthreads();
     block_exclusive_scan(tot, E, base, offsets);
-    warp_bases(E, hist, base);
-    warp_scatter(ids, 0, P, E, hist, perm, inv_perm);
+    warp_bases<NW>(E, hist, base);
+    warp_scatter<NW>(ids, 0, P, E, hist, perm, inv_perm);
 }
 
 // Multi-CTA pass 1: chunk_hist[c*E + e].
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kChunkThreads)
 permute_count_kernel(const int32_t *__restrict__ ids, int P, int E, int32_t *__restrict__ chunk_hist, int *err) {
+    constexpr int NW = kChunkThreads / 32;
     extern __shared__ int smem[];
     const int begin = blockIdx.x * kChunk;
     const int n = min(kChunk, P - begin);
-    warp_histograms(ids, begin, n, E, smem, err);
-    for (int e = threadIdx.x; e < E; e += kThreads) {
+    warp_histograms<NW>(ids, begin, n, E, smem, err);
+    for (int e = threadIdx.x; e < E; e += kChunkThreads) {
         int s = 0;
-        for (int w = 0; w < kWarps; ++w) s += smem[w * E + e];
+        for (int w = 0; w < NW; ++w) s += smem[w * E + e];
         chunk_hist[static_cast<size_t>(blockIdx.x) * E + e] = s;
     }
 }
@@ -182,18 +190,20 @@ permute_scan_kernel(int nchunks, int E, int32_t *__restrict__ chunk_hist, int32_
 }
 
 // Multi-CTA pass 3: scatter each chunk from its per-expert first rows.
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kChunkThreads)
 permute_scatter_kernel(const int32_t *__restrict__ ids, int P, int E, const int32_t *__restrict__ chunk_base,
                        int32_t *__restrict__ perm, int32_t *__restrict__ inv_perm) {
+    constexpr int NW = kChunkThreads / 32;
     extern __shared__ int smem[];
-    int *hist = smem;                 // [kWarps * E]
-    int *base = hist + kWarps * E;    // [E]
+    int *hist = smem;                 // [NW * E]
+    int *base = hist + NW * E;        // [E]
     const int begin = blockIdx.x * kChunk;
     const int n = min(kChunk, P - begin);
-    for (int e = threadIdx.x; e < E; e += kThreads) base[e] = chunk_base[static_cast<size_t>(blockIdx.x) * E + e];
-    warp_histograms(ids, begin, n, E, hist, nullptr);
-    warp_bases(E, hist, base);
-    warp_scatter(ids, begin, n, E, hist, perm, inv_perm);
+    for (int e = threadIdx.x; e < E; e += kChunkThreads)
+        base[e] = chunk_base[static_cast<size_t>(blockIdx.x) * E + e];
+    warp_histograms<NW>(ids, begin, n, E, hist, nullptr);
+    warp_bases<NW>(E, hist, base);
+    warp_scatter<NW>(ids, begin, n, E, hist, perm, inv_perm);
 }
 
 // hidden_perm[r] = hidden[perm[r] / k]: one warp per row, 16-byte vectors.
@@ -206,14 +216,17 @@ gather_rows_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__
         const int p = __ldg(perm + r);
         const uint4 *src = hidden + static_cast<size_t>(p / k) * vecs_per_row;
         uint4 *dst = out + static_cast<size_t>(r) * vecs_per_row;
-        for (int v = lane; v < vecs_per_row; v += 32) dst[v] = __ldg(src + v);
+        // the copy is written once and read once by the next kernel: stream it
+        // past L2 so that the k-times-reused hidden rows stay resident
+#pragma unroll 4
+        for (int v = lane; v < vecs_per_row; v += 32) __stcs(dst + v, __ldg(src + v));
     }
 }
 
 }  // namespace
 
 size_t permute_scratch_bytes(long long P, int E) {
-    if (P <= kChunk) return 0;
+    if (P <= kSingleMax) return 0;
     const long long nchunks = (P + kChunk - 1) / kChunk;
     return static_cast<size_t>(nchunks) * E * sizeof(int32_t);
 }
@@ -221,8 +234,8 @@ size_t permute_scratch_bytes(long long P, int E) {
 cudaError_t launch_permute(const int32_t *ids, int P, int E, int32_t *counts, int32_t *offsets, int32_t *perm,
                            int32_t *inv_perm, void *scratch, int *err, cudaStream_t s) {
     cudaError_t st;
-    if (P <= kChunk) {
-        const size_t sm = (static_cast<size_t>(kWarps) * E + 2 * E) * sizeof(int);
+    if (P <= kSingleMax) {
+        const size_t sm = (static_cast<size_t>(kThreads / 32) * E + 2 * E) * sizeof(int);
         st = cudaFuncSetAttribute(permute_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(sm));
         if (st != cudaSuccess) return st;
@@ -231,17 +244,17 @@ cudaError_t launch_permute(const int32_t *ids, int P, int E, int32_t *counts, in
     }
     const int nchunks = (P + kChunk - 1) / kChunk;
     int32_t *chunk_hist = static_cast<int32_t *>(scratch);
-    const size_t sm_hist = static_cast<size_t>(kWarps) * E * sizeof(int);
-    const size_t sm_scatter = (static_cast<size_t>(kWarps) * E + E) * sizeof(int);
+    const size_t sm_hist = static_cast<size_t>(kChunkThreads / 32) * E * sizeof(int);
+    const size_t sm_scatter = (static_cast<size_t>(kChunkThreads / 32) * E + E) * sizeof(int);
     st = cudaFuncSetAttribute(permute_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(sm_hist));
     if (st != cudaSuccess) return st;
     st = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(sm_scatter));
     if (st != cudaSuccess) return st;
-    permute_count_kernel<<<nchunks, kThreads, sm_hist, s>>>(ids, P, E, chunk_hist, err);
+    permute_count_kernel<<<nchunks, kChunkThreads, sm_hist, s>>>(ids, P, E, chunk_hist, err);
     permute_scan_kernel<<<1, kThreads, 2 * E * sizeof(int), s>>>(nchunks, E, chunk_hist, counts, offsets);
-    permute_scatter_kernel<<<nchunks, kThreads, sm_scatter, s>>>(ids, P, E, chunk_hist, perm, inv_perm);
+    permute_scatter_kernel<<<nchunks, kChunkThreads, sm_scatter, s>>>(ids, P, E, chunk_hist, perm, inv_perm);
     return cudaGetLastError();
 }
 

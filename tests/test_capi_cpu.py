@@ -72,10 +72,10 @@ def test_workspace_size_validates_the_shape(shape, ok):
 def test_workspace_grows_with_tokens():
     a = moe.moe_workspace_size(moe.Shape.of(64, 2048, 768, 128, 8))
     b = moe.moe_workspace_size(moe.Shape.of(128, 2048, 768, 128, 8))
-    assert b > a > 64 * 8 * (2048 * 2 * 2 + 768 * 2)
+    assert b > a > 64 * 8 * (2048 * 2 + 768 * 2)
     assert moe.moe_forward_host_workspace_size(moe.Shape.of(64, 2048, 768, 128, 8)) > a
     assert moe.moe_permute_workspace_size(moe.Shape.of(64, 2048, 768, 128, 8)) == 0
-    assert moe.moe_permute_workspace_size(moe.Shape.of(8192, 2048, 768, 128, 8)) == 8 * 128 * 4
+    assert moe.moe_permute_workspace_size(moe.Shape.of(8192, 2048, 768, 128, 8)) == 32 * 128 * 4
 
 
 def test_bad_arguments_are_rejected_before_any_launch():
@@ -86,8 +86,8 @@ def test_bad_arguments_are_rejected_before_any_launch():
     assert L.moe_route(None, byref(sh), None, None, None) == 1
     assert L.moe_finalize(None, None, None, byref(sh), None, None) == 1
     assert L.moe_forward(None, None, None, None, None, None, byref(sh), None, None, 0, None) == 1
-    # a fused gather in the gate/up GEMM is not offered
-    assert L.moe_grouped_gemm_swiglu(16, 16, 16, 16, None, byref(sh), 16, None) == 2
+    # misaligned perm for the fused gather
+    assert L.moe_grouped_gemm_swiglu(16, 18, 16, 16, None, byref(sh), 16, None) == 1
     # misaligned hidden
     assert L.moe_forward(17, 16, 16, None, 16, None, byref(sh), 16, 256, 1 << 30, None) == 1
     # scales given for bf16 weights

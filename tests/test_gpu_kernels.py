@@ -194,7 +194,9 @@ GEMM_CFGS = [
     moe_synth.get_config("qwen3_decode", T=200, E=16),                 # many rows per expert: several N blocks
     moe_synth.get_config("tiny", T=33, H=72, I=40, E=5, k=3),           # ragged H, I < 128
     moe_synth.get_config("skewed", T=96, H=256, I=192, E=16, k=3),      # uneven, empty experts
-    moe_synth.get_config("qwen3_prefill", T=700, H=512, I=256, E=8, k=2),  # BN = 128 path, ragged tail
+    moe_synth.get_config("qwen3_prefill", T=700, H=512, I=256, E=8, k=2),  # tokens-on-M kernel, ragged tail
+    moe_synth.get_config("qwen3_prefill", T=1024, H=512, I=384, E=8, k=2),  # CTA-pair kernel
+    moe_synth.get_config("qwen3_prefill", T=1100, H=264, I=200, E=4, k=2),  # CTA-pair, ragged H and I
 ]
 
 
@@ -224,6 +226,26 @@ def test_grouped_gemm_swiglu_and_down_match_oracle(cfg):
     torch.cuda.synchronize()
     gemm_rows_close(bf16_bits(act), r["act"], "act")
     gemm_rows_close(bf16_bits(y), r["y"], "y")
+
+
+@pytest.mark.parametrize("cfg", [GEMM_CFGS[1], GEMM_CFGS[2], GEMM_CFGS[3], GEMM_CFGS[5],
+                                 moe_synth.MoeConfig("int4_gather", T=48, H=1024, I=384, E=12, k=4, fmt="int4_g128")],
+                         ids=lambda c: f"T{c.T}H{c.H}I{c.I}E{c.E}k{c.k}{c.fmt}")
+def test_grouped_gemm_swiglu_gathers_through_perm(cfg):
+    """perm given: the GEMM reads hidden rows through perm (TMA gather4) and
+    must give the same act as from the materialised permuted rows."""
+    inp, r, hp = gemm_case(cfg)
+    sh = moe.Shape.of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.fmt)
+    offsets = dev(r["offsets"], torch.int32)
+    act_g = torch.empty(cfg.P, cfg.I, dtype=torch.bfloat16, device=DEV)
+    act_m = torch.empty(cfg.P, cfg.I, dtype=torch.bfloat16, device=DEV)
+    moe.moe_grouped_gemm_swiglu(dev(inp["hidden"]), dev(r["perm"], torch.int32), offsets, wdev(inp, "w_gu"),
+                                wdev(inp, "w_gu_scales"), sh, act_g)
+    moe.moe_grouped_gemm_swiglu(dev(bits_to_bf16(hp)), None, offsets, wdev(inp, "w_gu"), wdev(inp, "w_gu_scales"),
+                                sh, act_m)
+    torch.cuda.synchronize()
+    assert torch.equal(act_g.view(torch.int16), act_m.view(torch.int16))
+    gemm_rows_close(bf16_bits(act_g), r["act"], "act (gathered)")
 
 
 def test_grouped_gemm_int4_matches_oracle():

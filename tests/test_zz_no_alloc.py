@@ -62,7 +62,7 @@ def test_noalloc_permute_matches_permute_on_two_calls_in_a_row(T, E, k, H):
 
 
 def test_noalloc_permute_rejects_calls_beyond_its_scratch():
-    # ceil(600000 / 8192) = 74 chunks x 1024 experts > 65536 entries
+    # ceil(600000 / 2048) = 293 chunks x 1024 experts > 65536 entries
     shape = moe.Shape.of(600000, 8, 8, 1024, 1)
     one = torch.zeros(4, dtype=torch.int32, device=DEV)
     status = moe.lib().moe_permute_noalloc(one.data_ptr(), moe.ctypes.byref(shape), one.data_ptr(), one.data_ptr(),
