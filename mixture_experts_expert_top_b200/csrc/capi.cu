@@ -130,10 +130,15 @@ moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const
     auto *act = reinterpret_cast<uint16_t *>(ws + L.act);
     auto *y = reinterpret_cast<uint16_t *>(ws + L.y);
     cudaError_t e;
-    if ((e = moe::launch_route(logits, T, E, k, ids, w, st)) != cudaSuccess) return cuda_status(e);
-    if ((e = moe::launch_permute(ids, P, E, counts, offsets, perm, inv, ws + L.scratch, error_flag_ptr(), st)) !=
-        cudaSuccess)
-        return cuda_status(e);
+    if (moe::route_permute_fusable(T, E, k)) {
+        e = moe::launch_route_permute(logits, T, E, k, ids, w, counts, offsets, perm, inv, error_flag_ptr(), st);
+        if (e != cudaSuccess) return cuda_status(e);
+    } else {
+        if ((e = moe::launch_route(logits, T, E, k, ids, w, st)) != cudaSuccess) return cuda_status(e);
+        if ((e = moe::launch_permute(ids, P, E, counts, offsets, perm, inv, ws + L.scratch, error_flag_ptr(), st)) !=
+            cudaSuccess)
+            return cuda_status(e);
+    }
     // Few rows per expert: the gate/up GEMM gathers the token rows itself (TMA
     // gather4 through perm). Many rows per expert: one gather kernel writes the
     // permuted rows and the GEMM reads them as whole 128-row tiles, which keeps

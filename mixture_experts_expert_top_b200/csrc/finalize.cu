@@ -14,6 +14,7 @@
 // y row it touches. HBM-bound: (k*H + H)*2 bytes + k*(4+4) bytes per token.
 #include "common.cuh"
 #include "launch.h"
+#include "launch_util.cuh"
 
 namespace moe {
 namespace {
@@ -30,6 +31,7 @@ template <int KT>
 __global__ void __launch_bounds__(256)
 finalize_kernel(const uint4 *__restrict__ y, const float *__restrict__ w, const int32_t *__restrict__ inv_perm,
                 int T, int vecs_per_row, int k_rt, int P, uint4 *__restrict__ out) {
+    griddep_wait();     // no early trigger: the next kernel's CTAs would share SMs with this one
     const int k = KT > 0 ? KT : k_rt;
     const long long total = static_cast<long long>(T) * vecs_per_row;
     for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
@@ -83,10 +85,10 @@ finalize_kernel(const uint4 *__restrict__ y, const float *__restrict__ w, const 
 }
 
 template <int KT>
-void launch_finalize_t(int blocks, cudaStream_t s, const uint16_t *y, const float *w, const int32_t *inv_perm, int T,
-                       int vpr, int k, int P, uint16_t *out) {
-    finalize_kernel<KT><<<blocks, 256, 0, s>>>(reinterpret_cast<const uint4 *>(y), w, inv_perm, T, vpr, k, P,
-                                               reinterpret_cast<uint4 *>(out));
+cudaError_t launch_finalize_t(int blocks, cudaStream_t s, const uint16_t *y, const float *w, const int32_t *inv_perm,
+                              int T, int vpr, int k, int P, uint16_t *out) {
+    return launch_pdl(finalize_kernel<KT>, dim3(blocks), dim3(256), 0, s, reinterpret_cast<const uint4 *>(y), w,
+                      inv_perm, T, vpr, k, P, reinterpret_cast<uint4 *>(out));
 }
 
 }  // namespace
@@ -100,14 +102,13 @@ cudaError_t launch_finalize(const uint16_t *y, const float *w, const int32_t *in
     if (blocks > 148LL * 32) blocks = 148LL * 32;
     const int b = static_cast<int>(blocks);
     switch (k) {
-        case 1: launch_finalize_t<1>(b, s, y, w, inv_perm, T, vpr, k, T * k, out); break;
-        case 2: launch_finalize_t<2>(b, s, y, w, inv_perm, T, vpr, k, T * k, out); break;
-        case 4: launch_finalize_t<4>(b, s, y, w, inv_perm, T, vpr, k, T * k, out); break;
-        case 6: launch_finalize_t<6>(b, s, y, w, inv_perm, T, vpr, k, T * k, out); break;
-        case 8: launch_finalize_t<8>(b, s, y, w, inv_perm, T, vpr, k, T * k, out); break;
-        default: launch_finalize_t<0>(b, s, y, w, inv_perm, T, vpr, k, T * k, out); break;
+        case 1: return launch_finalize_t<1>(b, s, y, w, inv_perm, T, vpr, k, T * k, out);
+        case 2: return launch_finalize_t<2>(b, s, y, w, inv_perm, T, vpr, k, T * k, out);
+        case 4: return launch_finalize_t<4>(b, s, y, w, inv_perm, T, vpr, k, T * k, out);
+        case 6: return launch_finalize_t<6>(b, s, y, w, inv_perm, T, vpr, k, T * k, out);
+        case 8: return launch_finalize_t<8>(b, s, y, w, inv_perm, T, vpr, k, T * k, out);
+        default: return launch_finalize_t<0>(b, s, y, w, inv_perm, T, vpr, k, T * k, out);
     }
-    return cudaGetLastError();
 }
 
 }  // namespace moe

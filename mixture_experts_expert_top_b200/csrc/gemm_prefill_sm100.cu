@@ -18,6 +18,7 @@
 // Warp roles as in gemm_sm100.cu: warp 0 TMA, warp 1 MMA + TMEM owner,
 // warps 2-5 epilogue over a double-buffered 2 x 256-column accumulator.
 #include "gemm_common.cuh"
+#include "launch_util.cuh"
 
 namespace moe {
 namespace {
@@ -139,6 +140,8 @@ grouped_gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
         tmem_relinquish();
     }
     // tiles of expert e: ceil(rows / 128) token blocks x NB feature blocks
+    // barriers, tensor maps and TMEM are set up while the previous kernel drains
+    griddep_wait();
     build_tile_prefix<192>(p.offsets, E, NB, kTokM, off_s, pre_s);
     tc_fence_before_sync();
     __syncthreads();
@@ -242,6 +245,8 @@ grouped_gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
         }
     }
 
+    // every role is done: the next kernel may start its set-up now
+    griddep_launch_dependents();
     __syncthreads();
     if (*abort_flag) {
         for (int i = 0; i < 1000; ++i) __nanosleep(1000);
@@ -319,6 +324,8 @@ grouped_gemm_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmA, const 
         tmem_alloc_pair(tmem_holder, 2 * kAccCols);
         tmem_relinquish_pair();
     }
+    // barriers, tensor maps and TMEM are set up while the previous kernel drains
+    griddep_wait();
     build_tile_prefix<192>(p.offsets, E, NB, kPairRows, off_s, pre_s);
     tc_fence_before_sync();
     __syncthreads();
@@ -415,6 +422,8 @@ grouped_gemm_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmA, const 
         }
     }
 
+    // every role is done: the next kernel may start its set-up now
+    griddep_launch_dependents();
     __syncthreads();
     if (*abort_flag) {
         for (int i = 0; i < 1000; ++i) __nanosleep(1000);
@@ -445,8 +454,7 @@ cudaError_t run_prefill_pair(const GemmArgs &g, cudaStream_t s) {
     const int pairs = static_cast<int>(std::min<long long>(num_sms() / 2, max_tiles));
     if (pairs <= 0) return cudaSuccess;
     Params p = make_params(g, kPairRows);
-    kern<<<2 * pairs, 192, C::kSmemBytes, s>>>(ta, tb, p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(2 * pairs), dim3(192), C::kSmemBytes, s, ta, tb, p);
 }
 
 template <bool SWIGLU>
@@ -468,8 +476,7 @@ cudaError_t run_prefill(const GemmArgs &g, cudaStream_t s) {
     const int grid = static_cast<int>(std::min<long long>(num_sms(), max_tiles));
     if (grid <= 0) return cudaSuccess;
     Params p = make_params(g, kTokM);
-    kern<<<grid, 192, C::kSmemBytes, s>>>(ta, tb, p);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(192), C::kSmemBytes, s, ta, tb, p);
 }
 
 }  // namespace

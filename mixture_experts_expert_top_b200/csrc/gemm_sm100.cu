@@ -32,6 +32,7 @@
 //  - Every wait is bounded (see mbar_wait); a timeout raises the device flag
 //    and unwinds the CTA.
 #include "gemm_common.cuh"
+#include "launch_util.cuh"
 
 namespace moe {
 namespace {
@@ -137,6 +138,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         tmem_alloc(tmem_holder, C::kTmemCols);
         tmem_relinquish();
     }
+    // barriers, tensor maps and TMEM are set up while the previous kernel drains
+    griddep_wait();
     build_tile_prefix<C::kThreads>(p.offsets, E, MB, BN, off_s, pre_s);
     tc_fence_before_sync();
     __syncthreads();
@@ -233,6 +236,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                                               abort_flag, 128);
     }
 
+    // every role is done: the next kernel may start its set-up now
+    griddep_launch_dependents();
     __syncthreads();
     if (*abort_flag) {
         // let copies already in flight land before the CTA's memory is reused
@@ -324,6 +329,8 @@ grouped_gemm_int4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
         tmem_alloc(tmem_holder, C::kTmemCols);
         tmem_relinquish();
     }
+    // barriers, tensor maps and TMEM are set up while the previous kernel drains
+    griddep_wait();
     build_tile_prefix<C::kThreads>(p.offsets, E, MB, BN, off_s, pre_s);
     tc_fence_before_sync();
     __syncthreads();
@@ -509,6 +516,8 @@ grouped_gemm_int4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
         }
     }
 
+    // every role is done: the next kernel may start its set-up now
+    griddep_launch_dependents();
     __syncthreads();
     if (*abort_flag) {
         for (int i = 0; i < 1000; ++i) __nanosleep(1000);
@@ -535,8 +544,7 @@ cudaError_t run_bf16(const GemmArgs &g, cudaStream_t s) {
     if (st != cudaSuccess) return st;
     const int grid = grid_for(g, BN);
     if (grid <= 0) return cudaSuccess;
-    kern<<<grid, C::kThreads, C::kSmemBytes, s>>>(ta, tb, make_params(g, BN));
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(C::kThreads), C::kSmemBytes, s, ta, tb, make_params(g, BN));
 }
 
 template <int BN, int STAGES, bool SWIGLU>
@@ -554,8 +562,7 @@ cudaError_t run_int4(const GemmArgs &g, cudaStream_t s) {
     if (st != cudaSuccess) return st;
     const int grid = grid_for(g, BN);
     if (grid <= 0) return cudaSuccess;
-    kern<<<grid, C::kThreads, C::kSmemBytes, s>>>(ta, tb, make_params(g, BN));
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3(grid), dim3(C::kThreads), C::kSmemBytes, s, ta, tb, make_params(g, BN));
 }
 
 template <bool SWIGLU>
@@ -587,6 +594,7 @@ cudaError_t dispatch_int4(const GemmArgs &g, cudaStream_t s) {
 // Standalone W4A16 decoding: the same dequant_word as the GEMMs' decode warps.
 __global__ void dequant_int4_kernel(const uint4 *__restrict__ q, const uint16_t *__restrict__ scales, int rows,
                                     int K, uint4 *__restrict__ out) {
+    griddep_wait();
     const long long chunks_per_row = K / 32;   // 16 packed bytes = 32 values
     const long long total = static_cast<long long>(rows) * chunks_per_row;
     for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
@@ -627,9 +635,8 @@ cudaError_t launch_dequant_int4(const uint8_t *q, const uint16_t *scales, int ro
     const long long total = static_cast<long long>(rows) * (K / 32);
     long long blocks = (total + 255) / 256;
     if (blocks > 148LL * 16) blocks = 148LL * 16;
-    dequant_int4_kernel<<<static_cast<int>(blocks), 256, 0, s>>>(reinterpret_cast<const uint4 *>(q), scales, rows,
-                                                                  K, reinterpret_cast<uint4 *>(out));
-    return cudaGetLastError();
+    return launch_pdl(dequant_int4_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0, s,
+                      reinterpret_cast<const uint4 *>(q), scales, rows, K, reinterpret_cast<uint4 *>(out));
 }
 
 }  // namespace moe

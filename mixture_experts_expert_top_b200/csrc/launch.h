@@ -21,6 +21,13 @@ int *device_error_flag();
 // ---- route.cu
 cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s);
 
+// ---- route_permute.cu
+// Routing and bucketing of a small batch by one CTA (same outputs as
+// launch_route followed by launch_permute).
+bool route_permute_fusable(int T, int E, int k);
+cudaError_t launch_route_permute(const float *logits, int T, int E, int k, int32_t *ids, float *w, int32_t *counts,
+                                 int32_t *offsets, int32_t *perm, int32_t *inv_perm, int *err, cudaStream_t s);
+
 // ---- permute.cu
 // Scratch bytes the permute needs for P pairs over E experts (0 when a
 // single CTA handles all pairs).

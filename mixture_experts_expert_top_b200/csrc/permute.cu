@@ -17,8 +17,10 @@
 // threads does everything when P <= kSingleMax; otherwise three kernels run:
 // per-chunk histograms (CTAs of 256 threads, kChunk pairs each), one scan CTA,
 // per-chunk scatter.
+#include "bucket_dev.cuh"
 #include "common.cuh"
 #include "launch.h"
+#include "launch_util.cuh"
 
 namespace moe {
 namespace {
@@ -28,126 +30,15 @@ constexpr int kSingleMax = 8192;      // pairs handled by the single-CTA path
 constexpr int kChunkThreads = 256;    // multi-CTA path
 constexpr int kChunk = 2048;          // pairs per CTA on the multi-CTA path
 
-// Slice of the chunk owned by each of NW warps: a multiple of 32 pairs.
-template <int NW>
-__device__ __forceinline__ int warp_slice(int chunk_pairs) {
-    return ((chunk_pairs + NW * 32 - 1) / (NW * 32)) * 32;
-}
-
-// hist[w*E + e] = pairs of warp w's slice routed to expert e.
-template <int NW>
-__device__ void warp_histograms(const int32_t *__restrict__ ids, int begin, int n, int E, int *hist, int *err) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    for (int i = threadIdx.x; i < NW * E; i += NW * 32) hist[i] = 0;
-    __syncthreads();
-    const int slice = warp_slice<NW>(n);
-    for (int it = 0; it < slice; it += 32) {
-        const int local = w * slice + it + lane;
-        const bool in = local < n;
-        const int e = in ? __ldg(ids + begin + local) : -1;
-        const bool ok = in && e >= 0 && e < E;
-        if (in && !ok) raise_error(err, kErrBadExpertId);
-        const unsigned m = __match_any_sync(0xffffffffu, ok ? e : -1);
-        if (ok && lane == __ffs(m) - 1) hist[w * E + e] += __popc(m);
-        __syncwarp();
-    }
-    __syncthreads();
-}
-
-// In place: hist[w*E+e] <- base[e] + sum_{w'<w} hist[w'*E+e].
-template <int NW>
-__device__ void warp_bases(int E, int *hist, const int *base) {
-    for (int e = threadIdx.x; e < E; e += NW * 32) {
-        int run = base[e];
-        for (int w = 0; w < NW; ++w) {
-            const int c = hist[w * E + e];
-            hist[w * E + e] = run;
-            run += c;
-        }
-    }
-    __syncthreads();
-}
-
-// Writes perm / inv_perm for the chunk, given per-warp starting rows.
-template <int NW>
-__device__ void warp_scatter(const int32_t *__restrict__ ids, int begin, int n, int E, int *hist,
-                             int32_t *__restrict__ perm, int32_t *__restrict__ inv_perm) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const int slice = warp_slice<NW>(n);
-    const unsigned lt = (1u << lane) - 1u;
-    for (int it = 0; it < slice; it += 32) {
-        const int local = w * slice + it + lane;
-        const bool in = local < n;
-        const int e = in ? __ldg(ids + begin + local) : -1;
-        const bool ok = in && e >= 0 && e < E;
-        const unsigned m = __match_any_sync(0xffffffffu, ok ? e : -1);
-        if (ok) {
-            const int r = hist[w * E + e] + __popc(m & lt);
-            perm[r] = begin + local;
-            inv_perm[begin + local] = r;
-        } else if (in) {
-            inv_perm[begin + local] = -1;
-        }
-        __syncwarp();
-        if (ok && lane == __ffs(m) - 1) hist[w * E + e] += __popc(m);
-        __syncwarp();
-    }
-}
-
-// Exclusive scan of counts[0..E) into offsets[0..E], offsets[E] = total.
-// Also leaves offsets in shared memory `base`. E <= kThreads.
-__device__ void block_exclusive_scan(const int *vals, int E, int *base, int32_t *__restrict__ offsets) {
-    __shared__ int warp_sums[kThreads / 32];
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    const int v = threadIdx.x < E ? vals[threadIdx.x] : 0;
-    int x = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) warp_sums[w] = x;
-    __syncthreads();
-    if (w == 0) {
-        int s = warp_sums[lane];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, s, o);
-            if (lane >= o) s += y;
-        }
-        warp_sums[lane] = s;   // inclusive over warps
-    }
-    __syncthreads();
-    const int excl = x - v + (w > 0 ? warp_sums[w - 1] : 0);
-    if (threadIdx.x < E) {
-        base[threadIdx.x] = excl;
-        offsets[threadIdx.x] = excl;
-    }
-    if (threadIdx.x == E - 1) offsets[E] = excl + v;
-    __syncthreads();
-}
-
 // All pairs in one CTA.
 __global__ void __launch_bounds__(kThreads, 1)
 permute_single_kernel(const int32_t *__restrict__ ids, int P, int E, int32_t *__restrict__ counts,
                       int32_t *__restrict__ offsets, int32_t *__restrict__ perm, int32_t *__restrict__ inv_perm,
                       int *err) {
     extern __shared__ int smem[];
-    constexpr int NW = kThreads / 32;
-    int *hist = smem;                 // [NW * E]
-    int *tot = hist + NW * E;         // [E]
-    int *base = tot + E;              // [E]
-    warp_histograms<NW>(ids, 0, P, E, hist, err);
-    for (int e = threadIdx.x; e < E; e += kThreads) {
-        int s = 0;
-        for (int w = 0; w < NW; ++w) s += hist[w * E + e];
-        tot[e] = s;
-        counts[e] = s;
-    }
-    __syncthreads();
-    block_exclusive_scan(tot, E, base, offsets);
-    warp_bases<NW>(E, hist, base);
-    warp_scatter<NW>(ids, 0, P, E, hist, perm, inv_perm);
+    griddep_launch_dependents();
+    griddep_wait();
+    bucket_single_cta<kThreads>(ids, P, E, counts, offsets, perm, inv_perm, smem, err);
 }
 
 // Multi-CTA pass 1: chunk_hist[c*E + e].
@@ -155,6 +46,8 @@ __global__ void __launch_bounds__(kChunkThreads)
 permute_count_kernel(const int32_t *__restrict__ ids, int P, int E, int32_t *__restrict__ chunk_hist, int *err) {
     constexpr int NW = kChunkThreads / 32;
     extern __shared__ int smem[];
+    griddep_launch_dependents();
+    griddep_wait();
     const int begin = blockIdx.x * kChunk;
     const int n = min(kChunk, P - begin);
     warp_histograms<NW>(ids, begin, n, E, smem, err);
@@ -171,6 +64,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 permute_scan_kernel(int nchunks, int E, int32_t *__restrict__ chunk_hist, int32_t *__restrict__ counts,
                     int32_t *__restrict__ offsets) {
     extern __shared__ int smem[];
+    griddep_launch_dependents();
+    griddep_wait();
     int *tot = smem;        // [E]
     int *base = tot + E;    // [E]
     for (int e = threadIdx.x; e < E; e += kThreads) {
@@ -184,7 +79,7 @@ permute_scan_kernel(int nchunks, int E, int32_t *__restrict__ chunk_hist, int32_
         counts[e] = run;
     }
     __syncthreads();
-    block_exclusive_scan(tot, E, base, offsets);
+    block_exclusive_scan<kThreads>(tot, E, base, offsets);
     for (int e = threadIdx.x; e < E; e += kThreads)
         for (int c = 0; c < nchunks; ++c) chunk_hist[static_cast<size_t>(c) * E + e] += base[e];
 }
@@ -197,6 +92,8 @@ permute_scatter_kernel(const int32_t *__restrict__ ids, int P, int E, const int3
     extern __shared__ int smem[];
     int *hist = smem;                 // [NW * E]
     int *base = hist + NW * E;        // [E]
+    griddep_launch_dependents();
+    griddep_wait();
     const int begin = blockIdx.x * kChunk;
     const int n = min(kChunk, P - begin);
     for (int e = threadIdx.x; e < E; e += kChunkThreads)
@@ -210,6 +107,8 @@ permute_scatter_kernel(const int32_t *__restrict__ ids, int P, int E, const int3
 __global__ void __launch_bounds__(256)
 gather_rows_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ perm, int P, int vecs_per_row,
                    int k, uint4 *__restrict__ out) {
+    griddep_launch_dependents();
+    griddep_wait();
     const int lane = threadIdx.x & 31;
     const int warps = gridDim.x * (blockDim.x >> 5);
     for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < P; r += warps) {
@@ -239,8 +138,8 @@ cudaError_t launch_permute(const int32_t *ids, int P, int E, int32_t *counts, in
         st = cudaFuncSetAttribute(permute_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   static_cast<int>(sm));
         if (st != cudaSuccess) return st;
-        permute_single_kernel<<<1, kThreads, sm, s>>>(ids, P, E, counts, offsets, perm, inv_perm, err);
-        return cudaGetLastError();
+        return launch_pdl(permute_single_kernel, dim3(1), dim3(kThreads), sm, s, ids, P, E, counts, offsets, perm,
+                          inv_perm, err);
     }
     const int nchunks = (P + kChunk - 1) / kChunk;
     int32_t *chunk_hist = static_cast<int32_t *>(scratch);
@@ -252,10 +151,14 @@ cudaError_t launch_permute(const int32_t *ids, int P, int E, int32_t *counts, in
     st = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               static_cast<int>(sm_scatter));
     if (st != cudaSuccess) return st;
-    permute_count_kernel<<<nchunks, kChunkThreads, sm_hist, s>>>(ids, P, E, chunk_hist, err);
-    permute_scan_kernel<<<1, kThreads, 2 * E * sizeof(int), s>>>(nchunks, E, chunk_hist, counts, offsets);
-    permute_scatter_kernel<<<nchunks, kChunkThreads, sm_scatter, s>>>(ids, P, E, chunk_hist, perm, inv_perm);
-    return cudaGetLastError();
+    if ((st = launch_pdl(permute_count_kernel, dim3(nchunks), dim3(kChunkThreads), sm_hist, s, ids, P, E, chunk_hist,
+                         err)) != cudaSuccess)
+        return st;
+    if ((st = launch_pdl(permute_scan_kernel, dim3(1), dim3(kThreads), 2 * E * sizeof(int), s, nchunks, E,
+                         chunk_hist, counts, offsets)) != cudaSuccess)
+        return st;
+    return launch_pdl(permute_scatter_kernel, dim3(nchunks), dim3(kChunkThreads), sm_scatter, s, ids, P, E,
+                      static_cast<const int32_t *>(chunk_hist), perm, inv_perm);
 }
 
 cudaError_t launch_gather(const uint16_t *hidden, const int32_t *perm, int P, int H, int k, uint16_t *hidden_perm,
@@ -264,9 +167,8 @@ cudaError_t launch_gather(const uint16_t *hidden, const int32_t *perm, int P, in
     const int rows_per_block = 8;
     int blocks = (P + rows_per_block - 1) / rows_per_block;
     if (blocks > 148 * 16) blocks = 148 * 16;
-    gather_rows_kernel<<<blocks, 32 * rows_per_block, 0, s>>>(reinterpret_cast<const uint4 *>(hidden), perm, P,
-                                                              H / 8, k, reinterpret_cast<uint4 *>(hidden_perm));
-    return cudaGetLastError();
+    return launch_pdl(gather_rows_kernel, dim3(blocks), dim3(32 * rows_per_block), 0, s,
+                      reinterpret_cast<const uint4 *>(hidden), perm, P, H / 8, k, reinterpret_cast<uint4 *>(hidden_perm));
 }
 
 }  // namespace moe
