@@ -16,53 +16,57 @@
 
 namespace moe {
 
+// Order-preserving map of a logit onto uint32: larger logit, larger key.
+// NaN counts as -inf and -0 as +0 (so that +0 and -0 tie, as they compare
+// equal in fp32). Key 0 is below every logit and marks "not a candidate".
+__device__ __forceinline__ uint32_t logit_key(float x) {
+    if (x != x) x = -INFINITY;
+    if (x == 0.f) x = 0.f;
+    const uint32_t b = __float_as_uint(x);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_logit(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 // Lane j of the warp ends with slot j's expert id and weight (j < k <= 32).
-// Logits are read with plain loads; NaN reads as -inf.
+// Expert e sits in lane e % 32, register e / 32. Each of the k rounds takes
+// two warp reductions: the largest key left, then the lowest expert id that
+// holds it; the winner's key is cleared.
 template <int PER_LANE>
 __device__ __forceinline__ void route_token(const float *row, int E, int k, int &my_id, float &my_w) {
     const int lane = threadIdx.x & 31;
-    float v[PER_LANE];
+    uint32_t key[PER_LANE];
 #pragma unroll
     for (int i = 0; i < PER_LANE; ++i) {
         const int e = lane + 32 * i;
-        const float x = e < E ? row[e] : -INFINITY;
-        v[i] = (x != x) ? -INFINITY : x;
+        key[i] = e < E ? logit_key(row[e]) : 0u;
     }
-    uint32_t taken = 0;                   // bit i: expert lane + 32 i already chosen
-#pragma unroll
-    for (int i = 0; i < PER_LANE; ++i)
-        if (lane + 32 * i >= E) taken |= 1u << i;
-
     my_id = 0;
-    float my_logit = 0.f;
+    uint32_t my_key = 0;
     for (int j = 0; j < k; ++j) {
-        float best = -INFINITY;
-        int bid = 0x7fffffff;
+        uint32_t local = 0;
 #pragma unroll
-        for (int i = 0; i < PER_LANE; ++i) {
-            const int e = lane + 32 * i;
-            if (!((taken >> i) & 1u) && (v[i] > best || (v[i] == best && e < bid))) {
-                best = v[i];
-                bid = e;
-            }
-        }
+        for (int i = 0; i < PER_LANE; ++i) local = max(local, key[i]);
+        const uint32_t best = __reduce_max_sync(0xffffffffu, local);
+        uint32_t cand = 0xffffffffu;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const float ob = __shfl_xor_sync(0xffffffffu, best, o);
-            const int oi = __shfl_xor_sync(0xffffffffu, bid, o);
-            if (ob > best || (ob == best && oi < bid)) {
-                best = ob;
-                bid = oi;
-            }
+        for (int i = PER_LANE - 1; i >= 0; --i)
+            if (key[i] == best) cand = static_cast<uint32_t>(lane + 32 * i);
+        const int bid = static_cast<int>(__reduce_min_sync(0xffffffffu, cand));
+        if ((bid & 31) == lane) {
+#pragma unroll
+            for (int i = 0; i < PER_LANE; ++i)
+                if (i == (bid >> 5)) key[i] = 0u;
         }
-        if ((bid & 31) == lane) taken |= 1u << (bid >> 5);
         if (lane == j) {
             my_id = bid;
-            my_logit = best;
+            my_key = best;
         }
     }
-    const float l0 = __shfl_sync(0xffffffffu, my_logit, 0);
-    const float ej = lane < k ? expf(my_logit - l0) : 0.f;
+    const float l0 = key_logit(__shfl_sync(0xffffffffu, my_key, 0));
+    const float ej = lane < k ? expf(key_logit(my_key) - l0) : 0.f;
     float sum = 0.f;
     for (int j = 0; j < k; ++j) sum += __shfl_sync(0xffffffffu, ej, j);   // slot order
     my_w = __fdiv_rn(ej, sum);

@@ -91,15 +91,20 @@ def test_route_matches_oracle(T, E, k, name):
 
 
 def test_route_ties_go_to_the_lower_expert():
-    logits = torch.zeros(6, 16)
+    logits = torch.zeros(8, 16)
     logits[1, 3] = logits[1, 9] = 1.0
     logits[2] = torch.arange(16) % 4 * 0.5
     logits[3, :] = -3.0
     logits[4, 15] = 5.0
+    logits[6, :] = -1.0                       # -0 and +0 compare equal: the lower id goes first
+    logits[6, 2], logits[6, 7] = -0.0, 0.0
+    logits[7, :] = -1.0
+    logits[7, 2], logits[7, 7] = 0.0, -0.0
     gi, gw = run_route(logits, 4)
     oi, ow = oracle.route(logits, 4)
     assert np.array_equal(gi, oi)
     assert np.array_equal(gi[3], [0, 1, 2, 3]) and np.all(gw[3] == 0.25)
+    assert np.array_equal(gi[6][:2], [2, 7]) and np.array_equal(gi[7][:2], [2, 7])
 
 
 # ---------------------------------------------------------------- permute --
