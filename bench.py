@@ -42,8 +42,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NORTH_STAR_HBM_GBS = 8000.0       # the roofline literals the layer's target is stated against
 NORTH_STAR_BF16_TFLOPS = 2250.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
+# the grouped-GEMM kernels' sources: a change to any of them invalidates stored counters
 KERNEL_SOURCES = ["mixture_experts_expert_top_b200/csrc/gemm_sm100.cu",
-                  "mixture_experts_expert_top_b200/csrc/common.cuh"]
+                  "mixture_experts_expert_top_b200/csrc/gemm_prefill_sm100.cu",
+                  "mixture_experts_expert_top_b200/csrc/gemm_common.cuh",
+                  "mixture_experts_expert_top_b200/csrc/common.cuh",
+                  "mixture_experts_expert_top_b200/csrc/launch_util.cuh"]
 
 
 # ----------------------------------------------------------------- helpers --

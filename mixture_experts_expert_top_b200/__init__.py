@@ -60,9 +60,14 @@ _lib: Optional[ctypes.CDLL] = None
 def lib() -> ctypes.CDLL:
     global _lib
     if _lib is None:
-        if not os.path.exists(library_path):
-            raise RuntimeError(f"{library_path} is missing: build it with "
-                               "`python -m mixture_experts_expert_top_b200.build` (needs nvcc)")
+        from . import build as _build
+        if not _build.up_to_date():
+            # a missing or stale library is rebuilt from the sources (needs nvcc); never skipped
+            try:
+                _build.build()
+            except Exception as e:      # noqa: BLE001 - re-raised with the path
+                raise RuntimeError(f"{library_path} is missing or older than its sources and could not be "
+                                   f"built ({e}): build it with `python -m mixture_experts_expert_top_b200.build`")
         L = ctypes.CDLL(library_path)
         vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
         sp = ctypes.POINTER(Shape)

@@ -18,7 +18,7 @@ namespace moe {
 namespace {
 
 constexpr int kThreads = 1024;
-constexpr int kMaxTokens = 256;     // at most 8 tokens per warp
+constexpr int kMaxTokens = 64;      // at most 2 tokens per warp: each token is latency-bound
 constexpr int kMaxPairs = 8192;
 constexpr int kMaxExperts = 256;    // at most 8 logits per lane
 
