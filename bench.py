@@ -338,7 +338,8 @@ def run_ours(args, rank, world, local):
             c()
             ev[r][i + 1].record(stream)
     torch.cuda.synchronize()
-    stage_ms = {s: sum(ev[r][i].elapsed_time(ev[r][i + 1]) for r in range(n_rep)) / n_rep
+    # median over repetitions: robust to the odd slow repetition (a clock dip)
+    stage_ms = {s: statistics.median(ev[r][i].elapsed_time(ev[r][i + 1]) for r in range(n_rep))
                 for i, s in enumerate(stages)}
     counts_h = counts.cpu().numpy()
     work = work_per_step(cfg, counts_h)
