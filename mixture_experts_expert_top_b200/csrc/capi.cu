@@ -144,16 +144,20 @@ moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const
     // permuted rows and the GEMM reads them as whole 128-row tiles, which keeps
     // its TMA unit from turning into the bottleneck.
     if (moe::gemm_gathers_in_kernel(P, E, s->fmt)) {
-        e = moe::launch_grouped_gemm(gemm_args(s, hidden, perm, offsets, w_gu, w_gu_scales, true, act), st);
+        moe::GemmArgs gu = gemm_args(s, hidden, perm, offsets, w_gu, w_gu_scales, true, act);
+        gu.hints = moe::kGemmHintPrefetchGuess;     // routing runs on few SMs: warm L2 meanwhile
+        e = moe::launch_grouped_gemm(gu, st);
     } else {
         auto *hperm = reinterpret_cast<uint16_t *>(ws + L.hperm);
         if ((e = moe::launch_gather(hidden, perm, P, H, k, hperm, st)) != cudaSuccess) return cuda_status(e);
         e = moe::launch_grouped_gemm(gemm_args(s, hperm, nullptr, offsets, w_gu, w_gu_scales, true, act), st);
     }
     if (e != cudaSuccess) return cuda_status(e);
-    if ((e = moe::launch_grouped_gemm(gemm_args(s, act, nullptr, offsets, w_d, w_d_scales, false, y), st)) !=
-        cudaSuccess)
-        return cuda_status(e);
+    // offsets were complete before the gate/up GEMM started, so the down GEMM
+    // may start loading weights while gate/up finishes
+    moe::GemmArgs dn = gemm_args(s, act, nullptr, offsets, w_d, w_d_scales, false, y);
+    dn.hints = moe::kGemmHintOffsetsReady;
+    if ((e = moe::launch_grouped_gemm(dn, st)) != cudaSuccess) return cuda_status(e);
     return cuda_status(moe::launch_finalize(y, w, inv, T, H, k, out, st));
 }
 

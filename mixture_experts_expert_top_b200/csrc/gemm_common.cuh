@@ -30,6 +30,7 @@ constexpr int kQuarters = 4;                        // 64-K quarters per int4 st
 constexpr int kPackedTile = kBM * 128;              // 16 KB: 128 rows x 128 packed bytes
 constexpr int kConvGroups = kQuarters;              // decode group g handles quarter g of every stage
 constexpr int kMaxTmemA = 8;
+constexpr int kGuessKBlocks = 8;                    // weight K-blocks prefetched on a guess
 
 struct Params {
     const int32_t *offsets;
@@ -40,6 +41,7 @@ struct Params {
     int *err;
     const uint16_t *w_scales;   // int4: [E * w_rows, K/128]
     int evict_first_weights;
+    int hints;                  // kGemmHint* bits
 };
 
 // Tile bookkeeping shared by the roles.
@@ -79,7 +81,9 @@ __device__ __forceinline__ void build_tile_prefix(const int32_t *offsets, int E,
                                                   int *pre_s) {
     __shared__ int wsum[NT / 32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    for (int i = threadIdx.x; i <= E; i += NT) off_s[i] = __ldg(offsets + i);
+    // L2 reads (no L1 line can be stale): a kernel launched with an early
+    // start may read offsets before griddepcontrol.wait (kGemmHintOffsetsReady)
+    for (int i = threadIdx.x; i <= E; i += NT) off_s[i] = __ldcg(offsets + i);
     __syncthreads();
     const int seg = (E + NT - 1) / NT;
     const int b0 = threadIdx.x * seg;
@@ -209,6 +213,7 @@ inline Params make_params(const GemmArgs &g, int BN) {
     p.err = g.err;
     p.w_scales = g.w_scales;
     p.evict_first_weights = BN <= 32;
+    p.hints = g.hints;
     return p;
 }
 

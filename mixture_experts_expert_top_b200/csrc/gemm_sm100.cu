@@ -139,7 +139,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         tmem_relinquish();
     }
     // barriers, tensor maps and TMEM are set up while the previous kernel drains
-    griddep_wait();
+    const bool early = (p.hints & kGemmHintOffsetsReady) && !p.perm;
+    if (!early) {
+        if (warp == 0 && lane == 0 && (p.hints & kGemmHintPrefetchGuess)) {
+            // the tile this CTA gets if every expert has rows and one token block
+            const int e = blockIdx.x / MB, mb = blockIdx.x % MB;
+            if (e < E) {
+                const int a_row = e * p.w_rows + mb * kBM;
+                for (int kb = 0; kb < KB && kb < kGuessKBlocks; ++kb) {
+                    tma_prefetch_l2_2d(&tmA, kb * kBK, a_row);
+                    if (SWIGLU) tma_prefetch_l2_2d(&tmA, kb * kBK, a_row + p.m_out);
+                }
+            }
+        }
+        griddep_wait();
+    }
     build_tile_prefix<C::kThreads>(p.offsets, E, MB, BN, off_s, pre_s);
     tc_fence_before_sync();
     __syncthreads();
@@ -156,6 +170,28 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
+        // early: the weight tiles of the first STAGES ring slots go out before
+        // the previous kernel has finished; their token tiles follow the wait
+        int preloaded = 0;
+        if (early) {
+            for (int tile = blockIdx.x; tile < total_tiles && preloaded < STAGES; tile += gridDim.x) {
+                const TileInfo ti = decode_tile(tile, pre_s, off_s, E, MB, BN);
+                const int a_row = ti.e * p.w_rows + ti.mb * kBM;
+                const uint32_t tx = C::kABytes + (ti.n_mma / kBoxN) * kBoxBytesB;
+                for (int kb = 0; kb < KB && preloaded < STAGES; ++kb, ++preloaded) {
+                    if (lane == 0) {
+                        uint8_t *st = ring + preloaded * C::kStageBytes;
+                        mbar_arrive_expect_tx(&full_bar[preloaded], tx);
+                        tma_load_2d(st, &tmA, &full_bar[preloaded], kb * kBK, a_row, pol_w);
+                        if (SWIGLU)
+                            tma_load_2d(st + kTileBytesA, &tmA, &full_bar[preloaded], kb * kBK, a_row + p.m_out,
+                                        pol_w);
+                    }
+                }
+            }
+            griddep_wait();
+        }
+        int it = 0;
         for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
             const TileInfo ti = decode_tile(tile, pre_s, off_s, E, MB, BN);
             const int nbox = ti.n_mma / kBoxN;
@@ -167,16 +203,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll
                 for (int j = 0; j < 4; ++j) tr[j] = token_row(p, ti.row0 + 4 * lane + j);
             }
-            for (int kb = 0; kb < KB; ++kb) {
+            for (int kb = 0; kb < KB; ++kb, ++it) {
                 if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.err, 0);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 uint8_t *st = ring + stage * C::kStageBytes;
                 uint8_t *sb = st + C::kABytes;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&full_bar[stage], tx);
-                    tma_load_2d(st, &tmA, &full_bar[stage], kb * kBK, a_row, pol_w);
-                    if (SWIGLU) tma_load_2d(st + kTileBytesA, &tmA, &full_bar[stage], kb * kBK, a_row + p.m_out, pol_w);
+                    if (it >= preloaded) {
+                        mbar_arrive_expect_tx(&full_bar[stage], tx);
+                        tma_load_2d(st, &tmA, &full_bar[stage], kb * kBK, a_row, pol_w);
+                        if (SWIGLU)
+                            tma_load_2d(st + kTileBytesA, &tmA, &full_bar[stage], kb * kBK, a_row + p.m_out, pol_w);
+                    }
                     if (!p.perm)
                         for (int b = 0; b < nbox; ++b)
                             tma_load_2d(sb + b * kBoxBytesB, &tmB, &full_bar[stage], kb * kBK, ti.row0 + b * kBoxN,
@@ -191,6 +230,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
     } else if (warp == 1) {
         // ================================ MMA issuer ============================
+        if (early) griddep_wait();
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
@@ -232,6 +272,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             mbar_wait(drain_bar, 0, &never, p.err);
         }
     } else {
+        if (early) griddep_wait();
         run_epilogue<BN, SWIGLU, C::kAccCols>(p, pre_s, off_s, total_tiles, MB, tmem_base, tfull_bar, tempty_bar,
                                               abort_flag, 128);
     }

@@ -57,7 +57,16 @@ struct GemmArgs {
     bool swiglu;
     uint16_t *out;              // [P, m_out] bf16
     int *err;
+    int hints = 0;              // kGemmHint* bits, set only by moe_forward
 };
+// The kernel before this GEMM on the stream started after `offsets` was
+// complete, so the GEMM may read offsets and load weight tiles before
+// griddepcontrol.wait (only the token operand depends on the kernel before).
+constexpr int kGemmHintOffsetsReady = 1;
+// Before griddepcontrol.wait, prefetch into L2 the weights of the tile this
+// CTA would get if every expert had one token block (a guess: a wrong one
+// costs only bandwidth).
+constexpr int kGemmHintPrefetchGuess = 2;
 cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t s);
 // True when the gate/up GEMM for this shape should read the token rows through
 // perm itself (few rows per expert) rather than from a gathered copy.
