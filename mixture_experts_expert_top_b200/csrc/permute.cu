@@ -15,7 +15,7 @@
 // contiguous slice of the chunk and walks it 32 pairs at a time, using
 // __match_any_sync to rank equal experts inside each step. One CTA of 1024
 // threads does everything when P <= kSingleMax; otherwise three kernels run:
-// per-chunk histograms (CTAs of 256 threads, kChunk pairs each), one scan CTA,
+// per-chunk histograms (CTAs of 512 threads, kChunk pairs each), one scan CTA,
 // per-chunk scatter.
 #include "bucket_dev.cuh"
 #include "common.cuh"
@@ -27,7 +27,7 @@ namespace {
 
 constexpr int kThreads = 1024;        // single-CTA path and the scan CTA
 constexpr int kSingleMax = 8192;      // pairs handled by the single-CTA path
-constexpr int kChunkThreads = 256;    // multi-CTA path
+constexpr int kChunkThreads = 512;    // multi-CTA path
 constexpr int kChunk = 2048;          // pairs per CTA on the multi-CTA path
 
 // All pairs in one CTA.
@@ -59,7 +59,10 @@ permute_count_kernel(const int32_t *__restrict__ ids, int P, int E, int32_t *__r
 }
 
 // Multi-CTA pass 2 (one CTA): counts, offsets, and chunk_hist turned into the
-// first row of each (chunk, expert).
+// first row of each (chunk, expert). G = kThreads / E threads (a power of two,
+// at most 32, so one warp segment) share an expert: thread `part` owns a
+// contiguous run of chunks. Loads go out 8 at a time, so the walk over the
+// chunks is not one L2 round trip per chunk.
 __global__ void __launch_bounds__(kThreads, 1)
 permute_scan_kernel(int nchunks, int E, int32_t *__restrict__ chunk_hist, int32_t *__restrict__ counts,
                     int32_t *__restrict__ offsets) {
@@ -68,20 +71,51 @@ permute_scan_kernel(int nchunks, int E, int32_t *__restrict__ chunk_hist, int32_
     griddep_wait();
     int *tot = smem;        // [E]
     int *base = tot + E;    // [E]
-    for (int e = threadIdx.x; e < E; e += kThreads) {
-        int run = 0;
-        for (int c = 0; c < nchunks; ++c) {
-            const int v = chunk_hist[static_cast<size_t>(c) * E + e];
-            chunk_hist[static_cast<size_t>(c) * E + e] = run;
-            run += v;
+    int G = 1;
+    while (G < 32 && 2 * G * E <= kThreads) G *= 2;
+    const int e = threadIdx.x / G, part = threadIdx.x % G;
+    const bool active = e < E;
+    const int per = (nchunks + G - 1) / G;
+    const int c0 = part * per, c1 = min(nchunks, c0 + per);
+    int sum = 0;
+    if (active) {
+        for (int c = c0; c < c1; c += 8) {
+            int v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = c + j < c1 ? __ldcg(chunk_hist + static_cast<size_t>(c + j) * E + e) : 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) sum += v[j];
         }
-        tot[e] = run;
-        counts[e] = run;
+    }
+    // exclusive scan of `sum` over the G threads of this expert (lanes of one segment)
+    const int lane = threadIdx.x & 31;
+    int incl = sum;
+    for (int o = 1; o < G; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if ((lane % G) >= o) incl += y;
+    }
+    const int seg_last = (lane / G) * G + G - 1;
+    const int total = __shfl_sync(0xffffffffu, incl, seg_last);
+    if (active && part == 0) {
+        tot[e] = total;
+        counts[e] = total;
     }
     __syncthreads();
     block_exclusive_scan<kThreads>(tot, E, base, offsets);
-    for (int e = threadIdx.x; e < E; e += kThreads)
-        for (int c = 0; c < nchunks; ++c) chunk_hist[static_cast<size_t>(c) * E + e] += base[e];
+    if (active) {
+        int run = base[e] + incl - sum;
+        for (int c = c0; c < c1; c += 8) {
+            int v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = c + j < c1 ? __ldcg(chunk_hist + static_cast<size_t>(c + j) * E + e) : 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (c + j < c1) {
+                    chunk_hist[static_cast<size_t>(c + j) * E + e] = run;
+                    run += v[j];
+                }
+        }
+    }
 }
 
 // Multi-CTA pass 3: scatter each chunk from its per-expert first rows.
@@ -115,10 +149,22 @@ gather_rows_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__
         const int p = __ldg(perm + r);
         const uint4 *src = hidden + static_cast<size_t>(p / k) * vecs_per_row;
         uint4 *dst = out + static_cast<size_t>(r) * vecs_per_row;
-        // the copy is written once and read once by the next kernel: stream it
-        // past L2 so that the k-times-reused hidden rows stay resident
-#pragma unroll 4
-        for (int v = lane; v < vecs_per_row; v += 32) __stcs(dst + v, __ldg(src + v));
+        // all loads of a 4 KB slice are in flight before its stores; the copy is
+        // written once and read once by the next kernel: stream it past L2 so
+        // that the k-times-reused hidden rows stay resident
+        for (int v0 = 0; v0 < vecs_per_row; v0 += 32 * 8) {
+            uint4 buf[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int v = v0 + 32 * j + lane;
+                if (v < vecs_per_row) buf[j] = __ldg(src + v);
+            }
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const int v = v0 + 32 * j + lane;
+                if (v < vecs_per_row) __stcs(dst + v, buf[j]);
+            }
+        }
     }
 }
 
