@@ -72,12 +72,16 @@ __device__ __forceinline__ __nv_bfloat162 bf16_pair(uint16_t bits) {
 // bf16 weights
 // =============================================================================
 
-template <int BN, int STAGES, bool SWIGLU>
+// KSUB 64-K sub-blocks per ring stage (down only): fewer, larger hand-offs
+// when the weight tile of a stage would otherwise be only 16 KB.
+template <int BN, int STAGES, bool SWIGLU, int KSUB = 1>
 struct Bf16Cfg {
-    static constexpr int kNumA = SWIGLU ? 2 : 1;
+    static_assert(KSUB == 1 || !SWIGLU, "gate/up stages already hold two weight tiles");
+    static constexpr int kNumA = SWIGLU ? 2 : KSUB;
     static constexpr int kThreads = 192;
     static constexpr int kABytes = kNumA * kTileBytesA;
-    static constexpr int kStageBytes = kABytes + BN * kBK * 2;
+    static constexpr int kBSub = BN * kBK * 2;                 // token rows of one 64-K sub-block
+    static constexpr int kStageBytes = kABytes + KSUB * kBSub;
     static constexpr int kAccCols = SWIGLU ? 2 * BN : BN;
     static constexpr int kTmemUsed = 2 * kAccCols;
     static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
@@ -91,11 +95,11 @@ struct Bf16Cfg {
     static_assert(kSmemBytes + 64 <= kSmemLimit, "shared memory");
 };
 
-template <int BN, int STAGES, bool SWIGLU>
+template <int BN, int STAGES, bool SWIGLU, int KSUB>
 __global__ void __launch_bounds__(192, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const Params p) {
-    using C = Bf16Cfg<BN, STAGES, SWIGLU>;
+    using C = Bf16Cfg<BN, STAGES, SWIGLU, KSUB>;
     extern __shared__ uint8_t smem_raw[];
     // operand tiles need 1024-byte alignment in the shared window (swizzle atoms)
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -115,7 +119,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const int lane = threadIdx.x & 31;
     const int E = p.E;
     const int MB = (p.m_out + kBM - 1) / kBM;
-    const int KB = (p.K + kBK - 1) / kBK;
+    const int KB = (p.K + KSUB * kBK - 1) / (KSUB * kBK);   // ring stages per tile
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -177,12 +181,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             for (int tile = blockIdx.x; tile < total_tiles && preloaded < STAGES; tile += gridDim.x) {
                 const TileInfo ti = decode_tile(tile, pre_s, off_s, E, MB, BN);
                 const int a_row = ti.e * p.w_rows + ti.mb * kBM;
-                const uint32_t tx = C::kABytes + (ti.n_mma / kBoxN) * kBoxBytesB;
+                const uint32_t tx = C::kABytes + KSUB * (ti.n_mma / kBoxN) * kBoxBytesB;
                 for (int kb = 0; kb < KB && preloaded < STAGES; ++kb, ++preloaded) {
                     if (lane == 0) {
                         uint8_t *st = ring + preloaded * C::kStageBytes;
                         mbar_arrive_expect_tx(&full_bar[preloaded], tx);
-                        tma_load_2d(st, &tmA, &full_bar[preloaded], kb * kBK, a_row, pol_w);
+                        for (int u = 0; u < KSUB; ++u)
+                            tma_load_2d(st + u * kTileBytesA, &tmA, &full_bar[preloaded], (kb * KSUB + u) * kBK,
+                                        a_row, pol_w);
                         if (SWIGLU)
                             tma_load_2d(st + kTileBytesA, &tmA, &full_bar[preloaded], kb * kBK, a_row + p.m_out,
                                         pol_w);
@@ -196,7 +202,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const TileInfo ti = decode_tile(tile, pre_s, off_s, E, MB, BN);
             const int nbox = ti.n_mma / kBoxN;
             const int a_row = ti.e * p.w_rows + ti.mb * kBM;
-            const uint32_t tx = C::kABytes + nbox * kBoxBytesB;
+            const uint32_t tx = C::kABytes + KSUB * nbox * kBoxBytesB;
             const bool gather_lane = p.perm && 4 * lane < ti.n_mma;
             int tr[4] = {0, 0, 0, 0};
             if (gather_lane) {
@@ -212,19 +218,23 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (lane == 0) {
                     if (it >= preloaded) {
                         mbar_arrive_expect_tx(&full_bar[stage], tx);
-                        tma_load_2d(st, &tmA, &full_bar[stage], kb * kBK, a_row, pol_w);
+                        for (int u = 0; u < KSUB; ++u)
+                            tma_load_2d(st + u * kTileBytesA, &tmA, &full_bar[stage], (kb * KSUB + u) * kBK, a_row,
+                                        pol_w);
                         if (SWIGLU)
                             tma_load_2d(st + kTileBytesA, &tmA, &full_bar[stage], kb * kBK, a_row + p.m_out, pol_w);
                     }
                     if (!p.perm)
-                        for (int b = 0; b < nbox; ++b)
-                            tma_load_2d(sb + b * kBoxBytesB, &tmB, &full_bar[stage], kb * kBK, ti.row0 + b * kBoxN,
-                                        pol_x);
+                        for (int u = 0; u < KSUB; ++u)
+                            for (int b = 0; b < nbox; ++b)
+                                tma_load_2d(sb + u * C::kBSub + b * kBoxBytesB, &tmB, &full_bar[stage],
+                                            (kb * KSUB + u) * kBK, ti.row0 + b * kBoxN, pol_x);
                 }
                 __syncwarp();
                 if (gather_lane)
-                    tma_gather4(sb + lane * 4 * kBK * 2, &tmB, &full_bar[stage], kb * kBK, tr[0], tr[1], tr[2], tr[3],
-                                pol_x);
+                    for (int u = 0; u < KSUB; ++u)
+                        tma_gather4(sb + u * C::kBSub + lane * 4 * kBK * 2, &tmB, &full_bar[stage],
+                                    (kb * KSUB + u) * kBK, tr[0], tr[1], tr[2], tr[3], pol_x);
                 if (++stage == STAGES) { stage = 0; phase ^= 1; }
             }
         }
@@ -249,15 +259,26 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     if (!ok) break;
                     tc_fence_after_sync();
                     const uint32_t st = smem_u32(ring + stage * C::kStageBytes);
-                    const uint64_t da0 = sw128_kmajor_desc(st);
-                    const uint64_t da1 = sw128_kmajor_desc(st + kTileBytesA);
-                    const uint64_t db = sw128_kmajor_desc(st + C::kABytes);
+                    if constexpr (SWIGLU) {
+                        const uint64_t da0 = sw128_kmajor_desc(st);
+                        const uint64_t da1 = sw128_kmajor_desc(st + kTileBytesA);
+                        const uint64_t db = sw128_kmajor_desc(st + C::kABytes);
 #pragma unroll
-                    for (int k = 0; k < kBK / 16; ++k) {
-                        const uint32_t acc = (kb | k) != 0;
-                        // +32 bytes per K step inside the swizzled row: +2 in the >>4 address field
-                        umma_bf16_ss(d0, da0 + 2 * k, db + 2 * k, idesc, acc);
-                        if (SWIGLU) umma_bf16_ss(d0 + BN, da1 + 2 * k, db + 2 * k, idesc, acc);
+                        for (int k = 0; k < kBK / 16; ++k) {
+                            const uint32_t acc = (kb | k) != 0;
+                            // +32 bytes per K step inside the swizzled row: +2 in the >>4 address field
+                            umma_bf16_ss(d0, da0 + 2 * k, db + 2 * k, idesc, acc);
+                            umma_bf16_ss(d0 + BN, da1 + 2 * k, db + 2 * k, idesc, acc);
+                        }
+                    } else {
+#pragma unroll
+                        for (int u = 0; u < KSUB; ++u) {
+                            const uint64_t da = sw128_kmajor_desc(st + u * kTileBytesA);
+                            const uint64_t db = sw128_kmajor_desc(st + C::kABytes + u * C::kBSub);
+#pragma unroll
+                            for (int k = 0; k < kBK / 16; ++k)
+                                umma_bf16_ss(d0, da + 2 * k, db + 2 * k, idesc, (kb | u | k) != 0);
+                        }
                     }
                     umma_commit(&empty_bar[stage]);
                     if (++stage == STAGES) { stage = 0; phase ^= 1; }
@@ -571,16 +592,16 @@ grouped_gemm_int4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
 
 // ------------------------------------------------------------------ host side
 
-template <int BN, int STAGES, bool SWIGLU>
+template <int BN, int STAGES, bool SWIGLU, int KSUB = 1>
 cudaError_t run_bf16(const GemmArgs &g, cudaStream_t s) {
-    using C = Bf16Cfg<BN, STAGES, SWIGLU>;
+    using C = Bf16Cfg<BN, STAGES, SWIGLU, KSUB>;
     CUtensorMap ta, tb;
     const uint64_t a_rows = static_cast<uint64_t>(g.E) * g.w_rows;
     bool ok = make_map(&ta, g.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.K, a_rows, kBK, kBM,
                        CU_TENSOR_MAP_SWIZZLE_128B) &&
               make_token_map(&tb, g, kBoxN);
     if (!ok) return cudaErrorInvalidValue;
-    auto kern = grouped_gemm_kernel<BN, STAGES, SWIGLU>;
+    auto kern = grouped_gemm_kernel<BN, STAGES, SWIGLU, KSUB>;
     cudaError_t st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (st != cudaSuccess) return st;
     const int grid = grid_for(g, BN);
@@ -614,7 +635,7 @@ cudaError_t dispatch_bf16(const GemmArgs &g, cudaStream_t s) {
         if (avg <= 48) return run_bf16<64, 5, SWIGLU>(g, s);
         return run_bf16<128, 4, SWIGLU>(g, s);
     } else {
-        if (avg <= 24) return run_bf16<32, 10, SWIGLU>(g, s);
+        if (avg <= 24) return run_bf16<32, 5, SWIGLU, 2>(g, s);          // 40 KB stages (two 64-K blocks)
         if (avg <= 48) return run_bf16<64, 8, SWIGLU>(g, s);
         return run_bf16<128, 6, SWIGLU>(g, s);
     }
