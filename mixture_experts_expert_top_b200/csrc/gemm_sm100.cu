@@ -315,8 +315,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 // W4A16: int4 weights (one bf16 scale per 128 K), bf16 tokens
 // =============================================================================
 
-template <int BN, int STAGES, bool SWIGLU>
+// GROUPS hand-off groups of decode warps: the 16 decode warps convert the
+// four 64-K quarters of a stage (one quarter per 4 warps, one warp per TMEM
+// lane quarter), and the quarters of one group share one TMEM ring slot, so
+// the MMA issuer is signalled GROUPS times per stage, not four.
+template <int BN, int STAGES, bool SWIGLU, int GROUPS = kConvGroups>
 struct Int4Cfg {
+    static_assert(kQuarters % GROUPS == 0, "groups split the four quarters evenly");
+    static constexpr int kQPG = kQuarters / GROUPS;                     // quarters per group (slot)
     static constexpr int kNumA = SWIGLU ? 2 : 1;
     static constexpr int kThreads = 192 + 128 * kConvGroups;
     static constexpr int kABytes = kNumA * kPackedTile;                 // packed A per stage (K = 256)
@@ -324,9 +330,11 @@ struct Int4Cfg {
     static constexpr int kStageBytes = kABytes + kQuarters * kBQuarter;
     static constexpr int kAccCols = SWIGLU ? 2 * BN : BN;
     static constexpr int kACols = kNumA * (kBK / 2);                    // TMEM columns per decoded quarter
-    static constexpr int kTmemAStages = (512 - 2 * kAccCols) / kACols < kMaxTmemA ? (512 - 2 * kAccCols) / kACols
-                                                                                 : kMaxTmemA;
-    static constexpr int kTmemUsed = 2 * kAccCols + kTmemAStages * kACols;
+    static constexpr int kSlotCols = kQPG * kACols;                     // TMEM columns per ring slot
+    static constexpr int kTmemAStages = (512 - 2 * kAccCols) / kSlotCols < kMaxTmemA
+                                            ? (512 - 2 * kAccCols) / kSlotCols
+                                            : kMaxTmemA;
+    static constexpr int kTmemUsed = 2 * kAccCols + kTmemAStages * kSlotCols;
     static constexpr int kTmemCols = kTmemUsed <= 32 ? 32 : kTmemUsed <= 64 ? 64 : kTmemUsed <= 128 ? 128
                                    : kTmemUsed <= 256 ? 256 : 512;
     static constexpr int kRingBytes = STAGES * kStageBytes;
@@ -334,16 +342,16 @@ struct Int4Cfg {
     static constexpr int kSmemBytes = 1024 + kRingBytes + 8 * kNumBars + 64 + 2 * (kMaxExperts + 1) * 4;
     static_assert(kStageBytes % 1024 == 0 && kBQuarter % 1024 == 0, "tiles must keep 1024-byte alignment");
     static_assert(kTmemUsed <= 512, "TMEM holds 512 32-bit columns");
-    static_assert(kTmemAStages >= kConvGroups, "every decode group needs a TMEM slot in flight");
+    static_assert(kTmemAStages >= GROUPS, "every decode group needs a TMEM slot in flight");
     static_assert(BN % kBoxN == 0 && BN <= 256, "BN");
     static_assert(kSmemBytes + 64 <= kSmemLimit, "shared memory");
 };
 
-template <int BN, int STAGES, bool SWIGLU>
-__global__ void __launch_bounds__(Int4Cfg<BN, STAGES, SWIGLU>::kThreads, 1)
+template <int BN, int STAGES, bool SWIGLU, int GROUPS>
+__global__ void __launch_bounds__(Int4Cfg<BN, STAGES, SWIGLU, GROUPS>::kThreads, 1)
 grouped_gemm_int4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                          const Params p) {
-    using C = Int4Cfg<BN, STAGES, SWIGLU>;
+    using C = Int4Cfg<BN, STAGES, SWIGLU, GROUPS>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *ring = smem;                                    // STAGES x [Aq0 | Aq1 | B quarter 0..3]
@@ -372,7 +380,7 @@ grouped_gemm_int4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
             mbar_init(&empty_bar[s], 1);
         }
         for (int t = 0; t < C::kTmemAStages; ++t) {
-            mbar_init(&tready_bar[t], 128);   // the 4 warps of one decode group
+            mbar_init(&tready_bar[t], 128 * C::kQPG);   // every warp of one decode group
             mbar_init(&tfree_bar[t], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -463,19 +471,23 @@ grouped_gemm_int4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
                 const uint32_t d0 = tmem_base + buf * C::kAccCols;
                 for (int ks = 0; ks < KS && ok; ++ks) {
                     const uint32_t sb = smem_u32(ring + stage * C::kStageBytes + C::kABytes);
-                    for (int j = 0; j < kQuarters; ++j) {
+                    for (int g = 0; g < GROUPS; ++g) {
                         // tready implies the stage's TMA data landed (the decode group waited for it)
                         ok = mbar_wait(&tready_bar[t], tphase, abort_flag, p.err, 0);
                         if (!ok) break;
                         tc_fence_after_sync();
-                        const uint32_t a0 = tmem_a0 + t * C::kACols;
-                        const uint64_t db = sw128_kmajor_desc(sb + j * C::kBQuarter);
 #pragma unroll
-                        for (int k = 0; k < kBK / 16; ++k) {
-                            const uint32_t acc = (ks | j | k) != 0;
-                            // 16 K elements = 8 TMEM columns of A; +32 bytes of B per K step
-                            umma_bf16_ts(d0, a0 + 8 * k, db + 2 * k, idesc, acc);
-                            if (SWIGLU) umma_bf16_ts(d0 + BN, a0 + 32 + 8 * k, db + 2 * k, idesc, acc);
+                        for (int qq = 0; qq < C::kQPG; ++qq) {
+                            const int j = g * C::kQPG + qq;                     // quarter of the stage
+                            const uint32_t a0 = tmem_a0 + t * C::kSlotCols + qq * C::kACols;
+                            const uint64_t db = sw128_kmajor_desc(sb + j * C::kBQuarter);
+#pragma unroll
+                            for (int k = 0; k < kBK / 16; ++k) {
+                                const uint32_t acc = (ks | j | k) != 0;
+                                // 16 K elements = 8 TMEM columns of A; +32 bytes of B per K step
+                                umma_bf16_ts(d0, a0 + 8 * k, db + 2 * k, idesc, acc);
+                                if (SWIGLU) umma_bf16_ts(d0 + BN, a0 + 32 + 8 * k, db + 2 * k, idesc, acc);
+                            }
                         }
                         umma_commit(&tfree_bar[t]);
                         if (++t == C::kTmemAStages) { t = 0; tphase ^= 1; }
@@ -496,11 +508,15 @@ grouped_gemm_int4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
         run_epilogue<BN, SWIGLU, C::kAccCols>(p, pre_s, off_s, total_tiles, MB, tmem_base, tfull_bar, tempty_bar,
                                               abort_flag);
     } else {
-        // ====== warps 6-21: decode group g = quarter g of every ring stage =======
+        // ====== warps 6-21: quarter g of every ring stage =======================
         // Row r of the tile, packed bytes [32g, 32g+32) of the stage's 128-byte
         // row (stored with the 128-byte swizzle: 16-byte chunk c of row r sits
-        // at chunk c ^ (r % 8)), K elements 64g .. 64g+63 of the stage.
+        // at chunk c ^ (r % 8)), K elements 64g .. 64g+63 of the stage. The
+        // quarter belongs to hand-off group g / kQPG, column block g % kQPG of
+        // that group's TMEM slot.
         const int g = (warp - 6) >> 2;
+        const int grp_id = g / C::kQPG;
+        const uint32_t qcol = static_cast<uint32_t>((g % C::kQPG) * C::kACols);
         const int q = warp & 3;                 // TMEM lane quarter = rows q*32 .. q*32+31
         const int r = q * 32 + lane;
         const int kgroups = p.K / 128;
@@ -542,8 +558,8 @@ grouped_gemm_int4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
         fetch(sb_next);
         int stage = 0;
         uint32_t sphase = 0;
-        int t = g % C::kTmemAStages;
-        uint32_t tphase = (g / C::kTmemAStages) & 1;
+        int t = grp_id % C::kTmemAStages;
+        uint32_t tphase = (grp_id / C::kTmemAStages) & 1;
         const int ch0 = ((2 * g) ^ (r & 7)) << 4, ch1 = ((2 * g + 1) ^ (r & 7)) << 4;
         while (c_tile < total_tiles) {
             const uint16_t sb0 = sb_cur[0], sb1 = sb_cur[1];
@@ -566,14 +582,15 @@ grouped_gemm_int4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
                 uint32_t out[32];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) dequant_word(words[i], s2, out + 4 * i);
-                tmem_st_32x32b_x32(tmem_a0 + (static_cast<uint32_t>(q * 32) << 16) + t * C::kACols + a * 32, out);
+                tmem_st_32x32b_x32(tmem_a0 + (static_cast<uint32_t>(q * 32) << 16) + t * C::kSlotCols + qcol + a * 32,
+                                   out);
             }
             tmem_wait_st();
             tc_fence_before_sync();
             mbar_arrive(&tready_bar[t]);
             if (++stage == STAGES) { stage = 0; sphase ^= 1; }
-            // this group's next quarter is kQuarters ring slots further on
-            t += kConvGroups;
+            // this group's slot for the next stage is GROUPS ring slots further on
+            t += GROUPS;
             while (t >= C::kTmemAStages) { t -= C::kTmemAStages; tphase ^= 1; }
         }
     }
@@ -609,9 +626,9 @@ cudaError_t run_bf16(const GemmArgs &g, cudaStream_t s) {
     return launch_pdl(kern, dim3(grid), dim3(C::kThreads), C::kSmemBytes, s, ta, tb, make_params(g, BN));
 }
 
-template <int BN, int STAGES, bool SWIGLU>
+template <int BN, int STAGES, bool SWIGLU, int GROUPS>
 cudaError_t run_int4(const GemmArgs &g, cudaStream_t s) {
-    using C = Int4Cfg<BN, STAGES, SWIGLU>;
+    using C = Int4Cfg<BN, STAGES, SWIGLU, GROUPS>;
     CUtensorMap ta, tb;
     const uint64_t a_rows = static_cast<uint64_t>(g.E) * g.w_rows;
     // packed weights: 128 bytes (K = 256) per row and stage, 128-byte swizzle
@@ -619,7 +636,7 @@ cudaError_t run_int4(const GemmArgs &g, cudaStream_t s) {
                        CU_TENSOR_MAP_SWIZZLE_128B) &&
               make_token_map(&tb, g, kBoxN);
     if (!ok) return cudaErrorInvalidValue;
-    auto kern = grouped_gemm_int4_kernel<BN, STAGES, SWIGLU>;
+    auto kern = grouped_gemm_int4_kernel<BN, STAGES, SWIGLU, GROUPS>;
     cudaError_t st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (st != cudaSuccess) return st;
     const int grid = grid_for(g, BN);
@@ -645,11 +662,11 @@ template <bool SWIGLU>
 cudaError_t dispatch_int4(const GemmArgs &g, cudaStream_t s) {
     const double avg = static_cast<double>(g.P) / g.E;
     if constexpr (SWIGLU) {
-        if (avg <= 24) return run_int4<32, 4, SWIGLU>(g, s);    // 48 KB stages
-        return run_int4<64, 3, SWIGLU>(g, s);                   // 64 KB stages
+        if (avg <= 24) return run_int4<32, 4, SWIGLU, 2>(g, s);    // 48 KB stages, 3 slots of 128 K
+        return run_int4<64, 3, SWIGLU, 4>(g, s);                   // 64 KB stages
     } else {
-        if (avg <= 24) return run_int4<32, 6, SWIGLU>(g, s);    // 32 KB stages
-        return run_int4<64, 4, SWIGLU>(g, s);                   // 48 KB stages
+        if (avg <= 24) return run_int4<32, 6, SWIGLU, 1>(g, s);    // 32 KB stages, 3 slots of 256 K
+        return run_int4<64, 4, SWIGLU, 2>(g, s);                   // 48 KB stages
     }
 }
 
