@@ -72,12 +72,12 @@ __device__ __forceinline__ __nv_bfloat162 bf16_pair(uint16_t bits) {
 // bf16 weights
 // =============================================================================
 
-// KSUB 64-K sub-blocks per ring stage (down only): fewer, larger hand-offs
-// when the weight tile of a stage would otherwise be only 16 KB.
+// KSUB 64-K sub-blocks per ring stage: fewer, larger hand-offs between the
+// producer and the MMA issuer. A stage holds, per sub-block u, the weight
+// tile (gate/up: the gate tile then the up tile) and then all token tiles.
 template <int BN, int STAGES, bool SWIGLU, int KSUB = 1>
 struct Bf16Cfg {
-    static_assert(KSUB == 1 || !SWIGLU, "gate/up stages already hold two weight tiles");
-    static constexpr int kNumA = SWIGLU ? 2 : KSUB;
+    static constexpr int kNumA = (SWIGLU ? 2 : 1) * KSUB;
     static constexpr int kThreads = 192;
     static constexpr int kABytes = kNumA * kTileBytesA;
     static constexpr int kBSub = BN * kBK * 2;                 // token rows of one 64-K sub-block
@@ -186,12 +186,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     if (lane == 0) {
                         uint8_t *st = ring + preloaded * C::kStageBytes;
                         mbar_arrive_expect_tx(&full_bar[preloaded], tx);
-                        for (int u = 0; u < KSUB; ++u)
-                            tma_load_2d(st + u * kTileBytesA, &tmA, &full_bar[preloaded], (kb * KSUB + u) * kBK,
-                                        a_row, pol_w);
-                        if (SWIGLU)
-                            tma_load_2d(st + kTileBytesA, &tmA, &full_bar[preloaded], kb * kBK, a_row + p.m_out,
-                                        pol_w);
+                        for (int u = 0; u < KSUB; ++u) {
+                            uint8_t *sa = st + (SWIGLU ? 2 * u : u) * kTileBytesA;
+                            const int x = (kb * KSUB + u) * kBK;
+                            tma_load_2d(sa, &tmA, &full_bar[preloaded], x, a_row, pol_w);
+                            if (SWIGLU) tma_load_2d(sa + kTileBytesA, &tmA, &full_bar[preloaded], x, a_row + p.m_out, pol_w);
+                        }
                     }
                 }
             }
@@ -218,11 +218,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 if (lane == 0) {
                     if (it >= preloaded) {
                         mbar_arrive_expect_tx(&full_bar[stage], tx);
-                        for (int u = 0; u < KSUB; ++u)
-                            tma_load_2d(st + u * kTileBytesA, &tmA, &full_bar[stage], (kb * KSUB + u) * kBK, a_row,
-                                        pol_w);
-                        if (SWIGLU)
-                            tma_load_2d(st + kTileBytesA, &tmA, &full_bar[stage], kb * kBK, a_row + p.m_out, pol_w);
+                        for (int u = 0; u < KSUB; ++u) {
+                            uint8_t *sa = st + (SWIGLU ? 2 * u : u) * kTileBytesA;
+                            const int x = (kb * KSUB + u) * kBK;
+                            tma_load_2d(sa, &tmA, &full_bar[stage], x, a_row, pol_w);
+                            if (SWIGLU) tma_load_2d(sa + kTileBytesA, &tmA, &full_bar[stage], x, a_row + p.m_out, pol_w);
+                        }
                     }
                     if (!p.perm)
                         for (int u = 0; u < KSUB; ++u)
@@ -259,25 +260,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     if (!ok) break;
                     tc_fence_after_sync();
                     const uint32_t st = smem_u32(ring + stage * C::kStageBytes);
-                    if constexpr (SWIGLU) {
-                        const uint64_t da0 = sw128_kmajor_desc(st);
-                        const uint64_t da1 = sw128_kmajor_desc(st + kTileBytesA);
-                        const uint64_t db = sw128_kmajor_desc(st + C::kABytes);
+#pragma unroll
+                    for (int u = 0; u < KSUB; ++u) {
+                        const uint32_t sa = st + (SWIGLU ? 2 * u : u) * kTileBytesA;
+                        const uint64_t da0 = sw128_kmajor_desc(sa);
+                        const uint64_t db = sw128_kmajor_desc(st + C::kABytes + u * C::kBSub);
 #pragma unroll
                         for (int k = 0; k < kBK / 16; ++k) {
-                            const uint32_t acc = (kb | k) != 0;
+                            const uint32_t acc = (kb | u | k) != 0;
                             // +32 bytes per K step inside the swizzled row: +2 in the >>4 address field
                             umma_bf16_ss(d0, da0 + 2 * k, db + 2 * k, idesc, acc);
-                            umma_bf16_ss(d0 + BN, da1 + 2 * k, db + 2 * k, idesc, acc);
-                        }
-                    } else {
-#pragma unroll
-                        for (int u = 0; u < KSUB; ++u) {
-                            const uint64_t da = sw128_kmajor_desc(st + u * kTileBytesA);
-                            const uint64_t db = sw128_kmajor_desc(st + C::kABytes + u * C::kBSub);
-#pragma unroll
-                            for (int k = 0; k < kBK / 16; ++k)
-                                umma_bf16_ss(d0, da + 2 * k, db + 2 * k, idesc, (kb | u | k) != 0);
+                            if (SWIGLU) umma_bf16_ss(d0 + BN, sw128_kmajor_desc(sa + kTileBytesA) + 2 * k, db + 2 * k, idesc, acc);
                         }
                     }
                     umma_commit(&empty_bar[stage]);
@@ -648,7 +641,7 @@ template <bool SWIGLU>
 cudaError_t dispatch_bf16(const GemmArgs &g, cudaStream_t s) {
     const double avg = static_cast<double>(g.P) / g.E;   // pairs per expert if the load were even
     if constexpr (SWIGLU) {
-        if (avg <= 24) return run_bf16<32, 6, SWIGLU>(g, s);
+        if (avg <= 24) return run_bf16<32, 3, SWIGLU, 2>(g, s);          // 72 KB stages (two 64-K blocks)
         if (avg <= 48) return run_bf16<64, 5, SWIGLU>(g, s);
         return run_bf16<128, 4, SWIGLU>(g, s);
     } else {
