@@ -141,6 +141,33 @@ def test_layer_is_deterministic():
     assert torch.equal(Lp.forward().view(torch.int16), a.view(torch.int16))
 
 
+@pytest.mark.parametrize("name", ["qwen3_decode", "w4a16_decode", "qwen3_prefill"])
+def test_back_to_back_calls_with_different_routing(name):
+    # moe_forward starts each kernel before the previous one on the stream has
+    # finished (programmatic dependent launch), and the decode down GEMM reads
+    # the expert offsets before its wait. Alternating two batches whose routing
+    # differs, with no synchronisation between the calls, would expose a kernel
+    # that sees the previous call's offsets or rows.
+    kw = {"T": 1024} if name == "qwen3_prefill" else {}
+    cfg = moe_synth.get_config(name, **kw)
+    A = Layer(cfg, seed=0)
+    # B: other tokens and logits, the same weights and the same workspace
+    B = Layer.__new__(Layer)
+    B.cfg, B.shape, B.ws = cfg, A.shape, A.ws
+    B.inp = dict(A.inp, hidden=moe_synth.gen_hidden(cfg, seed=7), logits=moe_synth.gen_logits(cfg, seed=7))
+    B.d = dict(A.d, hidden=B.inp["hidden"].to(DEV), logits=B.inp["logits"].to(DEV))
+    ref_a = A.steps()["out"].clone()
+    ref_b = B.steps()["out"].clone()
+    assert not torch.equal(ref_a.view(torch.int16), ref_b.view(torch.int16))
+    outs = []
+    for i in range(6):
+        outs.append((A if i % 2 == 0 else B).forward())
+    torch.cuda.synchronize()
+    for i, o in enumerate(outs):
+        ref = ref_a if i % 2 == 0 else ref_b
+        assert torch.equal(o.view(torch.int16), ref.view(torch.int16)), f"call {i}"
+
+
 def test_forward_host_matches_forward():
     L = Layer(moe_synth.get_config("qwen3_decode"))
     ref = L.forward()
