@@ -179,6 +179,16 @@ MOE_API moe_status_t moe_dequant_int4(const uint8_t *q, const moe_bf16_t *scales
  * timed out) and clears it. */
 MOE_API moe_status_t moe_get_device_error(int32_t *code);
 
+/* Self-test of the bounded waits behind device error code 2 (no counterpart
+ * on the pages). Enqueues one CTA that waits on a pipeline barrier that
+ * nothing ever arrives on; after limit_ns nanoseconds of %globaltimer the
+ * wait gives up, sets the device error flag to 2 and the kernel returns.
+ * Nothing faults or traps and the context stays usable: a following
+ * moe_get_device_error() reads 2 and clears it.
+ *   limit_ns  1 .. 1e9 (one second at most), else MOE_ERR_INVALID_ARG
+ *             and nothing is enqueued. */
+MOE_API moe_status_t moe_selftest_bounded_wait(int64_t limit_ns, moe_stream_t stream);
+
 /* moe_permute for callers that cannot allocate device memory: the same
  * outputs, bit for bit, with the scratch taken from a fixed 256 KiB array
  * built into the library instead of a caller workspace. It is meant for code

@@ -327,6 +327,12 @@ moe_status_t moe_get_device_error(int32_t *code) {
     return MOE_OK;
 }
 
+moe_status_t moe_selftest_bounded_wait(int64_t limit_ns, moe_stream_t stream) {
+    if (limit_ns < 1 || limit_ns > 1000000000LL) return MOE_ERR_INVALID_ARG;
+    return cuda_status(moe::launch_bounded_wait_selftest(static_cast<unsigned long long>(limit_ns), error_flag_ptr(),
+                                                         static_cast<cudaStream_t>(stream)));
+}
+
 const char *moe_status_string(moe_status_t status) {
     switch (status) {
         case MOE_OK: return "ok";

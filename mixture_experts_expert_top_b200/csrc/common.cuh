@@ -70,7 +70,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 // doing work (a long cap for waits that span whole tiles; 0 = never sleep, for
 // waits on the critical path).
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort, int *err,
-                                          uint32_t max_sleep_ns = 64) {
+                                          uint32_t max_sleep_ns = 64,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     uint32_t n = 0, sleep_ns = 8;
@@ -81,7 +82,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
         }
         if ((n & 63u) == 0u) {
             if (*abort) return false;
-            if (globaltimer_ns() - t0 > kWaitLimitNs) {
+            if (globaltimer_ns() - t0 > limit_ns) {
                 raise_error(err, kErrTimeout);
                 *abort = 1;
                 return false;

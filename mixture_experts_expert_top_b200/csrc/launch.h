@@ -18,6 +18,11 @@ moe_status_t validate_shape(const moe_shape_t *shape);
 // Device address of the library's error flag word on the current device.
 int *device_error_flag();
 
+// ---- selftest.cu
+// One CTA waits limit_ns on an mbarrier that nothing arrives on (the
+// bounded-wait path: the wait gives up and raises the timeout code).
+cudaError_t launch_bounded_wait_selftest(unsigned long long limit_ns, int *err, cudaStream_t s);
+
 // ---- route.cu
 cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s);
 

@@ -104,6 +104,9 @@ def test_bad_arguments_are_rejected_before_any_launch():
     assert L.moe_permute(16, byref(sh), 16, 16, 16, 16, 16, None, None, 0, None) == 1
     # dequant: K not a multiple of 128
     assert L.moe_dequant_int4(16, 16, 4, 100, 16, None) == 1
+    # bounded-wait self-test: limit outside 1 ns .. 1 s
+    assert L.moe_selftest_bounded_wait(0, None) == 1
+    assert L.moe_selftest_bounded_wait(2_000_000_000, None) == 1
 
 
 def test_empty_batch_is_a_no_op():

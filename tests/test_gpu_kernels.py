@@ -256,3 +256,19 @@ def test_grouped_gemm_swiglu_gathers_through_perm(cfg):
 def test_grouped_gemm_int4_matches_oracle():
     cfg = moe_synth.MoeConfig("int4_mid", T=48, H=1024, I=384, E=12, k=4, fmt="int4_g128")
     test_grouped_gemm_swiglu_and_down_match_oracle(cfg)
+
+
+# ------------------------------------------------------------ failure path --
+
+def test_a_wait_that_never_completes_gives_up_and_reports_a_timeout():
+    # One CTA waits on a pipeline barrier that nothing arrives on, with a
+    # 20 ms limit: the wait must give up, raise code 2 and let the kernel end,
+    # and the context must stay usable afterwards.
+    assert moe.moe_get_device_error() == 0
+    moe.moe_selftest_bounded_wait(20_000_000)
+    assert moe.moe_get_device_error() == 2      # synchronises, reads and clears
+    assert moe.moe_get_device_error() == 0
+    logits = torch.randn(40, 64, generator=torch.Generator().manual_seed(3))
+    gi, _ = run_route(logits, 6)
+    oi, _ = oracle.route(logits, 6)
+    assert np.array_equal(gi, oi)
