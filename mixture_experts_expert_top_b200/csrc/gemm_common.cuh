@@ -28,7 +28,7 @@ constexpr int kEpiThreads = 128;                    // warps 2-5
 // int4 kernel (gemm_sm100.cu)
 constexpr int kQuarters = 4;                        // 64-K quarters per int4 stage (K = 256)
 constexpr int kPackedTile = kBM * 128;              // 16 KB: 128 rows x 128 packed bytes
-constexpr int kConvGroups = kQuarters;              // decode group g handles quarter g of every stage
+constexpr int kConvGroups = kQuarters;              // 4 x 4 decode warps: one set of 4 per quarter
 constexpr int kMaxTmemA = 8;
 constexpr int kGuessKBlocks = 8;                    // weight K-blocks prefetched on a guess
 
