@@ -446,7 +446,7 @@ cudaError_t run_prefill_pair(const GemmArgs &g, cudaStream_t s) {
                        CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok || g.perm) return cudaErrorInvalidValue;
     auto kern = grouped_gemm_prefill_pair_kernel<SWIGLU, STAGES>;
-    cudaError_t st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    cudaError_t st = ensure_dynamic_smem(kern, C::kSmemBytes);
     if (st != cudaSuccess) return st;
     constexpr int kFeat = SWIGLU ? 128 : 256;
     const long long NB = (g.m_out + kFeat - 1) / kFeat;
@@ -468,7 +468,7 @@ cudaError_t run_prefill(const GemmArgs &g, cudaStream_t s) {
                        CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return cudaErrorInvalidValue;
     auto kern = grouped_gemm_prefill_kernel<SWIGLU, STAGES>;
-    cudaError_t st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    cudaError_t st = ensure_dynamic_smem(kern, C::kSmemBytes);
     if (st != cudaSuccess) return st;
     constexpr int kFeat = SWIGLU ? 128 : 256;
     const long long NB = (g.m_out + kFeat - 1) / kFeat;

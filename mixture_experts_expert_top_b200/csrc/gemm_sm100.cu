@@ -612,7 +612,7 @@ cudaError_t run_bf16(const GemmArgs &g, cudaStream_t s) {
               make_token_map(&tb, g, kBoxN);
     if (!ok) return cudaErrorInvalidValue;
     auto kern = grouped_gemm_kernel<BN, STAGES, SWIGLU, KSUB>;
-    cudaError_t st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    cudaError_t st = ensure_dynamic_smem(kern, C::kSmemBytes);
     if (st != cudaSuccess) return st;
     const int grid = grid_for(g, BN);
     if (grid <= 0) return cudaSuccess;
@@ -630,7 +630,7 @@ cudaError_t run_int4(const GemmArgs &g, cudaStream_t s) {
               make_token_map(&tb, g, kBoxN);
     if (!ok) return cudaErrorInvalidValue;
     auto kern = grouped_gemm_int4_kernel<BN, STAGES, SWIGLU, GROUPS>;
-    cudaError_t st = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    cudaError_t st = ensure_dynamic_smem(kern, C::kSmemBytes);
     if (st != cudaSuccess) return st;
     const int grid = grid_for(g, BN);
     if (grid <= 0) return cudaSuccess;

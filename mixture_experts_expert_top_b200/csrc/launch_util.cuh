@@ -16,6 +16,8 @@
 
 #include <cuda_runtime.h>
 
+#include <map>
+#include <mutex>
 #include <utility>
 
 namespace moe {
@@ -24,6 +26,24 @@ __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wa
 
 __device__ __forceinline__ void griddep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) once per kernel, device and
+// size: it is a driver call that would otherwise run on every launch.
+template <typename... KArgs>
+inline cudaError_t ensure_dynamic_smem(void (*kernel)(KArgs...), size_t bytes) {
+    static std::mutex mu;
+    static std::map<std::pair<const void *, int>, size_t> done;
+    int dev = 0;
+    cudaError_t st = cudaGetDevice(&dev);
+    if (st != cudaSuccess) return st;
+    const auto key = std::make_pair(reinterpret_cast<const void *>(kernel), dev);
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = done.find(key);
+    if (it != done.end() && it->second >= bytes) return cudaSuccess;
+    st = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+    if (st == cudaSuccess) done[key] = bytes;
+    return st;
 }
 
 template <typename... KArgs, typename... Args>

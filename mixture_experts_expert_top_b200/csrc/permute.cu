@@ -181,8 +181,7 @@ cudaError_t launch_permute(const int32_t *ids, int P, int E, int32_t *counts, in
     cudaError_t st;
     if (P <= kSingleMax) {
         const size_t sm = (static_cast<size_t>(kThreads / 32) * E + 2 * E) * sizeof(int);
-        st = cudaFuncSetAttribute(permute_single_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                  static_cast<int>(sm));
+        st = ensure_dynamic_smem(permute_single_kernel, sm);
         if (st != cudaSuccess) return st;
         return launch_pdl(permute_single_kernel, dim3(1), dim3(kThreads), sm, s, ids, P, E, counts, offsets, perm,
                           inv_perm, err);
@@ -191,11 +190,9 @@ cudaError_t launch_permute(const int32_t *ids, int P, int E, int32_t *counts, in
     int32_t *chunk_hist = static_cast<int32_t *>(scratch);
     const size_t sm_hist = static_cast<size_t>(kChunkThreads / 32) * E * sizeof(int);
     const size_t sm_scatter = (static_cast<size_t>(kChunkThreads / 32) * E + E) * sizeof(int);
-    st = cudaFuncSetAttribute(permute_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(sm_hist));
+    st = ensure_dynamic_smem(permute_count_kernel, sm_hist);
     if (st != cudaSuccess) return st;
-    st = cudaFuncSetAttribute(permute_scatter_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              static_cast<int>(sm_scatter));
+    st = ensure_dynamic_smem(permute_scatter_kernel, sm_scatter);
     if (st != cudaSuccess) return st;
     if ((st = launch_pdl(permute_count_kernel, dim3(nchunks), dim3(kChunkThreads), sm_hist, s, ids, P, E, chunk_hist,
                          err)) != cudaSuccess)

@@ -51,8 +51,7 @@ template <int PER_LANE>
 cudaError_t launch_t(const float *logits, int T, int E, int k, int32_t *ids, float *w, int32_t *counts,
                      int32_t *offsets, int32_t *perm, int32_t *inv_perm, int *err, cudaStream_t s) {
     const size_t sm = (static_cast<size_t>(kThreads / 32 + 2) * E + static_cast<size_t>(T) * k) * sizeof(int);
-    const cudaError_t st = cudaFuncSetAttribute(route_permute_kernel<PER_LANE>,
-                                                cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm));
+    const cudaError_t st = ensure_dynamic_smem(route_permute_kernel<PER_LANE>, sm);
     if (st != cudaSuccess) return st;
     return launch_pdl(route_permute_kernel<PER_LANE>, dim3(1), dim3(kThreads), sm, s, logits, T, E, k, ids, w,
                       counts, offsets, perm, inv_perm, err);
