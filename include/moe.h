@@ -118,7 +118,8 @@ MOE_API moe_status_t moe_permute(const int32_t *topk_ids, const moe_shape_t *sha
  *   w_gu    MOE_W_BF16: [E,2I,H] bf16, rows [0,I) gate, rows [I,2I) up.
  *           MOE_W_INT4_G128: [E,2I,H/2] bytes, low nibble = even K index,
  *           two's complement int4; w_gu_scales [E,2I,H/128] bf16.
- *           w = bf16(q * scale) is formed in shared memory before the MMA.
+ *           w = bf16(q * scale) is formed on chip (in tensor memory, the
+ *           MMA's A operand) before the MMA; it never reaches HBM.
  *   act     [T*top_k,I] bf16 out: act = bf16(silu(g) * u), g/u fp32 accumulated.
  * Experts with no rows cost no tiles. */
 MOE_API moe_status_t moe_grouped_gemm_swiglu(const moe_bf16_t *a, const int32_t *perm, const int32_t *offsets,
@@ -167,8 +168,8 @@ MOE_API moe_status_t moe_forward_host(const moe_bf16_t *hidden_host, const float
                               const moe_shape_t *shape, moe_bf16_t *out_host,
                               void *ws, size_t ws_bytes, moe_stream_t stream);
 
-/* W4A16 weight decoding on its own (the step the int4 GEMMs run in shared
- * memory). FlashInfer PR #7196 analysis §2-§3.
+/* W4A16 weight decoding on its own (the step the int4 GEMMs run on chip
+ * before their MMAs). FlashInfer PR #7196 analysis §2-§3.
  *   q [rows, K/2] bytes, scales [rows, K/128] bf16 -> out [rows, K] bf16,
  *   out = bf16_rne(q * scale). K a multiple of 128. */
 MOE_API moe_status_t moe_dequant_int4(const uint8_t *q, const moe_bf16_t *scales, int32_t rows, int32_t K,
