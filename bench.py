@@ -228,8 +228,9 @@ def work_per_step(cfg, counts):
 
 
 def launches_per_step(cfg) -> int:
-    P = cfg.T * cfg.k
-    return 1 + (1 if P <= 8192 else 3) + 1 + 2 + 1   # route, permute, gather, 2 GEMMs, finalize
+    """Kernels one moe_forward call enqueues for this workload (the library's own count)."""
+    import mixture_experts_expert_top_b200 as moe
+    return moe.moe_forward_kernel_count(moe.Shape.of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.fmt))
 
 
 # ------------------------------------------------------------------ our arm --

@@ -150,6 +150,10 @@ MOE_API moe_status_t moe_finalize(const moe_bf16_t *y, const float *topk_w, cons
  * synchronisation.
  *   hidden [T,H] bf16, logits [T,E] fp32, weights as above, out [T,H] bf16.
  *   ws: at least moe_workspace_size(shape) bytes, 256-byte aligned. */
+/* Number of kernels moe_forward enqueues for this shape (0 when T = 0, -1
+ * when the shape is invalid). Host-side only; launches nothing. */
+MOE_API int32_t moe_forward_kernel_count(const moe_shape_t *shape);
+
 MOE_API moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits,
                          const void *w_gu, const moe_bf16_t *w_gu_scales,
                          const void *w_d, const moe_bf16_t *w_d_scales,

@@ -24,7 +24,8 @@ __all__ = [
     "moe_workspace_size", "moe_permute_workspace_size", "moe_forward_host_workspace_size",
     "moe_route", "moe_permute", "moe_grouped_gemm_swiglu", "moe_grouped_gemm_down",
     "moe_finalize", "moe_forward", "moe_forward_host", "moe_dequant_int4",
-    "moe_get_device_error", "moe_status_string", "moe_permute_noalloc", "moe_selftest_bounded_wait", "forward",
+    "moe_get_device_error", "moe_status_string", "moe_permute_noalloc", "moe_selftest_bounded_wait", "moe_forward_kernel_count",
+    "forward",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -86,6 +87,7 @@ def lib() -> ctypes.CDLL:
             "moe_permute_noalloc": ([vp, sp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
             "moe_get_device_error": ([ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
             "moe_selftest_bounded_wait": ([ctypes.c_int64, vp], ctypes.c_int),
+            "moe_forward_kernel_count": ([sp], ctypes.c_int32),
             "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
         }
         for name, (args, res) in sigs.items():
@@ -199,6 +201,10 @@ def moe_forward_host(hidden_host, logits_host, w_gu, w_gu_scales, w_d, w_d_scale
 
 def moe_dequant_int4(q, scales, rows: int, K: int, out, stream=None) -> None:
     _check(lib().moe_dequant_int4(_p(q), _p(scales), int(rows), int(K), _p(out), _s(stream)), "moe_dequant_int4")
+
+
+def moe_forward_kernel_count(shape) -> int:
+    return int(lib().moe_forward_kernel_count(ctypes.byref(_shape(shape))))
 
 
 def moe_selftest_bounded_wait(limit_ns: int, stream=None) -> None:

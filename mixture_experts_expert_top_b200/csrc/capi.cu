@@ -259,6 +259,20 @@ moe_status_t moe_finalize(const moe_bf16_t *y, const float *topk_w, const int32_
                                             static_cast<cudaStream_t>(stream)));
 }
 
+int32_t moe_forward_kernel_count(const moe_shape_t *shape) {
+    if (check_shape(shape) != MOE_OK) return -1;
+    if (shape->T == 0) return 0;
+    const int T = shape->T, k = shape->top_k, E = shape->E;
+    const long long P = static_cast<long long>(T) * k;
+    int32_t n = 0;
+    if (moe::route_permute_fusable(T, E, k))
+        n += 1;                                                       // route + permute in one CTA
+    else
+        n += 1 + (moe::permute_scratch_bytes(P, E) == 0 ? 1 : 3);     // route; permute in 1 or 3 kernels
+    if (!moe::gemm_gathers_in_kernel(static_cast<int>(P), E, shape->fmt)) n += 1;   // gather
+    return n + 3;                                                     // gate/up, down, finalize
+}
+
 moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits, const void *w_gu,
                          const moe_bf16_t *w_gu_scales, const void *w_d, const moe_bf16_t *w_d_scales,
                          const moe_shape_t *shape, moe_bf16_t *out, void *ws, size_t ws_bytes,

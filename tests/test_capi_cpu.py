@@ -7,6 +7,7 @@ import re
 
 import pytest
 
+import moe_synth
 import mixture_experts_expert_top_b200 as moe
 from mixture_experts_expert_top_b200 import build as moe_build
 
@@ -117,3 +118,16 @@ def test_empty_batch_is_a_no_op():
     assert L.moe_permute(None, byref(sh), None, None, None, None, None, None, None, 0, None) == 0
     assert L.moe_forward(None, None, None, None, None, None, byref(sh), None, None, 0, None) == 0
     assert L.moe_finalize(None, None, None, byref(sh), None, None) == 0
+
+
+def test_forward_kernel_count():
+    # one-CTA route+permute for T <= 64; the decode-shaped gate/up gathers its
+    # own rows; prefill shapes add the three bucketing kernels and the gather
+    count = lambda c: moe.moe_forward_kernel_count(moe.Shape.of(c.T, c.H, c.I, c.E, c.k, c.fmt))
+    assert count(moe_synth.get_config("qwen3_decode")) == 4
+    assert count(moe_synth.get_config("tiny")) == 4
+    assert count(moe_synth.get_config("w4a16_decode")) == 5
+    assert count(moe_synth.get_config("qwen3_prefill")) == 8
+    assert count(moe_synth.get_config("skewed")) == 8
+    assert count(moe_synth.get_config("tiny", T=0)) == 0
+    assert moe.moe_forward_kernel_count(moe.Shape.of(16, 128, 64, 8, 9)) == -1     # k > E
