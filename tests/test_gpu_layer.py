@@ -168,6 +168,61 @@ def test_back_to_back_calls_with_different_routing(name):
         assert torch.equal(o.view(torch.int16), ref.view(torch.int16)), f"call {i}"
 
 
+def _capture_forward(L, out):
+    """moe_forward captured in a CUDA graph (programmatic launches become
+    programmatic edges of the graph)."""
+    try:
+        g = torch.cuda.CUDAGraph(keep_graph=True)
+    except TypeError:
+        g = torch.cuda.CUDAGraph()
+    d = L.d
+    with torch.cuda.graph(g):
+        moe.moe_forward(d["hidden"], d["logits"], d["w_gu"], d.get("w_gu_scales"), d["w_d"], d.get("w_d_scales"),
+                        L.shape, out, L.ws, torch.cuda.current_stream())
+    return g
+
+
+@pytest.mark.parametrize("name", ["qwen3_decode", "qwen3_prefill"])
+def test_forward_replays_from_a_cuda_graph(name):
+    cfg = moe_synth.get_config(name, **({"T": 1024} if name == "qwen3_prefill" else {}))
+    L = Layer(cfg)
+    ref = L.forward().clone()
+    out = torch.zeros_like(ref)
+    g = _capture_forward(L, out)
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    # new tokens copied into the captured input buffers: the replay routes them afresh
+    h2, l2 = moe_synth.gen_hidden(cfg, seed=9), moe_synth.gen_logits(cfg, seed=9)
+    L.d["hidden"].copy_(h2)
+    L.d["logits"].copy_(l2)
+    g.replay()
+    torch.cuda.synchronize()
+    L2 = Layer.__new__(Layer)
+    L2.cfg, L2.shape, L2.ws = cfg, L.shape, torch.empty_like(L.ws)
+    L2.inp = dict(L.inp, hidden=h2, logits=l2)
+    L2.d = dict(L.d)
+    assert torch.equal(out.view(torch.int16), L2.steps()["out"].view(torch.int16))
+
+
+def test_captured_forward_has_the_advertised_number_of_kernels():
+    cudart = pytest.importorskip("cuda.bindings.runtime")
+    L = Layer(moe_synth.get_config("qwen3_decode"))
+    L.forward()
+    out = torch.empty(L.cfg.T, L.cfg.H, dtype=torch.bfloat16, device=DEV)
+    g = _capture_forward(L, out)
+    try:
+        raw = g.raw_cuda_graph()
+    except Exception as e:      # noqa: BLE001 - torch without the raw handle
+        pytest.skip(f"no raw CUDA graph handle: {e}")
+    err, _, n = cudart.cudaGraphGetNodes(cudart.cudaGraph_t(init_value=int(raw)), 0)
+    assert err == cudart.cudaError_t.cudaSuccess
+    err, nodes, n = cudart.cudaGraphGetNodes(cudart.cudaGraph_t(init_value=int(raw)), n)
+    kinds = [cudart.cudaGraphNodeGetType(nd)[1] for nd in nodes]
+    kernels = sum(k == cudart.cudaGraphNodeType.cudaGraphNodeTypeKernel for k in kinds)
+    assert kernels == moe.moe_forward_kernel_count(L.shape) == 4
+
+
 def test_forward_host_matches_forward():
     L = Layer(moe_synth.get_config("qwen3_decode"))
     ref = L.forward()
