@@ -53,7 +53,8 @@ typedef enum {
     MOE_ERR_UNSUPPORTED = 2,          /* valid but outside this build's limits */
     MOE_ERR_WORKSPACE_TOO_SMALL = 3,  /* ws_bytes below the matching *_workspace_size */
     MOE_ERR_CUDA = 4,                 /* a CUDA runtime/driver call failed */
-    MOE_ERR_DEVICE_FLAG = 5           /* a kernel raised the device error flag */
+    MOE_ERR_DEVICE_FLAG = 5           /* reserved: kernels report through the device error
+                                         flag, which moe_get_device_error() reads */
 } moe_status_t;
 
 typedef enum {
