@@ -315,15 +315,20 @@ def run_ours(args, rank, world, local):
     offsets = torch.empty(cfg.E + 1, **i32)
     perm = torch.empty(P, **i32)
     inv = torch.empty(P, **i32)
-    hp = torch.empty(P, cfg.H, dtype=torch.bfloat16, device=dev)
+    # the same gate/up kernel as moe_forward: rows read through perm, or a gathered copy
+    in_gemm = moe.moe_forward_gathers_in_gemm(shape)
+    hp = None if in_gemm else torch.empty(P, cfg.H, dtype=torch.bfloat16, device=dev)
     act = torch.empty(P, cfg.I, dtype=torch.bfloat16, device=dev)
     y = torch.empty(P, cfg.H, dtype=torch.bfloat16, device=dev)
     pws = torch.empty(max(1, moe.moe_permute_workspace_size(shape)), dtype=torch.uint8, device=dev)
     stages = ["route", "permute", "gemm_swiglu", "gemm_down", "finalize"]
     calls = [
         lambda: moe.moe_route(d["logits"], shape, ids, wts, stream),
-        lambda: moe.moe_permute(ids, shape, counts, offsets, perm, inv, d["hidden"], hp, pws, stream),
-        lambda: moe.moe_grouped_gemm_swiglu(hp, None, offsets, d["w_gu"], scales[0], shape, act, stream),
+        (lambda: moe.moe_permute(ids, shape, counts, offsets, perm, inv, None, None, pws, stream)) if in_gemm else
+        (lambda: moe.moe_permute(ids, shape, counts, offsets, perm, inv, d["hidden"], hp, pws, stream)),
+        (lambda: moe.moe_grouped_gemm_swiglu(d["hidden"], perm, offsets, d["w_gu"], scales[0], shape, act, stream))
+        if in_gemm else
+        (lambda: moe.moe_grouped_gemm_swiglu(hp, None, offsets, d["w_gu"], scales[0], shape, act, stream)),
         lambda: moe.moe_grouped_gemm_down(act, offsets, d["w_d"], scales[1], shape, y, stream),
         lambda: moe.moe_finalize(y, wts, inv, shape, out, stream),
     ]

@@ -155,6 +155,12 @@ MOE_API moe_status_t moe_finalize(const moe_bf16_t *y, const float *topk_w, cons
  * when the shape is invalid). Host-side only; launches nothing. */
 MOE_API int32_t moe_forward_kernel_count(const moe_shape_t *shape);
 
+/* 1 when moe_forward's gate/up GEMM reads the token rows through perm itself
+ * (no gathered copy is written), 0 when it gathers first, -1 for an invalid
+ * shape. The same choice for moe_grouped_gemm_swiglu with a non-NULL perm
+ * runs the kernel moe_forward runs. Host-side only. */
+MOE_API int32_t moe_forward_gathers_in_gemm(const moe_shape_t *shape);
+
 MOE_API moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits,
                          const void *w_gu, const moe_bf16_t *w_gu_scales,
                          const void *w_d, const moe_bf16_t *w_d_scales,

@@ -24,7 +24,7 @@ __all__ = [
     "moe_workspace_size", "moe_permute_workspace_size", "moe_forward_host_workspace_size",
     "moe_route", "moe_permute", "moe_grouped_gemm_swiglu", "moe_grouped_gemm_down",
     "moe_finalize", "moe_forward", "moe_forward_host", "moe_dequant_int4",
-    "moe_get_device_error", "moe_status_string", "moe_permute_noalloc", "moe_selftest_bounded_wait", "moe_forward_kernel_count",
+    "moe_get_device_error", "moe_status_string", "moe_permute_noalloc", "moe_selftest_bounded_wait", "moe_forward_kernel_count", "moe_forward_gathers_in_gemm",
     "forward",
 ]
 
@@ -88,6 +88,7 @@ def lib() -> ctypes.CDLL:
             "moe_get_device_error": ([ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
             "moe_selftest_bounded_wait": ([ctypes.c_int64, vp], ctypes.c_int),
             "moe_forward_kernel_count": ([sp], ctypes.c_int32),
+            "moe_forward_gathers_in_gemm": ([sp], ctypes.c_int32),
             "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
         }
         for name, (args, res) in sigs.items():
@@ -205,6 +206,13 @@ def moe_dequant_int4(q, scales, rows: int, K: int, out, stream=None) -> None:
 
 def moe_forward_kernel_count(shape) -> int:
     return int(lib().moe_forward_kernel_count(ctypes.byref(_shape(shape))))
+
+
+def moe_forward_gathers_in_gemm(shape) -> bool:
+    v = int(lib().moe_forward_gathers_in_gemm(ctypes.byref(_shape(shape))))
+    if v < 0:
+        raise MoeError(1, "moe_forward_gathers_in_gemm: invalid shape")
+    return v == 1
 
 
 def moe_selftest_bounded_wait(limit_ns: int, stream=None) -> None:

@@ -273,6 +273,11 @@ int32_t moe_forward_kernel_count(const moe_shape_t *shape) {
     return n + 3;                                                     // gate/up, down, finalize
 }
 
+int32_t moe_forward_gathers_in_gemm(const moe_shape_t *shape) {
+    if (check_shape(shape) != MOE_OK) return -1;
+    return moe::gemm_gathers_in_kernel(shape->T * shape->top_k, shape->E, shape->fmt) ? 1 : 0;
+}
+
 moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits, const void *w_gu,
                          const moe_bf16_t *w_gu_scales, const void *w_d, const moe_bf16_t *w_d_scales,
                          const moe_shape_t *shape, moe_bf16_t *out, void *ws, size_t ws_bytes,

@@ -121,13 +121,18 @@ def test_empty_batch_is_a_no_op():
 
 
 def test_forward_kernel_count():
-    # one-CTA route+permute for T <= 64; the decode-shaped gate/up gathers its
-    # own rows; prefill shapes add the three bucketing kernels and the gather
-    count = lambda c: moe.moe_forward_kernel_count(moe.Shape.of(c.T, c.H, c.I, c.E, c.k, c.fmt))
+    # one-CTA route+permute for T <= 64; the decode-shaped gate/up reads its
+    # token rows through perm; prefill shapes add the three bucketing kernels
+    # and the gather
+    sh = lambda c: moe.Shape.of(c.T, c.H, c.I, c.E, c.k, c.fmt)
+    count = lambda c: moe.moe_forward_kernel_count(sh(c))
     assert count(moe_synth.get_config("qwen3_decode")) == 4
     assert count(moe_synth.get_config("tiny")) == 4
     assert count(moe_synth.get_config("w4a16_decode")) == 5
     assert count(moe_synth.get_config("qwen3_prefill")) == 8
     assert count(moe_synth.get_config("skewed")) == 8
+    assert moe.moe_forward_gathers_in_gemm(sh(moe_synth.get_config("qwen3_decode")))
+    assert moe.moe_forward_gathers_in_gemm(sh(moe_synth.get_config("w4a16_decode")))
+    assert not moe.moe_forward_gathers_in_gemm(sh(moe_synth.get_config("qwen3_prefill")))
     assert count(moe_synth.get_config("tiny", T=0)) == 0
     assert moe.moe_forward_kernel_count(moe.Shape.of(16, 128, 64, 8, 9)) == -1     # k > E

@@ -233,12 +233,14 @@ def test_grouped_gemm_swiglu_and_down_match_oracle(cfg):
     gemm_rows_close(bf16_bits(y), r["y"], "y")
 
 
-@pytest.mark.parametrize("cfg", [GEMM_CFGS[1], GEMM_CFGS[2], GEMM_CFGS[3], GEMM_CFGS[5],
+@pytest.mark.parametrize("cfg", [GEMM_CFGS[1], GEMM_CFGS[2], GEMM_CFGS[3], GEMM_CFGS[5], GEMM_CFGS[6], GEMM_CFGS[7],
+                                 moe_synth.get_config("qwen3_prefill", T=3000, H=1024, I=512, E=6, k=2),
                                  moe_synth.MoeConfig("int4_gather", T=48, H=1024, I=384, E=12, k=4, fmt="int4_g128")],
                          ids=lambda c: f"T{c.T}H{c.H}I{c.I}E{c.E}k{c.k}{c.fmt}")
 def test_grouped_gemm_swiglu_gathers_through_perm(cfg):
-    """perm given: the GEMM reads hidden rows through perm (TMA gather4) and
-    must give the same act as from the materialised permuted rows."""
+    """perm given: the GEMM reads hidden rows through perm (TMA gather4; at
+    CTA-pair shapes the single-CTA kernel takes the call) and must give the
+    same act as from the materialised permuted rows."""
     inp, r, hp = gemm_case(cfg)
     sh = moe.Shape.of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.fmt)
     offsets = dev(r["offsets"], torch.int32)
