@@ -268,7 +268,7 @@ int32_t moe_forward_kernel_count(const moe_shape_t *shape) {
     if (moe::route_permute_fusable(T, E, k))
         n += 1;                                                       // route + permute in one CTA
     else
-        n += 1 + (moe::permute_scratch_bytes(P, E) == 0 ? 1 : 3);     // route; permute in 1 or 3 kernels
+        n += 1 + moe::permute_kernel_count(P, E);                     // route; permute in 1, 2 or 3 kernels
     if (!moe::gemm_gathers_in_kernel(static_cast<int>(P), E, shape->fmt)) n += 1;   // gather
     return n + 3;                                                     // gate/up, down, finalize
 }

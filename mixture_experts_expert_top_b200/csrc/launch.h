@@ -37,6 +37,8 @@ cudaError_t launch_route_permute(const float *logits, int T, int E, int k, int32
 // Scratch bytes the permute needs for P pairs over E experts (0 when a
 // single CTA handles all pairs).
 size_t permute_scratch_bytes(long long P, int E);
+// Kernels launch_permute enqueues for P pairs over E experts (1, 2 or 3).
+int permute_kernel_count(long long P, int E);
 cudaError_t launch_permute(const int32_t *ids, int P, int E, int32_t *counts, int32_t *offsets, int32_t *perm,
                            int32_t *inv_perm, void *scratch, int *err, cudaStream_t s);
 cudaError_t launch_gather(const uint16_t *hidden, const int32_t *perm, int P, int H, int k, uint16_t *hidden_perm,

@@ -118,6 +118,66 @@ permute_scan_kernel(int nchunks, int E, int32_t *__restrict__ chunk_hist, int32_
     }
 }
 
+// Multi-CTA passes 2 and 3 in one kernel, for few chunks (E <= the CTA's
+// threads): every CTA derives its chunk's first rows from all the chunk
+// counts itself (nchunks * E ints from L2), so neither the scan CTA nor its
+// launch is needed. G threads share an expert, as in permute_scan_kernel.
+// CTA 0 also writes counts and offsets.
+constexpr int kFusedScanMaxChunks = 64;
+
+__global__ void __launch_bounds__(kChunkThreads)
+permute_scan_scatter_kernel(const int32_t *__restrict__ ids, int P, int E, int nchunks,
+                            const int32_t *__restrict__ chunk_hist, int32_t *__restrict__ counts,
+                            int32_t *__restrict__ offsets, int32_t *__restrict__ perm,
+                            int32_t *__restrict__ inv_perm) {
+    constexpr int NW = kChunkThreads / 32;
+    extern __shared__ int smem[];
+    int *hist = smem;                 // [NW * E]
+    int *tot = hist + NW * E;         // [E] rows of expert e
+    int *base = tot + E;              // [E] first row of expert e, then of this chunk's rows of e
+    int *before = base + E;           // [E] rows of expert e in the chunks before this one
+    int *offs_local = before + E;     // [E + 1] where CTAs other than 0 put the offsets
+    griddep_launch_dependents();
+    griddep_wait();
+    int G = 1;
+    while (G < 32 && 2 * G * E <= kChunkThreads) G *= 2;
+    const int e = threadIdx.x / G, part = threadIdx.x % G;
+    const bool active = e < E;
+    const int per = (nchunks + G - 1) / G;
+    const int c0 = part * per, c1 = min(nchunks, c0 + per);
+    const int me = static_cast<int>(blockIdx.x);
+    int sum = 0, pre = 0;
+    if (active) {
+        for (int c = c0; c < c1; c += 8) {
+            int v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) v[j] = c + j < c1 ? __ldcg(chunk_hist + static_cast<size_t>(c + j) * E + e) : 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                sum += v[j];
+                if (c + j < me) pre += v[j];
+            }
+        }
+    }
+    for (int o = G / 2; o > 0; o >>= 1) {      // over the G lanes of the expert (an aligned lane segment)
+        sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        pre += __shfl_xor_sync(0xffffffffu, pre, o);
+    }
+    if (active && part == 0) {
+        tot[e] = sum;
+        before[e] = pre;
+        if (me == 0) counts[e] = sum;
+    }
+    __syncthreads();
+    block_exclusive_scan<kChunkThreads>(tot, E, base, me == 0 ? offsets : offs_local);
+    for (int i = threadIdx.x; i < E; i += kChunkThreads) base[i] += before[i];
+    const int begin = me * kChunk;
+    const int n = min(kChunk, P - begin);
+    warp_histograms<NW>(ids, begin, n, E, hist, nullptr);   // its first barrier also orders base
+    warp_bases<NW>(E, hist, base);
+    warp_scatter<NW>(ids, begin, n, E, hist, perm, inv_perm);
+}
+
 // Multi-CTA pass 3: scatter each chunk from its per-expert first rows.
 __global__ void __launch_bounds__(kChunkThreads)
 permute_scatter_kernel(const int32_t *__restrict__ ids, int P, int E, const int32_t *__restrict__ chunk_base,
@@ -170,6 +230,12 @@ gather_rows_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__
 
 }  // namespace
 
+int permute_kernel_count(long long P, int E) {
+    if (P <= kSingleMax) return 1;
+    const long long nchunks = (P + kChunk - 1) / kChunk;
+    return nchunks <= kFusedScanMaxChunks && E <= kChunkThreads ? 2 : 3;
+}
+
 size_t permute_scratch_bytes(long long P, int E) {
     if (P <= kSingleMax) return 0;
     const long long nchunks = (P + kChunk - 1) / kChunk;
@@ -197,6 +263,12 @@ cudaError_t launch_permute(const int32_t *ids, int P, int E, int32_t *counts, in
     if ((st = launch_pdl(permute_count_kernel, dim3(nchunks), dim3(kChunkThreads), sm_hist, s, ids, P, E, chunk_hist,
                          err)) != cudaSuccess)
         return st;
+    if (permute_kernel_count(P, E) == 2) {
+        const size_t sm_fused = (static_cast<size_t>(kChunkThreads / 32) * E + 4 * E + 1) * sizeof(int);
+        if ((st = ensure_dynamic_smem(permute_scan_scatter_kernel, sm_fused)) != cudaSuccess) return st;
+        return launch_pdl(permute_scan_scatter_kernel, dim3(nchunks), dim3(kChunkThreads), sm_fused, s, ids, P, E,
+                          nchunks, static_cast<const int32_t *>(chunk_hist), counts, offsets, perm, inv_perm);
+    }
     if ((st = launch_pdl(permute_scan_kernel, dim3(1), dim3(kThreads), 2 * E * sizeof(int), s, nchunks, E,
                          chunk_hist, counts, offsets)) != cudaSuccess)
         return st;

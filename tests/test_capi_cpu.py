@@ -122,15 +122,16 @@ def test_empty_batch_is_a_no_op():
 
 def test_forward_kernel_count():
     # one-CTA route+permute for T <= 64; the decode-shaped gate/up reads its
-    # token rows through perm; prefill shapes add the three bucketing kernels
-    # and the gather
+    # token rows through perm; prefill shapes add two bucketing kernels (three
+    # past 64 chunks of 2048 pairs or 512 experts) and the gather
     sh = lambda c: moe.Shape.of(c.T, c.H, c.I, c.E, c.k, c.fmt)
     count = lambda c: moe.moe_forward_kernel_count(sh(c))
     assert count(moe_synth.get_config("qwen3_decode")) == 4
     assert count(moe_synth.get_config("tiny")) == 4
     assert count(moe_synth.get_config("w4a16_decode")) == 5
-    assert count(moe_synth.get_config("qwen3_prefill")) == 8
-    assert count(moe_synth.get_config("skewed")) == 8
+    assert count(moe_synth.get_config("qwen3_prefill")) == 7
+    assert count(moe_synth.get_config("skewed")) == 7
+    assert count(moe_synth.get_config("qwen3_prefill", T=20000)) == 8           # 79 chunks: separate scan
     assert moe.moe_forward_gathers_in_gemm(sh(moe_synth.get_config("qwen3_decode")))
     assert moe.moe_forward_gathers_in_gemm(sh(moe_synth.get_config("w4a16_decode")))
     assert not moe.moe_forward_gathers_in_gemm(sh(moe_synth.get_config("qwen3_prefill")))

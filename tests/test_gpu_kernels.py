@@ -109,8 +109,10 @@ def test_route_ties_go_to_the_lower_expert():
 
 # ---------------------------------------------------------------- permute --
 
+# single CTA (P <= 8192); chunk counts scanned inside the scatter CTAs (<= 64
+# chunks of 2048 pairs, E <= 512); separate scan CTA (more chunks, or E > 512)
 PERMUTE_CASES = [(16, 8, 2), (64, 128, 8), (256, 256, 8), (1024, 8, 8), (1025, 64, 8), (8192, 128, 8),
-                 (4096, 64, 6), (1, 4, 4), (3000, 1024, 3), (20000, 2, 1)]
+                 (4096, 64, 6), (1, 4, 4), (3000, 1024, 3), (20000, 2, 1), (3000, 512, 4), (20000, 64, 8)]
 
 
 @pytest.mark.parametrize("T,E,k", PERMUTE_CASES)

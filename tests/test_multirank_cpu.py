@@ -84,7 +84,7 @@ def test_bench_work_accounting():
     assert w["weight_bytes"] == 120 * 3 * 2048 * 768 * 2
     assert w["layer_flops"] == 2 * 64 * 8 * 3 * 2048 * 768
     assert bench.launches_per_step(cfg) == 4          # route+permute, gate/up (own gather), down, finalize
-    assert bench.launches_per_step(moe_synth.get_config("qwen3_prefill")) == 8
+    assert bench.launches_per_step(moe_synth.get_config("qwen3_prefill")) == 7
     q = moe_synth.get_config("w4a16_decode")
     wq = bench.work_per_step(q, [8] * 256)
     assert wq["weight_bytes"] == 256 * (2 * 2048 * (7168 // 2 + 56 * 2) + 7168 * (2048 // 2 + 16 * 2))
