@@ -50,7 +50,7 @@ extern "C" {
 typedef enum {
     MOE_OK = 0,
     MOE_ERR_INVALID_ARG = 1,          /* null pointer, bad size, misalignment */
-    MOE_ERR_UNSUPPORTED = 2,          /* valid but outside this build's limits */
+    MOE_ERR_UNSUPPORTED = 2,          /* valid but outside the library's limits */
     MOE_ERR_WORKSPACE_TOO_SMALL = 3,  /* ws_bytes below the matching *_workspace_size */
     MOE_ERR_CUDA = 4,                 /* a CUDA runtime/driver call failed */
     MOE_ERR_DEVICE_FLAG = 5           /* reserved: kernels report through the device error
