@@ -24,8 +24,8 @@ __all__ = [
     "moe_workspace_size", "moe_permute_workspace_size", "moe_forward_host_workspace_size",
     "moe_route", "moe_permute", "moe_grouped_gemm_swiglu", "moe_grouped_gemm_down",
     "moe_finalize", "moe_forward", "moe_forward_host", "moe_dequant_int4",
-    "moe_get_device_error", "moe_status_string", "moe_permute_noalloc", "moe_selftest_bounded_wait", "moe_forward_kernel_count", "moe_forward_gathers_in_gemm",
-    "forward",
+    "moe_get_device_error", "moe_status_string", "moe_permute_noalloc", "moe_selftest_bounded_wait",
+    "moe_forward_kernel_count", "moe_forward_gathers_in_gemm", "forward",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -101,12 +101,18 @@ def lib() -> ctypes.CDLL:
 
 # ---- marshalling helpers ---------------------------------------------------
 
-def _p(t) -> Optional[int]:
-    """Device (or host) address of a tensor, None for None."""
+BF16, F32, I32, U8 = torch.bfloat16, torch.float32, torch.int32, torch.uint8
+
+
+def _p(t, *dtypes) -> Optional[int]:
+    """Device (or host) address of a tensor, None for None. With dtypes, a
+    tensor of another dtype is refused (the C ABI takes untyped pointers)."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if dtypes and t.dtype not in dtypes:
+        raise TypeError(f"libmoe_b200: expected a tensor of {' or '.join(map(str, dtypes))}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError("tensors passed to libmoe_b200 must be contiguous")
     return t.data_ptr()
@@ -146,15 +152,17 @@ def moe_forward_host_workspace_size(shape) -> int:
 
 
 def moe_route(logits, shape, topk_ids, topk_w, stream=None) -> None:
-    _check(lib().moe_route(_p(logits), ctypes.byref(_shape(shape)), _p(topk_ids), _p(topk_w), _s(stream)),
+    _check(lib().moe_route(_p(logits, F32), ctypes.byref(_shape(shape)), _p(topk_ids, I32), _p(topk_w, F32),
+                           _s(stream)),
            "moe_route")
 
 
 def moe_permute(topk_ids, shape, counts, offsets, perm, inv_perm, hidden=None, hidden_perm=None,
                 ws=None, stream=None) -> None:
     nbytes = 0 if ws is None else ws.numel() * ws.element_size()
-    _check(lib().moe_permute(_p(topk_ids), ctypes.byref(_shape(shape)), _p(counts), _p(offsets), _p(perm),
-                             _p(inv_perm), _p(hidden), _p(hidden_perm), _p(ws), nbytes, _s(stream)),
+    _check(lib().moe_permute(_p(topk_ids, I32), ctypes.byref(_shape(shape)), _p(counts, I32), _p(offsets, I32),
+                             _p(perm, I32), _p(inv_perm, I32), _p(hidden, BF16), _p(hidden_perm, BF16), _p(ws),
+                             nbytes, _s(stream)),
            "moe_permute")
 
 
@@ -162,46 +170,51 @@ def moe_permute_noalloc(topk_ids, shape, counts, offsets, perm, inv_perm, hidden
                         stream=None) -> None:
     """moe_permute without a workspace: its scratch is a fixed array inside the
     library (for callers that cannot allocate device memory)."""
-    _check(lib().moe_permute_noalloc(_p(topk_ids), ctypes.byref(_shape(shape)), _p(counts), _p(offsets), _p(perm),
-                                     _p(inv_perm), _p(hidden), _p(hidden_perm), _s(stream)),
+    _check(lib().moe_permute_noalloc(_p(topk_ids, I32), ctypes.byref(_shape(shape)), _p(counts, I32),
+                                     _p(offsets, I32), _p(perm, I32), _p(inv_perm, I32), _p(hidden, BF16),
+                                     _p(hidden_perm, BF16), _s(stream)),
            "moe_permute_noalloc")
 
 
 def moe_grouped_gemm_swiglu(a, perm, offsets, w_gu, w_gu_scales, shape, act, stream=None) -> None:
-    _check(lib().moe_grouped_gemm_swiglu(_p(a), _p(perm), _p(offsets), _p(w_gu), _p(w_gu_scales),
-                                         ctypes.byref(_shape(shape)), _p(act), _s(stream)),
+    _check(lib().moe_grouped_gemm_swiglu(_p(a, BF16), _p(perm, I32), _p(offsets, I32), _p(w_gu, BF16, U8),
+                                         _p(w_gu_scales, BF16), ctypes.byref(_shape(shape)), _p(act, BF16),
+                                         _s(stream)),
            "moe_grouped_gemm_swiglu")
 
 
 def moe_grouped_gemm_down(act, offsets, w_d, w_d_scales, shape, y, stream=None) -> None:
-    _check(lib().moe_grouped_gemm_down(_p(act), _p(offsets), _p(w_d), _p(w_d_scales),
-                                       ctypes.byref(_shape(shape)), _p(y), _s(stream)),
+    _check(lib().moe_grouped_gemm_down(_p(act, BF16), _p(offsets, I32), _p(w_d, BF16, U8), _p(w_d_scales, BF16),
+                                       ctypes.byref(_shape(shape)), _p(y, BF16), _s(stream)),
            "moe_grouped_gemm_down")
 
 
 def moe_finalize(y, topk_w, inv_perm, shape, out, stream=None) -> None:
-    _check(lib().moe_finalize(_p(y), _p(topk_w), _p(inv_perm), ctypes.byref(_shape(shape)), _p(out), _s(stream)),
+    _check(lib().moe_finalize(_p(y, BF16), _p(topk_w, F32), _p(inv_perm, I32), ctypes.byref(_shape(shape)),
+                              _p(out, BF16), _s(stream)),
            "moe_finalize")
 
 
 def moe_forward(hidden, logits, w_gu, w_gu_scales, w_d, w_d_scales, shape, out, ws, stream=None) -> None:
     nbytes = ws.numel() * ws.element_size()
-    _check(lib().moe_forward(_p(hidden), _p(logits), _p(w_gu), _p(w_gu_scales), _p(w_d), _p(w_d_scales),
-                             ctypes.byref(_shape(shape)), _p(out), _p(ws), nbytes, _s(stream)),
+    _check(lib().moe_forward(_p(hidden, BF16), _p(logits, F32), _p(w_gu, BF16, U8), _p(w_gu_scales, BF16),
+                             _p(w_d, BF16, U8), _p(w_d_scales, BF16), ctypes.byref(_shape(shape)), _p(out, BF16),
+                             _p(ws), nbytes, _s(stream)),
            "moe_forward")
 
 
 def moe_forward_host(hidden_host, logits_host, w_gu, w_gu_scales, w_d, w_d_scales, shape, out_host, ws,
                      stream=None) -> None:
     nbytes = ws.numel() * ws.element_size()
-    _check(lib().moe_forward_host(_p(hidden_host), _p(logits_host), _p(w_gu), _p(w_gu_scales), _p(w_d),
-                                  _p(w_d_scales), ctypes.byref(_shape(shape)), _p(out_host), _p(ws), nbytes,
-                                  _s(stream)),
+    _check(lib().moe_forward_host(_p(hidden_host, BF16), _p(logits_host, F32), _p(w_gu, BF16, U8),
+                                  _p(w_gu_scales, BF16), _p(w_d, BF16, U8), _p(w_d_scales, BF16),
+                                  ctypes.byref(_shape(shape)), _p(out_host, BF16), _p(ws), nbytes, _s(stream)),
            "moe_forward_host")
 
 
 def moe_dequant_int4(q, scales, rows: int, K: int, out, stream=None) -> None:
-    _check(lib().moe_dequant_int4(_p(q), _p(scales), int(rows), int(K), _p(out), _s(stream)), "moe_dequant_int4")
+    _check(lib().moe_dequant_int4(_p(q, U8), _p(scales, BF16), int(rows), int(K), _p(out, BF16), _s(stream)),
+           "moe_dequant_int4")
 
 
 def moe_forward_kernel_count(shape) -> int:

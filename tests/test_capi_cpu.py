@@ -137,3 +137,15 @@ def test_forward_kernel_count():
     assert not moe.moe_forward_gathers_in_gemm(sh(moe_synth.get_config("qwen3_prefill")))
     assert count(moe_synth.get_config("tiny", T=0)) == 0
     assert moe.moe_forward_kernel_count(moe.Shape.of(16, 128, 64, 8, 9)) == -1     # k > E
+
+
+def test_binding_refuses_tensors_of_the_wrong_dtype():
+    # checked in the binding before the library is called: no GPU needed
+    import torch
+    sh = moe.Shape.of(4, 128, 64, 8, 2)
+    f32 = torch.zeros(4, 8)
+    with pytest.raises(TypeError):
+        moe.moe_route(f32.to(torch.float64), sh, torch.zeros(4, 2, dtype=torch.int32), torch.zeros(4, 2))
+    with pytest.raises(TypeError):
+        moe.moe_finalize(torch.zeros(8, 128), torch.zeros(4, 2), torch.zeros(8, dtype=torch.int32), sh,
+                         torch.zeros(4, 128, dtype=torch.bfloat16))

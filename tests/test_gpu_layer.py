@@ -269,5 +269,6 @@ def test_zero_inputs_give_zero_output():
 def test_empty_batch():
     cfg = moe_synth.get_config("tiny", T=0)
     sh = moe.Shape.of(0, cfg.H, cfg.I, cfg.E, cfg.k)
-    moe.moe_forward(torch.empty(0, device=DEV), torch.empty(0, device=DEV), torch.empty(0, device=DEV), None,
-                    torch.empty(0, device=DEV), None, sh, torch.empty(0, device=DEV), torch.empty(1, device=DEV))
+    bf = dict(dtype=torch.bfloat16, device=DEV)
+    moe.moe_forward(torch.empty(0, **bf), torch.empty(0, device=DEV), torch.empty(0, **bf), None,
+                    torch.empty(0, **bf), None, sh, torch.empty(0, **bf), torch.empty(1, dtype=torch.uint8, device=DEV))
