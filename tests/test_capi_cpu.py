@@ -149,3 +149,50 @@ def test_binding_refuses_tensors_of_the_wrong_dtype():
     with pytest.raises(TypeError):
         moe.moe_finalize(torch.zeros(8, 128), torch.zeros(4, 2), torch.zeros(8, dtype=torch.int32), sh,
                          torch.zeros(4, 128, dtype=torch.bfloat16))
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "moe.h"
+
+int main(void) {
+    moe_shape_t s;
+    s.T = 64; s.H = 2048; s.I = 768; s.E = 128; s.top_k = 8; s.fmt = MOE_W_BF16;
+    size_t ws = moe_workspace_size(&s);
+    moe_shape_t bad = s;
+    bad.top_k = 129;
+    int rc = 0;
+    if (ws == 0) rc = 1;
+    if (moe_workspace_size(&bad) != 0) rc = 2;
+    if (moe_forward_kernel_count(&s) != 4) rc = 3;
+    if (strcmp(moe_status_string(MOE_OK), "ok") != 0) rc = 4;
+    /* T = 0 enqueues nothing and succeeds without a GPU */
+    s.T = 0;
+    if (moe_forward(NULL, NULL, NULL, NULL, NULL, NULL, &s, NULL, NULL, 0, NULL) != MOE_OK) rc = 5;
+    printf("%zu %d\n", ws, rc);
+    return rc;
+}
+"""
+
+
+def test_the_header_compiles_as_c99_and_a_c_program_links_and_runs(tmp_path):
+    # the boundary is a C ABI: plain C must be able to include moe.h, link
+    # libmoe_b200.so and call the host-side entry points (no GPU needed)
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no gcc")
+    moe_build.build()
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    inc = os.path.join(os.path.dirname(os.path.dirname(moe.__file__)), "include")
+    libdir = os.path.dirname(moe.library_path)
+    r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", inc, str(src), "-o", str(exe),
+                        "-L", libdir, "-l:libmoe_b200.so", f"-Wl,-rpath,{libdir}"],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0, (r.stdout, r.stderr)
+    assert int(r.stdout.split()[0]) > 0
