@@ -196,3 +196,25 @@ def test_the_header_compiles_as_c99_and_a_c_program_links_and_runs(tmp_path):
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, (r.stdout, r.stderr)
     assert int(r.stdout.split()[0]) > 0
+
+
+@pytest.mark.parametrize("shape,status", [
+    ((16, 128, 64, 8, 9, 0), 1),            # k > E: invalid
+    ((16, 128, 64, 0, 1, 0), 1),            # E = 0: invalid
+    ((16, 128, 64, 8, 2, 7), 1),            # unknown format: invalid
+    ((16, 128, 64, 2048, 2, 0), 2),         # E > 1024: outside the library's limits
+    ((16, 128, 64, 64, 33, 0), 2),          # k > 32
+    ((16, 130, 64, 8, 2, 0), 2),            # H not a multiple of 8
+    ((16, 192, 128, 8, 2, 1), 2),           # int4 needs H % 128 == 0
+    ((300_000_000, 128, 64, 16, 8, 0), 2),  # T * k >= 2^31
+])
+def test_shape_checks_return_the_documented_status(shape, status):
+    L = moe.lib()
+    assert L.moe_route(16, ctypes.byref(moe.Shape.of(*shape)), 16, 16, None) == status
+
+
+def test_noalloc_permute_refuses_shapes_beyond_its_scratch_before_any_launch():
+    # ceil(600000 / 2048) = 293 chunks x 1024 experts > 65536 scratch entries
+    L = moe.lib()
+    sh = moe.Shape.of(600000, 8, 8, 1024, 1)
+    assert L.moe_permute_noalloc(16, ctypes.byref(sh), 16, 16, 16, 16, None, None, None) == 2
