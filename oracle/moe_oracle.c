@@ -31,9 +31,9 @@
  * each entry point that does fp32 arithmetic.
  *
  * Readings of points the sources leave open (each also stated where used):
- *  R1 top-k selects on the softmax probabilities (monotone in the logits);
- *     equal probabilities go to the lower expert id; slot order is
- *     descending probability.
+ *  R1 top-k selects on the fp32 logits (softmax is monotone in them): slot
+ *     order is descending logit, equal logits go to the lower expert id,
+ *     -0 equals +0 and NaN ranks as -inf.
  *  R2 weights are renormalised over the k selected experts.
  *  R3 rows [0,I) of W_gu[e] are the gate projection and rows [I,2I) the up
  *     projection.
@@ -112,40 +112,61 @@ void oracle_set_num_threads(int n) {
 }
 
 /* ---- step 1: routing ------------------------------------------------------
- * Softmax over all E logits, keep the k most probable experts (R1), then
+ * Keep the k experts with the largest softmax probabilities (R1), then
  * renormalise their probabilities to sum to one (R2). InfiniLM PR #500 §2.1,
  * §2.4 (op::topksoftmax); the renormalisation is Qwen3's norm_topk_prob.
+ *
+ * Softmax is strictly increasing in the logit, so the k most probable experts
+ * are the k largest fp32 logits; the selection compares the logits as given,
+ * never a rounded probability (two distinct logits can round to the same
+ * probability in any finite precision). Equal logits go to the lower expert
+ * id; -0 equals +0, as in IEEE comparison; a NaN logit ranks as -inf.
+ * The weights are exp(l_j - l_0) / sum_{i<k} exp(l_i - l_0) in double, l_0 the
+ * largest logit: the full-softmax denominator cancels in the renormalisation.
  * Returns 0, or -1 on bad sizes.
  */
+
+/* The value a logit ranks with: NaN as -inf, -0 as +0. */
+static double rank_value(float l) {
+    if (l != l) return -INFINITY;
+    if (l == 0.0f) return 0.0;
+    return (double)l;
+}
+
+/* Does expert a come before expert b (larger logit, then lower id)? */
+static int ranks_before(const float *l, int a, int b) {
+    double va = rank_value(l[a]), vb = rank_value(l[b]);
+    if (va != vb) return va > vb;
+    return a < b;
+}
+
 int oracle_route(const float *logits, int T, int E, int k, int32_t *ids, float *w) {
     if (T < 0 || E < 1 || k < 1 || k > E) return -1;
     int bad = 0;
 #pragma omp parallel for schedule(static)
     for (int t = 0; t < T; ++t) {
         const float *l = logits + (size_t)t * E;
-        double *p = (double *)malloc(sizeof(double) * (size_t)E);
+        int32_t *id = ids + (size_t)t * k;
         char *taken = (char *)calloc((size_t)E, 1);
-        if (!p || !taken) { bad = 1; free(p); free(taken); continue; }
-        double m = -INFINITY;
-        for (int e = 0; e < E; ++e) if ((double)l[e] > m) m = (double)l[e];
-        double z = 0.0;
-        for (int e = 0; e < E; ++e) { p[e] = exp((double)l[e] - m); z += p[e]; }
-        for (int e = 0; e < E; ++e) p[e] /= z;
-        double s = 0.0;
+        double *p = (double *)malloc(sizeof(double) * (size_t)k);
+        if (!taken || !p) { bad = 1; free(taken); free(p); continue; }
+        /* selection: k passes, each takes the first expert in rank order */
         for (int j = 0; j < k; ++j) {
             int best = -1;
-            for (int e = 0; e < E; ++e) {
-                if (taken[e]) continue;
-                if (best < 0 || p[e] > p[best]) best = e;   /* strict: ties keep the lower id */
-            }
+            for (int e = 0; e < E; ++e)
+                if (!taken[e] && (best < 0 || ranks_before(l, e, best))) best = e;
             taken[best] = 1;
-            ids[(size_t)t * k + j] = best;
-            s += p[best];
+            id[j] = best;
         }
-        for (int j = 0; j < k; ++j)
-            w[(size_t)t * k + j] = (float)(p[ids[(size_t)t * k + j]] / s);
-        free(p);
+        /* renormalised softmax over the selected logits, summed in slot order */
+        double l0 = rank_value(l[id[0]]), s = 0.0;
+        for (int j = 0; j < k; ++j) {
+            p[j] = exp(rank_value(l[id[j]]) - l0);
+            s += p[j];
+        }
+        for (int j = 0; j < k; ++j) w[(size_t)t * k + j] = (float)(p[j] / s);
         free(taken);
+        free(p);
     }
     return bad ? -1 : 0;
 }

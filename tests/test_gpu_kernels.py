@@ -107,6 +107,29 @@ def test_route_ties_go_to_the_lower_expert():
     assert np.array_equal(gi[6][:2], [2, 7]) and np.array_equal(gi[7][:2], [2, 7])
 
 
+@pytest.mark.parametrize("E", [6, 64, 256])
+def test_route_orders_by_logit_where_probabilities_tie(E):
+    """The rows where a rounded probability would tie distinct logits (far
+    below the max, or underflowed), NaN logits and signed zeros. Row 0 pads
+    the planted row with NaN (ranked last, after the row's own entries, by
+    id), so its ids are the hand-derived order; rows 1 and 2 put the planted
+    row in the top lanes or pad it with -1e30, and are compared with the
+    oracle."""
+    import test_oracle_pins as pins
+    for row, k, expect in pins.ROUTE_EDGE_ROWS:
+        n = len(row)
+        logits = torch.full((3, E), -1e30)
+        logits[0, :] = float("nan")
+        logits[0, :n] = torch.tensor(row)
+        logits[1, E - n:] = torch.tensor(row)
+        logits[2, :n] = torch.tensor(row)
+        gi, gw = run_route(logits, k)
+        oi, ow = oracle.route(logits, k)
+        assert np.array_equal(gi, oi), (row, gi, oi)
+        assert gi[0].tolist() == expect
+        assert np.allclose(gw, ow, rtol=2 ** -20, atol=0)
+
+
 # ---------------------------------------------------------------- permute --
 
 # single CTA (P <= 8192); chunk counts scanned inside the scatter CTAs (<= 64

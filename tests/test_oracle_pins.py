@@ -47,6 +47,41 @@ def test_route_ids_are_a_stable_descending_sort(T, E, k):
     assert np.array_equal(ids, ref.numpy().astype(np.int32))
 
 
+# Rows where the order of the logits and the order of any rounded probability
+# part ways. Softmax is strictly increasing, so the k most probable experts are
+# the k largest logits (InfiniLM PR #500 report §2.1, top-k softmax routing;
+# ties to the lower expert id as the layer's statement of the problem fixes);
+# each expected order below is read off the logits by hand.
+ROUTE_EDGE_ROWS = [
+    # distinct logits far below the max: their probabilities round to the same
+    # double (1 + 1e-30 == 1 + 2e-30), but 2e-30 > 1e-30
+    ([1.0, 1e-30, 2e-30, -1.0], 3, [0, 2, 1]),
+    # probabilities of 0 and 1 underflow to 0.0 next to 1000; 1 > 0 still
+    ([1000.0, 0.0, 1.0], 3, [0, 2, 1]),
+    # NaN ranks as -inf; -0 and +0 tie and go to the lower id
+    ([0.5, float("nan"), -0.0, 0.0, float("nan"), -2.0], 6, [0, 2, 3, 5, 1, 4]),
+    ([0.0, -0.0, float("nan"), -float("inf"), 1.0], 4, [4, 0, 1, 2]),
+]
+
+
+@pytest.mark.parametrize("row,k,expect", ROUTE_EDGE_ROWS)
+def test_route_orders_by_logit_where_probabilities_tie(row, k, expect):
+    logits = torch.tensor([row], dtype=torch.float32)
+    ids, w = oracle.route(logits, k)
+    assert ids[0].tolist() == expect
+    # library pin of the same reading: a stable descending sort of the logits
+    # with NaN read as -inf and -0 as +0
+    clean = torch.where(torch.isnan(logits), torch.tensor(-float("inf")), logits) + 0.0
+    ref = torch.sort(clean, dim=1, descending=True, stable=True).indices[:, :k]
+    assert ids[0].tolist() == ref[0].tolist()
+    # weights: the renormalised softmax of the selected logits in double, with
+    # NaN contributing exp(-inf) = 0
+    sel = clean[0, ids[0].astype(np.int64)].double()
+    p = torch.exp(sel - sel[0])
+    assert np.allclose(w[0], (p / p.sum()).numpy(), rtol=2 ** -24, atol=0)
+    assert abs(float(w[0].astype(np.float64).sum()) - 1.0) <= 1e-6
+
+
 @pytest.mark.parametrize("T,E,k", [(50, 8, 2), (64, 128, 8), (40, 64, 6), (7, 256, 8)])
 def test_route_weights_match_library_softmax(T, E, k):
     g = torch.Generator().manual_seed(E + k)
