@@ -315,17 +315,17 @@ int oracle_forward(int fmt, const uint16_t *hidden, const float *logits,
     size_t gu_elems = fmt == 0 ? (size_t)2 * I * H : (size_t)2 * I * (H / 2);
     size_t d_elems = fmt == 0 ? (size_t)H * I : (size_t)H * (I / 2);
     size_t esz = fmt == 0 ? 2 : 1;
-    for (int e = 0; e < E; ++e) {
+    /* every row r of expert e's segment [offsets[e], offsets[e+1]) is one
+       token through that expert's FFN; rows are independent */
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < P; ++r) {
+        int p = perm[r], t = p / k, e = ids[p];
         const char *wgu_e = (const char *)w_gu + (size_t)e * gu_elems * esz;
         const char *wd_e = (const char *)w_d + (size_t)e * d_elems * esz;
         const uint16_t *sgu_e = fmt == 1 ? w_gu_s + (size_t)e * 2 * I * (H / 128) : NULL;
         const uint16_t *sd_e = fmt == 1 ? w_d_s + (size_t)e * H * (I / 128) : NULL;
-#pragma omp parallel for schedule(dynamic, 1)
-        for (int r = offsets[e]; r < offsets[e + 1]; ++r) {
-            int t = perm[r] / k;
-            oracle_expert_ffn(fmt, hidden + (size_t)t * H, wgu_e, sgu_e, wd_e, sd_e, H, I,
-                              act + (size_t)r * I, y + (size_t)r * H);
-        }
+        oracle_expert_ffn(fmt, hidden + (size_t)t * H, wgu_e, sgu_e, wd_e, sd_e, H, I,
+                          act + (size_t)r * I, y + (size_t)r * H);
     }
     oracle_finalize(y, w, inv_perm, T, H, k, out);
     return 0;

@@ -192,6 +192,23 @@ def test_finalize_bit_exact(T, H, k):
     assert np.array_equal(run_finalize(y_bits, w, inv, T, H, k), oracle.finalize(y_bits, w, inv, T, H, k))
 
 
+def test_finalize_flags_out_of_range_rows():
+    # A corrupted inverse permutation must not pass silently: an index outside
+    # [0, T*k) contributes 0 (as a +0 row would) and raises device error 3.
+    T, H, k = 5, 64, 3
+    rng = np.random.default_rng(11)
+    y_bits = bf16_bits(torch.from_numpy(rng.standard_normal((T * k, H)).astype(np.float32)).to(torch.bfloat16))
+    w = rng.random((T, k)).astype(np.float32)
+    inv = rng.permutation(T * k).astype(np.int32)
+    inv[4], inv[9] = T * k, -2
+    assert moe.moe_get_device_error() == 0
+    out = run_finalize(y_bits, w, inv, T, H, k)
+    assert moe.moe_get_device_error() == 3
+    y_ext = np.concatenate([y_bits, np.zeros((1, H), np.uint16)])
+    inv_ref = np.where((inv < 0) | (inv >= T * k), T * k, inv).astype(np.int32)
+    assert np.array_equal(out, oracle.finalize(y_ext, w, inv_ref, T, H, k))
+
+
 def test_finalize_special_cases_from_the_golden_file():
     import test_oracle_pins as pins
     for k, v, w, exp, why in pins._golden_finalize_cases():
@@ -227,6 +244,8 @@ GEMM_CFGS = [
     moe_synth.get_config("qwen3_prefill", T=700, H=512, I=256, E=8, k=2),  # tokens-on-M kernel, ragged tail
     moe_synth.get_config("qwen3_prefill", T=1024, H=512, I=384, E=8, k=2),  # CTA-pair kernel
     moe_synth.get_config("qwen3_prefill", T=1100, H=264, I=200, E=4, k=2),  # CTA-pair, ragged H and I
+    moe_synth.get_config("qwen3_decode", T=448, H=1024, I=384, E=64, k=8),  # weights on M, 128-token blocks
+    moe_synth.MoeConfig("int4_bn64", T=96, H=1024, I=384, E=24, k=8, fmt="int4_g128"),  # int4, 64-token blocks
 ]
 
 
