@@ -30,6 +30,10 @@
  *    descending logit; equal logits go to the lower expert id.
  *  - No C++ exception crosses this interface. Entry points are reentrant
  *    given distinct workspaces and outputs.
+ *  - The library keeps, per device, the device address of its error flag
+ *    (and of moe_permute_noalloc's scratch array), looked up on first use.
+ *    These belong to the device's context: do not call the library again
+ *    after a cudaDeviceReset in the same process.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
@@ -72,8 +76,11 @@ typedef uint16_t moe_bf16_t;   /* bit pattern of a bfloat16 value */
 typedef void *moe_stream_t;    /* cudaStream_t */
 
 /* Bytes of device workspace moe_forward needs for this shape (0 if the shape
- * is invalid). It holds the routing, the permutation, act [T*k,I], y [T*k,H]
- * and, when many tokens share each expert, the gathered rows [T*k,H]. */
+ * is invalid). It holds the intermediates between the steps of InfiniLM PR
+ * #500 report §2.2 (routing ids and weights, per-expert counts and offsets,
+ * the permutation and its inverse, act [T*k,I] between the gate/up and down
+ * grouped GEMMs, y [T*k,H] before the weighted scatter back) and, when many
+ * tokens share each expert, the gathered rows [T*k,H] of §2.2 step 2. */
 MOE_API size_t moe_workspace_size(const moe_shape_t *shape);
 
 /* Bytes of scratch moe_permute needs (may be 0). */
@@ -141,16 +148,11 @@ MOE_API moe_status_t moe_grouped_gemm_down(const moe_bf16_t *act, const int32_t 
  *   nearest), then acc = fma(v_j, w_j, acc) for j = 1..top_k-1 (round to
  *   nearest, no flush-to-zero), v_j = y[inv_perm[t*top_k+j], h],
  *   w_j = topk_w[t*top_k+j]. Signed zeros and subnormals are kept.
- *   A row index outside [0, T*top_k) reads as 0. Bit-exact and deterministic. */
+ *   A row index outside [0, T*top_k) reads as 0 and raises device error 3
+ *   (moe_get_device_error). Bit-exact and deterministic. */
 MOE_API moe_status_t moe_finalize(const moe_bf16_t *y, const float *topk_w, const int32_t *inv_perm,
                           const moe_shape_t *shape, moe_bf16_t *out, moe_stream_t stream);
 
-/* The whole layer: route, permute (with the gather when many tokens share
- * each expert; otherwise the gate/up GEMM gathers through perm itself),
- * gate/up + SwiGLU, down, finalize, enqueued on one stream with no host
- * synchronisation.
- *   hidden [T,H] bf16, logits [T,E] fp32, weights as above, out [T,H] bf16.
- *   ws: at least moe_workspace_size(shape) bytes, 256-byte aligned. */
 /* Number of kernels moe_forward enqueues for this shape (0 when T = 0, -1
  * when the shape is invalid). Host-side only; launches nothing. */
 MOE_API int32_t moe_forward_kernel_count(const moe_shape_t *shape);
@@ -161,6 +163,18 @@ MOE_API int32_t moe_forward_kernel_count(const moe_shape_t *shape);
  * runs the kernel moe_forward runs. Host-side only. */
 MOE_API int32_t moe_forward_gathers_in_gemm(const moe_shape_t *shape);
 
+/* The whole layer, in the order of InfiniLM PR #500 report §2.2 (bucket the
+ * routing indices, gather, grouped GEMMs gate/up and down with SwiGLU between
+ * them, scale by the routing weights and scatter back) with the routing of
+ * §2.1/§2.4 and the finalize arithmetic of FlashInfer PR #7196 analysis §1:
+ * route, permute (with the gather when many tokens share each expert;
+ * otherwise the gate/up GEMM gathers through perm itself), gate/up + SwiGLU,
+ * down, finalize, enqueued on one stream with no host synchronisation. The
+ * result equals the step entry points called in that order.
+ *   hidden [T,H] bf16, logits [T,E] fp32, weights as above, out [T,H] bf16.
+ *   ws: at least moe_workspace_size(shape) bytes, 256-byte aligned; the
+ *   call overwrites it, so calls that overlap on the GPU need distinct
+ *   workspaces. */
 MOE_API moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits,
                          const void *w_gu, const moe_bf16_t *w_gu_scales,
                          const void *w_d, const moe_bf16_t *w_d_scales,
@@ -188,7 +202,8 @@ MOE_API moe_status_t moe_dequant_int4(const uint8_t *q, const moe_bf16_t *scales
 
 /* Device error flag of the current device: waits for all work on the device,
  * stores the flag in *code (0 = none; 1 = bad expert id; 2 = a pipeline wait
- * timed out) and clears it. */
+ * timed out; 3 = a finalize row index out of range) and clears it. The first
+ * error raised since the last read is the one kept. */
 MOE_API moe_status_t moe_get_device_error(int32_t *code);
 
 /* Self-test of the bounded waits behind device error code 2 (no counterpart

@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "launch.h"
 #include "moe.h"
@@ -16,15 +17,22 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// Device address of g_moe_error_flag on the current device, looked up on the
+// first call made with that device current. Concurrent first calls may both
+// look it up; they store the same address. The cached address belongs to the
+// device's context, so the library must not be used across a cudaDeviceReset.
 int *error_flag_ptr() {
-    static int *ptrs[kMaxDevices] = {};
+    static std::atomic<int *> ptrs[kMaxDevices] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    if (!ptrs[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_moe_error_flag) == cudaSuccess) ptrs[dev] = static_cast<int *>(p);
+    int *p = ptrs[dev].load(std::memory_order_acquire);
+    if (!p) {
+        void *q = nullptr;
+        if (cudaGetSymbolAddress(&q, g_moe_error_flag) != cudaSuccess) return nullptr;
+        p = static_cast<int *>(q);
+        ptrs[dev].store(p, std::memory_order_release);
     }
-    return ptrs[dev];
+    return p;
 }
 
 inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -158,7 +166,7 @@ moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const
     moe::GemmArgs dn = gemm_args(s, act, nullptr, offsets, w_d, w_d_scales, false, y);
     dn.hints = moe::kGemmHintOffsetsReady;
     if ((e = moe::launch_grouped_gemm(dn, st)) != cudaSuccess) return cuda_status(e);
-    return cuda_status(moe::launch_finalize(y, w, inv, T, H, k, out, st));
+    return cuda_status(moe::launch_finalize(y, w, inv, T, H, k, out, error_flag_ptr(), st));
 }
 
 }  // namespace
@@ -256,7 +264,7 @@ moe_status_t moe_finalize(const moe_bf16_t *y, const float *topk_w, const int32_
         !aligned(inv_perm, 4))
         return MOE_ERR_INVALID_ARG;
     return cuda_status(moe::launch_finalize(y, topk_w, inv_perm, shape->T, shape->H, shape->top_k, out,
-                                            static_cast<cudaStream_t>(stream)));
+                                            error_flag_ptr(), static_cast<cudaStream_t>(stream)));
 }
 
 int32_t moe_forward_kernel_count(const moe_shape_t *shape) {

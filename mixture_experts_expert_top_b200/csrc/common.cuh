@@ -11,7 +11,7 @@
 namespace moe {
 
 // Device error codes (the flag word moe_get_device_error reads).
-enum : int { kErrBadExpertId = 1, kErrTimeout = 2 };
+enum : int { kErrBadExpertId = 1, kErrTimeout = 2, kErrBadRow = 3 };
 
 // A pipeline wait that has not completed after this long gives up, raises
 // kErrTimeout and lets the kernel unwind instead of hanging the GPU.

@@ -46,7 +46,7 @@ cudaError_t launch_gather(const uint16_t *hidden, const int32_t *perm, int P, in
 
 // ---- finalize.cu
 cudaError_t launch_finalize(const uint16_t *y, const float *w, const int32_t *inv_perm, int T, int H, int k,
-                            uint16_t *out, cudaStream_t s);
+                            uint16_t *out, int *err, cudaStream_t s);
 
 // ---- gemm_sm100.cu
 struct GemmArgs {

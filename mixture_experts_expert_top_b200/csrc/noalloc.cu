@@ -14,6 +14,8 @@
 // device, on the first call made with that device current.
 #include <stdint.h>
 
+#include <atomic>
+
 #include "launch.h"
 #include "moe.h"
 
@@ -29,16 +31,19 @@ static __device__ __align__(256) int32_t g_permute_scratch[kScratchInts];
 // Device address of g_permute_scratch on the current device (nullptr on
 // failure). In host code the symbol's name is only a host-side stand-in, so
 // the address has to come from cudaGetSymbolAddress with the device current.
+// Concurrent first calls on one device may both look it up; they store the
+// same address. The address belongs to the device's context, so it is not
+// valid across a cudaDeviceReset.
 int32_t *scratch_ptr() {
-    static int32_t *ptrs[kMaxDevices] = {};
+    static std::atomic<int32_t *> ptrs[kMaxDevices] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-    if (!ptrs[dev]) {
-        int32_t *p = nullptr;
+    int32_t *p = ptrs[dev].load(std::memory_order_acquire);
+    if (!p) {
         if (cudaGetSymbolAddress(reinterpret_cast<void **>(&p), g_permute_scratch) != cudaSuccess) return nullptr;
-        ptrs[dev] = p;
+        ptrs[dev].store(p, std::memory_order_release);
     }
-    return ptrs[dev];
+    return p;
 }
 
 inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
