@@ -3,20 +3,25 @@
 
 One step = one whole layer call (route, permute + gather, grouped GEMM
 gate/up + SwiGLU, grouped GEMM down, finalize) over one batch of synthetic
-tokens, through the C ABI. The default workload is the Qwen3-30B-A3B-shaped
-decode layer: T=64, H=2048, I=768, E=128, top_k=8, bf16 weights (1.2 GB of
-expert weights, larger than the 126 MB L2, so no flush is needed between
-steps).
+tokens, through the C ABI (moe_forward). The headline workload is the
+largest single-GPU one, the Qwen3-30B-A3B-shaped prefill layer: T=8192,
+H=2048, I=768, E=128, top_k=8, bf16 weights. The same run also times the
+other graded workloads (Qwen3 decode, the skewed Zipf layer and the W4A16
+decode layer) and reports them under "workloads". Every workload reads more
+than the 126 MB L2 per step (its expert weights), so no flush is needed
+between steps.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                  [--extra all|none|NAME,...] [--impl ours|reference]
 
-With --gpus N > 1 (one process per GPU under torchrun) every rank runs its
-own replica on its own token batch (token-sharded data parallel: the layer
-needs no exchange between ranks), and value = all ranks' tokens / the
-slowest rank's time.
+With --gpus N > 1 (one process per GPU under torchrun; started without
+torchrun, bench.py relaunches itself under torchrun) every rank runs its own
+replica on its own token batch (token-sharded data parallel: the layer needs
+no exchange between ranks), and value = all ranks' tokens / the slowest
+rank's time.
 
 --impl reference times the CPU oracle (the plain C reference in oracle/) on
-the host cores, on the same workload, metric and unit.
+the host cores, on the headline workload, metric and unit.
 """
 
 from __future__ import annotations
@@ -26,6 +31,7 @@ import hashlib
 import json
 import os
 import re
+import socket
 import statistics
 import subprocess
 import sys
@@ -38,6 +44,12 @@ if ROOT not in sys.path:
 
 METRIC = "MoE-layer tokens/s on 1 B200; fraction of HBM / bf16 tensor-core roofline"
 UNIT = "tokens/s"
+HEADLINE = "qwen3_prefill"
+EXTRA = ["qwen3_decode", "skewed", "w4a16_decode"]
+# the layer's targets: decode layers against 8 TB/s of activated weight bytes,
+# prefill-like layers against 2.25 PFLOP/s dense bf16
+TARGETS = {"qwen3_decode": ("hbm", 0.70), "w4a16_decode": ("hbm", 0.70),
+           "qwen3_prefill": ("tensor", 0.60), "skewed": ("tensor", 0.60), "tiny": (None, None)}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NORTH_STAR_HBM_GBS = 8000.0       # the roofline literals the layer's target is stated against
 NORTH_STAR_BF16_TFLOPS = 2250.0
@@ -55,11 +67,13 @@ KERNEL_SOURCES = ["mixture_experts_expert_top_b200/csrc/gemm_sm100.cu",
 def parse_args(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="qwen3_decode")
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=HEADLINE)
+    ap.add_argument("--extra", default="all",
+                    help="other workloads timed in the same run: all, none, or a comma list")
     ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
-                    help="override a workload field (T, H, I, E, k), e.g. for a smaller profiling case")
+                    help="override a field (T, H, I, E, k) of the headline workload, e.g. for a profiling case")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -70,7 +84,16 @@ def parse_args(argv=None):
         ap.error("--warmup must be >= 3")
     if a.steps < 1:
         ap.error("--steps must be >= 1")
+    if a.gpus < 1:
+        ap.error("--gpus must be >= 1")
     return a
+
+
+def extra_workloads(args):
+    if args.set or args.extra == "none":
+        return []
+    names = EXTRA if args.extra == "all" else [n for n in args.extra.split(",") if n]
+    return [n for n in names if n != args.workload]
 
 
 def dist_env():
@@ -108,6 +131,18 @@ def read_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def host_cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def kernel_source_hash() -> str:
     h = hashlib.sha256()
     for rel in KERNEL_SOURCES:
@@ -132,34 +167,78 @@ def profiled_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    """SM clock, power and clock-event reasons of one GPU, polled through NVML
+    every couple of milliseconds in a background thread (so that even a timed
+    region of a few milliseconds holds samples); falls back to nvidia-smi
+    polling when NVML is not importable."""
 
-    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
-              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
-              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+    REASONS = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, gpu_id: str, period_ms: int = 50):
-        self.gpu_id = gpu_id
-        self.period_ms = period_ms
-        self.proc = None
-        self.lines = []
+    def __init__(self, uuid: str, index: int, period_s: float = 0.002):
+        self.uuid, self.index, self.period_s = uuid, index, period_s
+        self.samples = []          # (time, sm_mhz, power_w, reasons)
+        self.sm_max = None
+        self.source = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
         self.t0 = self.t1 = None
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={','.join(self.FIELDS)}",
-                 "--format=csv,noheader,nounits", f"-lms", str(self.period_ms)],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
-            return
-        self._reader = threading.Thread(target=self._read, daemon=True)
-        self._reader.start()
+            import pynvml as nv
+            nv.nvmlInit()
+            try:
+                h = nv.nvmlDeviceGetHandleByUUID(self.uuid)
+            except Exception:      # noqa: BLE001 - UUID form not accepted: fall back to the index
+                h = nv.nvmlDeviceGetHandleByIndex(self.index)
+            self.sm_max = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons",
+                                  getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons", None))
+            bits = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+                    "sw_power_cap": 0x4}
+            self.source = "nvml"
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append((time.time(), line.strip()))
+            def loop():
+                while not self._stop.is_set():
+                    try:
+                        t = time.time()
+                        sm = float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM))
+                        pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        r = int(get_reasons(h)) if get_reasons else 0
+                        self.samples.append((t, sm, pw, [n for n, b in bits.items() if r & b]))
+                    except Exception:  # noqa: BLE001 - a failed poll is skipped
+                        pass
+                    self._stop.wait(self.period_s)
+
+            self._thread = threading.Thread(target=loop, daemon=True)
+            self._thread.start()
+            return
+        except Exception:          # noqa: BLE001 - no NVML: nvidia-smi below
+            pass
+        fields = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+                  "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+                  "clocks_event_reasons.sw_power_cap"]
+        try:
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.uuid, f"--query-gpu={','.join(fields)}", "--format=csv,noheader,nounits",
+                 "-lms", "20"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self._proc = None
+            return
+        self.source = "nvidia-smi"
+
+        def read():
+            for line in self._proc.stdout:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) != 7 or not _isnum(p[0]):
+                    continue
+                self.sm_max = float(p[1]) if _isnum(p[1]) else self.sm_max
+                self.samples.append((time.time(), float(p[0]), float(p[2]) if _isnum(p[2]) else None,
+                                     [n for n, v in zip(self.REASONS, p[3:]) if v.lower().startswith("active")]))
+
+        self._thread = threading.Thread(target=read, daemon=True)
+        self._thread.start()
 
     def mark_begin(self):
         self.t0 = time.time()
@@ -168,29 +247,27 @@ class ClockSampler:
         self.t1 = time.time()
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        time.sleep(2 * self.period_ms / 1000.0)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        rows = []
-        for ts, line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) != len(self.FIELDS):
-                continue
-            rows.append((ts, parts))
-        inside = [r for ts, r in rows if self.t0 is not None and self.t0 <= ts <= (self.t1 or ts)]
-        use = inside or [r for _, r in rows]
-        sm = [float(r[1]) for r in use if _isnum(r[1])]
-        smax = [float(r[2]) for r in use if _isnum(r[2])]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({n for r in use for n, v in zip(names, r[5:9]) if v.lower().startswith("active")})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
-                "reasons": reasons, "samples": len(use), "samples_inside_timed_region": len(inside),
-                "power_w_max": max((float(r[3]) for r in use if _isnum(r[3])), default=None)}
+        time.sleep(0.01)
+        self._stop.set()
+        if self._proc is not None:
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self._proc.kill()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+
+    def summary(self, t0=None, t1=None):
+        """Samples inside [t0, t1] (default: the marked region)."""
+        t0 = self.t0 if t0 is None else t0
+        t1 = self.t1 if t1 is None else t1
+        inside = [s for s in list(self.samples) if t0 is not None and t1 is not None and t0 <= s[0] <= t1]
+        sm = [s[1] for s in inside]
+        pw = [s[2] for s in inside if s[2] is not None]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.sm_max,
+                "reasons": sorted({r for s in inside for r in s[3]}), "samples_inside_timed_region": len(inside),
+                "power_w_max": max(pw) if pw else None, "source": self.source}
 
 
 def _isnum(s):
@@ -199,6 +276,12 @@ def _isnum(s):
         return True
     except ValueError:
         return False
+
+
+def free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
 
 
 # -------------------------------------------------------- workload accounting --
@@ -233,13 +316,11 @@ def launches_per_step(cfg) -> int:
     return moe.moe_forward_kernel_count(moe.Shape.of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.fmt))
 
 
-# ------------------------------------------------------------------ our arm --
-
-def workload(args):
+def get_workload(name, sets=()):
     import moe_synth
-    cfg = moe_synth.get_config(args.workload)
+    cfg = moe_synth.get_config(name)
     over = {}
-    for kv in args.set:
+    for kv in sets:
         k, v = kv.split("=", 1)
         if k not in ("T", "H", "I", "E", "k"):
             raise SystemExit(f"--set: unknown field {k}")
@@ -249,26 +330,50 @@ def workload(args):
     return cfg
 
 
-def run_ours(args, rank, world, local):
-    import numpy as np
+def config_of(cfg, world):
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": cfg.describe(), "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "top_k": cfg.k,
+            "weights": cfg.fmt, "global_batch": world * cfg.T,
+            "parallelism": "replicas (token-sharded, no collective)" if world > 1 else "single GPU",
+            "l2": f"inputs larger than L2: {expert_weight_bytes(cfg) / 1e9:.3f} GB of expert weights, of which "
+                  "each step reads its activated experts' (> 126 MB); no flush"}
+
+
+def expert_weight_bytes(cfg):
+    """Bytes of all E experts' weights (and int4 scales) of a workload."""
+    if cfg.fmt == "bf16":
+        return cfg.E * 3 * cfg.H * cfg.I * 2
+    return cfg.E * (2 * cfg.I * (cfg.H // 2 + cfg.H // 64) + cfg.H * (cfg.I // 2 + cfg.I // 64))
+
+
+def layer_fractions(cfg, work, layer_s, peaks):
+    bound, target = TARGETS.get(cfg.name.split("+")[0], (None, None))
+    f = {"active_experts": work["active_experts"], "weight_bytes": work["weight_bytes"],
+         "flops": work["layer_flops"],
+         "hbm_frac_of_8TBps": work["weight_bytes"] / layer_s / (NORTH_STAR_HBM_GBS * 1e9),
+         "hbm_frac_of_measured": work["weight_bytes"] / layer_s / (peaks["hbm_gbs"] * 1e9),
+         "tensor_frac_of_2250TF": work["layer_flops"] / layer_s / (NORTH_STAR_BF16_TFLOPS * 1e12),
+         "tensor_frac_of_measured_burst": work["layer_flops"] / layer_s / (peaks["bf16_tflops"] * 1e12)}
+    if bound:
+        got = f["hbm_frac_of_8TBps"] if bound == "hbm" else f["tensor_frac_of_2250TF"]
+        f["target"] = {"bound": bound, "frac": target, "achieved": got, "met": got >= target}
+    return f
+
+
+# ------------------------------------------------------------------ our arm --
+
+def measure(cfg, args, dev, world, rank, sampler, headline):
+    """Time one workload: K whole-layer steps (the value), a per-step pass
+    (median and minimum), a CUDA-graph replay for decode batches, a per-stage
+    pass (the roofline of the dominant kernel) and K steps end to end through
+    moe_forward_host."""
     import torch
-    import torch.distributed as dist
 
     import moe_synth
     import mixture_experts_expert_top_b200 as moe
 
-    if not torch.cuda.is_available():
-        raise SystemExit("bench.py needs a CUDA device (B200)")
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-    moe.lib()
-    cfg = workload(args)
-    # weights are the same on every rank (replicas); each rank draws its own tokens
     inp = moe_synth.gen_inputs(cfg, seed=args.seed)
-    if rank:
+    if rank:   # weights are the same on every rank (replicas); each rank draws its own tokens
         inp["hidden"] = moe_synth.gen_hidden(cfg, seed=args.seed + rank)
         inp["logits"] = moe_synth.gen_logits(cfg, seed=args.seed + rank)
     d = {n: t.to(dev) for n, t in inp.items()}
@@ -277,36 +382,65 @@ def run_ours(args, rank, world, local):
     out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
     scales = (d.get("w_gu_scales"), d.get("w_d_scales"))
+    K, W = args.steps, args.warmup
 
-    def step():
-        moe.moe_forward(d["hidden"], d["logits"], d["w_gu"], scales[0], d["w_d"], scales[1], shape, out, ws, stream)
+    def step(s=stream):
+        moe.moe_forward(d["hidden"], d["logits"], d["w_gu"], scales[0], d["w_d"], scales[1], shape, out, ws, s)
 
-    # ---- device-timed value: K whole-layer steps ---------------------------
-    for _ in range(args.warmup):
+    def ev():
+        return torch.cuda.Event(enable_timing=True)
+
+    # ---- value: exactly K steps, barrier + synchronize on both sides --------
+    for _ in range(W):
         step()
     torch.cuda.synchronize()
-    props = torch.cuda.get_device_properties(dev)
-    gpu_id = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
-    sampler = ClockSampler(gpu_id)
-    sampler.start()
-    time.sleep(0.2)
     barrier()
     torch.cuda.synchronize()
-    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a, b = ev(), ev()
     sampler.mark_begin()
-    t_start.record(stream)
-    for _ in range(args.steps):
+    a.record(stream)
+    for _ in range(K):
         step()
-    t_end.record(stream)
+    b.record(stream)
     torch.cuda.synchronize()
     sampler.mark_end()
     barrier()
-    ms = t_start.elapsed_time(t_end)
-    clocks = sampler.stop()
-    ms_max = max_over_ranks(ms)
-    value = world * cfg.T * args.steps / (ms_max / 1e3)
+    clocks = sampler.summary()
+    ms_max = max_over_ranks(a.elapsed_time(b))
+    value = world * cfg.T * K / (ms_max / 1e3)
 
-    # ---- per-kernel durations (same kernels, one C-ABI call per stage) -----
+    # ---- per-step distribution: at least 50 steps, each between events -----
+    n_it = max(50, min(K, 500))
+    evs = [ev() for _ in range(n_it + 1)]
+    evs[0].record(stream)
+    for i in range(n_it):
+        step()
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize()
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(n_it)]
+    step_ms = {"median": statistics.median(per), "min": min(per), "n": n_it,
+               "note": "an event between steps keeps the next step from starting early"}
+
+    # ---- CUDA-graph replay of one captured step (decode batches) ------------
+    graph = None
+    if cfg.T <= 256:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(torch.cuda.current_stream(dev))
+        for _ in range(W):
+            g.replay()
+        torch.cuda.synchronize()
+        ga, gb = ev(), ev()
+        ga.record(stream)
+        for _ in range(K):
+            g.replay()
+        gb.record(stream)
+        torch.cuda.synchronize()
+        gms = max_over_ranks(ga.elapsed_time(gb))
+        graph = {"ms_per_step": gms / K, "value": world * cfg.T * K / (gms / 1e3), "steps": K}
+        del g
+
+    # ---- per-stage pass: one C-ABI call per stage, events between ------------
     P = cfg.P
     i32 = dict(dtype=torch.int32, device=dev)
     ids = torch.empty(cfg.T, cfg.k, **i32)
@@ -332,23 +466,22 @@ def run_ours(args, rank, world, local):
         lambda: moe.moe_grouped_gemm_down(act, offsets, d["w_d"], scales[1], shape, y, stream),
         lambda: moe.moe_finalize(y, wts, inv, shape, out, stream),
     ]
-    for _ in range(args.warmup):
+    for _ in range(W):
         for c in calls:
             c()
     torch.cuda.synchronize()
-    n_rep = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(n_rep)]
+    n_rep = max(20, min(K, 200))
+    se = [[ev() for _ in range(len(calls) + 1)] for _ in range(n_rep)]
     for r in range(n_rep):
-        ev[r][0].record(stream)
+        se[r][0].record(stream)
         for i, c in enumerate(calls):
             c()
-            ev[r][i + 1].record(stream)
+            se[r][i + 1].record(stream)
     torch.cuda.synchronize()
     # median over repetitions: robust to the odd slow repetition (a clock dip)
-    stage_ms = {s: statistics.median(ev[r][i].elapsed_time(ev[r][i + 1]) for r in range(n_rep))
+    stage_ms = {s: statistics.median(se[r][i].elapsed_time(se[r][i + 1]) for r in range(n_rep))
                 for i, s in enumerate(stages)}
-    counts_h = counts.cpu().numpy()
-    work = work_per_step(cfg, counts_h)
+    work = work_per_step(cfg, counts.cpu().numpy())
 
     # ---- end to end through moe_forward_host (pinned host buffers) ----------
     hws = torch.empty(moe.moe_forward_host_workspace_size(shape), dtype=torch.uint8, device=dev)
@@ -359,67 +492,103 @@ def run_ours(args, rank, world, local):
     def e2e_step():
         moe.moe_forward_host(h_host, l_host, d["w_gu"], scales[0], d["w_d"], scales[1], shape, o_host, hws, stream)
 
-    for _ in range(args.warmup):
+    for _ in range(W):
         e2e_step()
     barrier()
     torch.cuda.synchronize()
-    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e_start.record(stream)
-    for _ in range(args.steps):
+    ea, eb = ev(), ev()
+    ea.record(stream)
+    for _ in range(K):
         e2e_step()
-    e_end.record(stream)
+    eb.record(stream)
     torch.cuda.synchronize()
-    e_ms = max_over_ranks(e_start.elapsed_time(e_end))
-    e2e_value = world * cfg.T * args.steps / (e_ms / 1e3)
-    h2d = h_host.numel() * h_host.element_size() + l_host.numel() * l_host.element_size()
-    d2h = o_host.numel() * o_host.element_size()
+    e_ms = max_over_ranks(ea.elapsed_time(eb))
+    e2e = {"value": world * cfg.T * K / (e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": h_host.numel() * h_host.element_size() + l_host.numel() * l_host.element_size(),
+           "d2h_bytes_per_step": o_host.numel() * o_host.element_size()}
 
     err = moe.moe_get_device_error()
     if err:
-        raise SystemExit(f"device error flag {err} raised during the benchmark")
+        raise SystemExit(f"device error flag {err} raised during the benchmark of {cfg.name}")
 
     # ---- roofline of the dominant kernel -------------------------------------
+    # each stage is timed on its own (a sub-millisecond launch between events),
+    # so a tensor-bound kernel is held against the burst bf16 peak
     peaks, peak_src = read_peaks()
     dom = max(("gemm_swiglu", "gemm_down"), key=lambda s: stage_ms[s])
     wk = work[dom]
-    ai = wk["flops"] / wk["bytes"]
-    ridge = peaks["bf16_tflops_sustained"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
     sec = stage_ms[dom] / 1e3
-    if ai < ridge:
+    if wk["flops"] / wk["bytes"] < ridge:
         roof = {"bound": "hbm", "achieved": wk["bytes"] / sec / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        which = "hbm_gbs"
     else:
-        roof = {"bound": "tensor", "achieved": wk["flops"] / sec / 1e12, "peak": peaks["bf16_tflops_sustained"],
+        roof = {"bound": "tensor", "achieved": wk["flops"] / sec / 1e12, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s"}
+        which = "bf16_tflops (burst: the kernel is timed alone)"
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = profiled_traffic(dom, cfg.name)
     roof["kernel"] = dom
     roof["algorithmic_per_launch"] = wk["bytes"] if roof["bound"] == "hbm" else wk["flops"]
-    roof["peak_source"] = f"{peak_src} ({'hbm_gbs' if roof['bound'] == 'hbm' else 'bf16_tflops_sustained'})"
+    roof["peak_source"] = f"{peak_src} {which}"
     roof["launch_ms"] = stage_ms[dom]
 
-    layer_s = ms_max / 1e3 / args.steps
+    layer_s = ms_max / 1e3 / K
+    res = {"value": value, "ms_per_step": ms_max / K, "steps": K, "step_ms": step_ms, "roofline": roof,
+           "layer": dict(layer_fractions(cfg, work, layer_s, peaks), stage_ms=stage_ms), "e2e": e2e,
+           "gpu_launches": launches_per_step(cfg) * K, "clocks": clocks}
+    if graph:
+        res["cuda_graph"] = graph
+    cpu = None
+    if headline and rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg, inp, args.cpu_budget_s)
+    del d, ws, out, ids, wts, counts, offsets, perm, inv, hp, act, y, pws, hws
+    torch.cuda.empty_cache()
+    return res, cpu
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+
+    import mixture_experts_expert_top_b200 as moe
+
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    moe.lib()
+    props = torch.cuda.get_device_properties(dev)
+    uuid = f"GPU-{props.uuid}" if getattr(props, "uuid", None) else str(local)
+    sampler = ClockSampler(uuid, local)
+    sampler.start()
+    try:
+        cfg = get_workload(args.workload, args.set)
+        head, cpu = measure(cfg, args, dev, world, rank, sampler, headline=True)
+        others = {}
+        for name in extra_workloads(args):
+            c = get_workload(name)
+            r, _ = measure(c, args, dev, world, rank, sampler, headline=False)
+            others[name] = dict(r, config=c.describe())
+    finally:
+        sampler.stop()
     result = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.fmt == "bf16" else "bf16 (int4 weights)",
         "data": "synthetic (seeded N(0,1) tokens and logits, N(0,0.02) random-init expert weights)",
-        "config": {"workload": cfg.describe(), "T": cfg.T, "H": cfg.H, "I": cfg.I, "E": cfg.E, "top_k": cfg.k,
-                   "weights": cfg.fmt, "global_batch": world * cfg.T,
-                   "parallelism": "replicas (token-sharded, no collective)" if world > 1 else "single GPU",
-                   "l2": f"inputs larger than L2: {work['weight_bytes'] / 1e9:.3f} GB of expert weights read per step"},
-        "roofline": roof,
-        "layer": {"active_experts": work["active_experts"], "weight_bytes": work["weight_bytes"],
-                  "flops": work["layer_flops"],
-                  "hbm_frac_of_measured": work["weight_bytes"] / layer_s / (peaks["hbm_gbs"] * 1e9),
-                  "hbm_frac_of_8TBps": work["weight_bytes"] / layer_s / (NORTH_STAR_HBM_GBS * 1e9),
-                  "tensor_frac_of_2250TF": work["layer_flops"] / layer_s / (NORTH_STAR_BF16_TFLOPS * 1e12),
-                  "stage_ms": stage_ms},
-        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step(cfg) * args.steps,
-        "clocks": clocks,
+        "config": config_of(cfg, world),
+        "roofline": head["roofline"], "layer": head["layer"], "step_ms": head["step_ms"], "e2e": head["e2e"],
+        "gpu_launches": head["gpu_launches"], "clocks": head["clocks"],
+        "workloads": others,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        result["cpu_baseline"] = cpu_baseline(cfg, inp, args.cpu_budget_s)
+    if "cuda_graph" in head:
+        result["cuda_graph"] = head["cuda_graph"]
+    if cpu:
+        result["cpu_baseline"] = cpu
     if world > 1:
         dist.destroy_process_group()
     return result
@@ -450,7 +619,8 @@ def cpu_baseline(cfg, inp, budget_s):
     per_tok = (time.perf_counter() - t0) / min(4, n)
     ntok = max(1, min(n, int(budget_s / max(per_tok, 1e-9))))
     v, reps, el = _oracle_tokens_per_s(cfg, inp, tokens[:ntok], budget_s)
-    return {"value": v, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+    return {"value": v, "unit": UNIT, "cores": oracle.num_threads(), "cpu_model": host_cpu_model(),
+            "kind": "oracle",
             "sample": f"{reps} x {ntok} tokens of {cfg.name} (all k={cfg.k} experts per token, full H/I), "
                       f"{el:.1f} s of CPU time on {oracle.num_threads()} threads"}
 
@@ -460,7 +630,7 @@ def run_reference(args, rank, world):
         return None
     import moe_synth
     import oracle
-    cfg = workload(args)
+    cfg = get_workload(args.workload, args.set)
     inp = moe_synth.gen_inputs(cfg, seed=args.seed)
     # size each step so that warmup + steps fit the budget
     t0 = time.perf_counter()
@@ -481,19 +651,30 @@ def run_reference(args, rank, world):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": el * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64 accumulate",
-        "data": "synthetic", "config": {"workload": cfg.describe(), "global_batch": cfg.T},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-                         "sample": sample},
+        "data": "synthetic (seeded N(0,1) tokens and logits, N(0,0.02) random-init expert weights)",
+        "config": config_of(cfg, world),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "cpu_model": host_cpu_model(),
+                         "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
+def relaunch_under_torchrun(args, argv) -> int:
+    """--gpus N > 1 started as a plain process: run the same command as N
+    ranks under torchrun (one process per GPU) and return its exit status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()), os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
 def main(argv=None):
+    argv = list(sys.argv[1:] if argv is None else argv)
     args = parse_args(argv)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        raise SystemExit(relaunch_under_torchrun(args, argv))
     rank, world, local = dist_env()
-    if world != args.gpus and "WORLD_SIZE" in os.environ:
+    if world != args.gpus:
         raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
-    world = max(world, 1)
     if args.impl == "reference":
         res = run_reference(args, rank, world)
     else:

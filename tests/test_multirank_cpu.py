@@ -71,6 +71,32 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0
     assert outs[1][0].strip() == ""
+    # the reference arm reports the same config object as our arm would
+    sys.path.insert(0, ROOT)
+    import bench
+    assert line["config"] == bench.config_of(bench.get_workload("tiny"), 2)
+
+
+def test_gpus_n_without_torchrun_relaunches_as_n_ranks():
+    # started as one plain process, --gpus 2 must run two ranks (torchrun,
+    # gloo-free here: the reference arm needs no process group) and print one line
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK")}
+    p = subprocess.run(
+        [sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+         "--workload", "tiny", "--steps", "3", "--warmup", "3", "--ref-budget-s", "2"],
+        env=env, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True, timeout=300)
+    assert p.returncode == 0, p.stderr[-3000:]
+    lines = [l for l in p.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    assert json.loads(lines[0])["n_gpus"] == 2
+
+
+def test_gpus_must_match_world_size():
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--workload", "tiny", "--steps", "1", "--warmup", "3"],
+                       env=env, stdout=subprocess.PIPE, stderr=subprocess.PIPE, text=True, timeout=300)
+    assert p.returncode != 0 and "WORLD_SIZE" in p.stderr
 
 
 def test_bench_work_accounting():
