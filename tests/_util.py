@@ -30,17 +30,39 @@ def gemm_rows_close(gpu_bits, ref_bits, what=""):
     return float((np.asarray(gpu_bits) == np.asarray(ref_bits)).mean())
 
 
+def bf16_step(x: torch.Tensor) -> torch.Tensor:
+    """The spacing of bf16 values at |x| (one unit in the last place of an
+    8-bit significand): 2^(floor(log2 |x|) - 7), and the subnormal spacing
+    2^-133 below the smallest normal."""
+    a = x.abs().clamp_min(2.0 ** -126)
+    return torch.pow(2.0, torch.floor(torch.log2(a)) - 7)
+
+
 def layer_output_close(gpu_bits, ref_bits, what="", scale_abs_by_rms=False):
-    """End-to-end bound on the layer output: max |err| <= 2e-2 and
-    relative L2 error <= 1e-2 against the oracle. With scale_abs_by_rms, the
-    absolute bound is 2e-2 * max(1, rms(ref)) (used where one bf16 step of the
-    output already exceeds 2e-2)."""
+    """End-to-end bound on the layer output against the oracle: relative L2
+    error <= 1e-2, and per element |err| <= A, with A = 2e-2 (2e-2 *
+    max(1, rms(ref)) with scale_abs_by_rms, used where the outputs' scale makes
+    one bf16 step exceed 2e-2 throughout).
+
+    Both sides round act, y and the output to bf16. Where the two fp32
+    accumulations straddle a bf16 rounding point the results differ by one
+    bf16 step of the output, plus at most one more from a y row that rounded
+    the other way; at |out| >= 2 one step is 2^-6 or more, and two exceed A.
+    So an element passes if |err| <= max(A, 2 bf16 steps of max(|gpu|, |ref|)),
+    and at most 1e-3 of the elements may need the second form. Returns
+    (max |err|, rel-L2, number of elements beyond A)."""
     g = bits_to_bf16(gpu_bits).double()
     r = bits_to_bf16(ref_bits).double()
     err = (g - r).abs()
     rms = float(r.pow(2).mean().sqrt())
     lim = 2e-2 * (max(1.0, rms) if scale_abs_by_rms else 1.0)
     rel = float((g - r).norm() / r.norm().clamp_min(1e-30))
-    assert float(err.max()) <= lim, f"{what}: max|err| {float(err.max()):.4g} > {lim:.4g}"
+    beyond = err > lim
+    n_beyond = int(beyond.sum())
+    steps = 2 * bf16_step(torch.maximum(g.abs(), r.abs()))
+    bad = beyond & (err > steps)
+    assert not bool(bad.any()), (
+        f"{what}: {int(bad.sum())} elements beyond max({lim:.4g}, 2 bf16 steps); max|err| {float(err.max()):.4g}")
+    assert n_beyond <= 1e-3 * err.numel(), f"{what}: {n_beyond} elements beyond {lim:.4g}"
     assert rel <= 1e-2, f"{what}: rel-L2 {rel:.4g} > 1e-2"
-    return float(err.max()), rel
+    return float(err.max()), rel, n_beyond
