@@ -195,6 +195,7 @@ size_t moe_permute_workspace_size(const moe_shape_t *shape) {
 
 moe_status_t moe_route(const float *logits, const moe_shape_t *shape, int32_t *topk_ids, float *topk_w,
                        moe_stream_t stream) {
+    const moe::NvtxRange nvtx("moe_route");
     moe_status_t st = check_shape(shape);
     if (st != MOE_OK) return st;
     if (shape->T == 0) return MOE_OK;
@@ -207,6 +208,7 @@ moe_status_t moe_route(const float *logits, const moe_shape_t *shape, int32_t *t
 moe_status_t moe_permute(const int32_t *topk_ids, const moe_shape_t *shape, int32_t *counts, int32_t *offsets,
                          int32_t *perm, int32_t *inv_perm, const moe_bf16_t *hidden, moe_bf16_t *hidden_perm,
                          void *ws, size_t ws_bytes, moe_stream_t stream) {
+    const moe::NvtxRange nvtx("moe_permute");
     moe_status_t st = check_shape(shape);
     if (st != MOE_OK) return st;
     if (shape->T == 0) return MOE_OK;
@@ -231,6 +233,7 @@ moe_status_t moe_permute(const int32_t *topk_ids, const moe_shape_t *shape, int3
 moe_status_t moe_grouped_gemm_swiglu(const moe_bf16_t *a, const int32_t *perm, const int32_t *offsets,
                                      const void *w_gu, const moe_bf16_t *w_gu_scales, const moe_shape_t *shape,
                                      moe_bf16_t *act, moe_stream_t stream) {
+    const moe::NvtxRange nvtx("moe_grouped_gemm_swiglu");
     moe_status_t st = check_shape(shape);
     if (st != MOE_OK) return st;
     if (shape->T == 0) return MOE_OK;
@@ -245,6 +248,7 @@ moe_status_t moe_grouped_gemm_swiglu(const moe_bf16_t *a, const int32_t *perm, c
 moe_status_t moe_grouped_gemm_down(const moe_bf16_t *act, const int32_t *offsets, const void *w_d,
                                    const moe_bf16_t *w_d_scales, const moe_shape_t *shape, moe_bf16_t *y,
                                    moe_stream_t stream) {
+    const moe::NvtxRange nvtx("moe_grouped_gemm_down");
     moe_status_t st = check_shape(shape);
     if (st != MOE_OK) return st;
     if (shape->T == 0) return MOE_OK;
@@ -257,6 +261,7 @@ moe_status_t moe_grouped_gemm_down(const moe_bf16_t *act, const int32_t *offsets
 
 moe_status_t moe_finalize(const moe_bf16_t *y, const float *topk_w, const int32_t *inv_perm,
                           const moe_shape_t *shape, moe_bf16_t *out, moe_stream_t stream) {
+    const moe::NvtxRange nvtx("moe_finalize");
     moe_status_t st = check_shape(shape);
     if (st != MOE_OK) return st;
     if (shape->T == 0) return MOE_OK;
@@ -290,6 +295,7 @@ moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits, const vo
                          const moe_bf16_t *w_gu_scales, const void *w_d, const moe_bf16_t *w_d_scales,
                          const moe_shape_t *shape, moe_bf16_t *out, void *ws, size_t ws_bytes,
                          moe_stream_t stream) {
+    const moe::NvtxRange nvtx("moe_forward");
     moe_status_t st = check_shape(shape);
     if (st != MOE_OK) return st;
     if (shape->T == 0) return MOE_OK;
@@ -308,6 +314,7 @@ moe_status_t moe_forward_host(const moe_bf16_t *hidden_host, const float *logits
                               const moe_bf16_t *w_gu_scales, const void *w_d, const moe_bf16_t *w_d_scales,
                               const moe_shape_t *shape, moe_bf16_t *out_host, void *ws, size_t ws_bytes,
                               moe_stream_t stream) {
+    const moe::NvtxRange nvtx("moe_forward_host");
     moe_status_t st = check_shape(shape);
     if (st != MOE_OK) return st;
     if (shape->T == 0) return MOE_OK;
@@ -336,6 +343,7 @@ moe_status_t moe_forward_host(const moe_bf16_t *hidden_host, const float *logits
 
 moe_status_t moe_dequant_int4(const uint8_t *q, const moe_bf16_t *scales, int32_t rows, int32_t K,
                               moe_bf16_t *out, moe_stream_t stream) {
+    const moe::NvtxRange nvtx("moe_dequant_int4");
     if (rows < 0 || K <= 0 || K % 128) return MOE_ERR_INVALID_ARG;
     if (rows == 0) return MOE_OK;
     if (!q || !scales || !out || !aligned(q, 16) || !aligned(out, 16) || !aligned(scales, 2))
@@ -344,6 +352,7 @@ moe_status_t moe_dequant_int4(const uint8_t *q, const moe_bf16_t *scales, int32_
 }
 
 moe_status_t moe_get_device_error(int32_t *code) {
+    const moe::NvtxRange nvtx("moe_get_device_error");
     if (!code) return MOE_ERR_INVALID_ARG;
     if (cudaDeviceSynchronize() != cudaSuccess) return MOE_ERR_CUDA;
     int v = 0;
@@ -355,6 +364,7 @@ moe_status_t moe_get_device_error(int32_t *code) {
 }
 
 moe_status_t moe_selftest_bounded_wait(int64_t limit_ns, moe_stream_t stream) {
+    const moe::NvtxRange nvtx("moe_selftest_bounded_wait");
     if (limit_ns < 1 || limit_ns > 1000000000LL) return MOE_ERR_INVALID_ARG;
     return cuda_status(moe::launch_bounded_wait_selftest(static_cast<unsigned long long>(limit_ns), error_flag_ptr(),
                                                          static_cast<cudaStream_t>(stream)));

@@ -9,8 +9,19 @@
 #include <stdint.h>
 
 #include "moe.h"
+#include "nvtx3/nvToolsExt.h"
 
 namespace moe {
+
+// An NVTX range named after a C-ABI entry point, open for the host-side
+// duration of the call (argument checks and enqueueing). Costs a predicted
+// branch when no profiler has attached an NVTX tool.
+struct NvtxRange {
+    explicit NvtxRange(const char *name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 // ---- capi.cu
 // The shape rules every entry point applies (MOE_OK or the status to return).
@@ -80,6 +91,9 @@ cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t s);
 bool gemm_gathers_in_kernel(int P, int E, int fmt);
 // ---- gemm_prefill_sm100.cu: bf16, tokens on the MMA's M side (many tokens per expert)
 cudaError_t launch_grouped_gemm_prefill(const GemmArgs &g, cudaStream_t s);
+// ---- gemm_wm_pair_sm100.cu: bf16, weights on M across a CTA pair (M = 256),
+// tokens on N with N = the tile's rows rounded up to 16 (permuted rows, no perm)
+cudaError_t launch_grouped_gemm_wm_pair(const GemmArgs &g, cudaStream_t s);
 cudaError_t launch_dequant_int4(const uint8_t *q, const uint16_t *scales, int rows, int K, uint16_t *out,
                                 cudaStream_t s);
 

@@ -54,6 +54,7 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t *topk_ids, const moe_s
                                             int32_t *offsets, int32_t *perm, int32_t *inv_perm,
                                             const moe_bf16_t *hidden, moe_bf16_t *hidden_perm,
                                             moe_stream_t stream) {
+    const moe::NvtxRange nvtx("moe_permute_noalloc");
     // the same argument rules as moe_permute
     const moe_status_t st = moe::validate_shape(shape);
     if (st != MOE_OK) return st;
