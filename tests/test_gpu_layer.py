@@ -11,7 +11,7 @@ import moe_synth
 import oracle
 import mixture_experts_expert_top_b200 as moe
 from mixture_experts_expert_top_b200 import build as moe_build
-from _util import bf16_bits, bits_to_bf16, gemm_rows_close, layer_output_close
+from _util import bf16_bits, bits_to_bf16, gemm_rows_close, layer_output_close, weighted_abs_y
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -95,7 +95,8 @@ def test_layer_matches_oracle_on_every_element(name):
     gemm_rows_close(bf16_bits(y), r["y"], "y")
     fin = oracle.finalize(bf16_bits(s["y"]), s["w"].cpu().numpy(), s["inv_perm"].cpu().numpy(), cfg.T, cfg.H, cfg.k)
     assert np.array_equal(bf16_bits(s["out"]), fin)
-    layer_output_close(bf16_bits(out), r["out"], name, scale_abs_by_rms=cfg.fmt == "int4_g128")
+    y_abs = weighted_abs_y(bf16_bits(s["y"]), s["w"].cpu().numpy(), s["inv_perm"].cpu().numpy(), cfg.T, cfg.H, cfg.k)
+    layer_output_close(bf16_bits(out), r["out"], name, scale_abs_by_rms=cfg.fmt == "int4_g128", y_abs=y_abs)
 
 
 def test_layer_is_deterministic():
