@@ -202,8 +202,11 @@ MOE_API moe_status_t moe_dequant_int4(const uint8_t *q, const moe_bf16_t *scales
 
 /* Device error flag of the current device: waits for all work on the device,
  * stores the flag in *code (0 = none; 1 = bad expert id; 2 = a pipeline wait
- * timed out; 3 = a finalize row index out of range) and clears it. The first
- * error raised since the last read is the one kept. */
+ * timed out; 3 = a finalize row index out of range; 4 = a permutation entry
+ * or an expert offset out of range, caught only by the range-checking build
+ * libmoe_b200_debug.so, compiled from the same sources with
+ * -DMOE_DEBUG_BOUNDS, which then uses an in-range value instead) and clears
+ * it. The first error raised since the last read is the one kept. */
 MOE_API moe_status_t moe_get_device_error(int32_t *code);
 
 /* Self-test of the bounded waits behind device error code 2 (no counterpart

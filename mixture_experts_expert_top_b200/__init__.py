@@ -25,7 +25,7 @@ __all__ = [
     "moe_route", "moe_permute", "moe_grouped_gemm_swiglu", "moe_grouped_gemm_down",
     "moe_finalize", "moe_forward", "moe_forward_host", "moe_dequant_int4",
     "moe_get_device_error", "moe_status_string", "moe_permute_noalloc", "moe_selftest_bounded_wait",
-    "moe_forward_kernel_count", "moe_forward_gathers_in_gemm", "forward",
+    "moe_forward_kernel_count", "moe_forward_gathers_in_gemm", "forward", "debug_bounds_library",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -56,47 +56,77 @@ class Shape(ctypes.Structure):
 
 
 _lib: Optional[ctypes.CDLL] = None
+_debug_lib: Optional[ctypes.CDLL] = None
+_use_debug = False
 
 
 def lib() -> ctypes.CDLL:
-    global _lib
+    """The loaded library (libmoe_b200.so; inside `debug_bounds_library()`,
+    the range-checking build libmoe_b200_debug.so)."""
+    global _lib, _debug_lib
+    if _use_debug:
+        if _debug_lib is None:
+            _debug_lib = _load(True)
+        return _debug_lib
     if _lib is None:
-        from . import build as _build
-        if not _build.up_to_date():
-            # a missing or stale library is rebuilt from the sources (needs nvcc); never skipped
-            try:
-                _build.build()
-            except Exception as e:      # noqa: BLE001 - re-raised with the path
-                raise RuntimeError(f"{library_path} is missing or older than its sources and could not be "
-                                   f"built ({e}): build it with `python -m mixture_experts_expert_top_b200.build`")
-        L = ctypes.CDLL(library_path)
-        vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
-        sp = ctypes.POINTER(Shape)
-        sigs = {
-            "moe_workspace_size": ([sp], sz),
-            "moe_permute_workspace_size": ([sp], sz),
-            "moe_forward_host_workspace_size": ([sp], sz),
-            "moe_route": ([vp, sp, vp, vp, vp], ctypes.c_int),
-            "moe_permute": ([vp, sp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
-            "moe_grouped_gemm_swiglu": ([vp, vp, vp, vp, vp, sp, vp, vp], ctypes.c_int),
-            "moe_grouped_gemm_down": ([vp, vp, vp, vp, sp, vp, vp], ctypes.c_int),
-            "moe_finalize": ([vp, vp, vp, sp, vp, vp], ctypes.c_int),
-            "moe_forward": ([vp, vp, vp, vp, vp, vp, sp, vp, vp, sz, vp], ctypes.c_int),
-            "moe_forward_host": ([vp, vp, vp, vp, vp, vp, sp, vp, vp, sz, vp], ctypes.c_int),
-            "moe_dequant_int4": ([vp, vp, i32, i32, vp, vp], ctypes.c_int),
-            "moe_permute_noalloc": ([vp, sp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
-            "moe_get_device_error": ([ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
-            "moe_selftest_bounded_wait": ([ctypes.c_int64, vp], ctypes.c_int),
-            "moe_forward_kernel_count": ([sp], ctypes.c_int32),
-            "moe_forward_gathers_in_gemm": ([sp], ctypes.c_int32),
-            "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
-        }
-        for name, (args, res) in sigs.items():
-            f = getattr(L, name)
-            f.argtypes = args
-            f.restype = res
-        _lib = L
+        _lib = _load(False)
     return _lib
+
+
+class debug_bounds_library:
+    """Context manager: the entry points of this module call the build made
+    with -DMOE_DEBUG_BOUNDS (perm-derived rows and expert offsets range-checked
+    in the kernels, device error 4 on a bad one) while it is active."""
+
+    def __enter__(self):
+        global _use_debug
+        self._prev = _use_debug
+        _use_debug = True
+        return lib()
+
+    def __exit__(self, *exc):
+        global _use_debug
+        _use_debug = self._prev
+        return False
+
+
+def _load(debug_bounds: bool) -> ctypes.CDLL:
+    from . import build as _build
+    path = _build.LIB_DEBUG if debug_bounds else library_path
+    if not _build.up_to_date(debug_bounds):
+        # a missing or stale library is rebuilt from the sources (needs nvcc); never skipped
+        try:
+            _build.build(debug_bounds=debug_bounds)
+        except Exception as e:      # noqa: BLE001 - re-raised with the path
+            raise RuntimeError(f"{path} is missing or older than its sources and could not be "
+                               f"built ({e}): build it with `python -m mixture_experts_expert_top_b200.build`")
+    L = ctypes.CDLL(path)
+    vp, sz, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32
+    sp = ctypes.POINTER(Shape)
+    sigs = {
+        "moe_workspace_size": ([sp], sz),
+        "moe_permute_workspace_size": ([sp], sz),
+        "moe_forward_host_workspace_size": ([sp], sz),
+        "moe_route": ([vp, sp, vp, vp, vp], ctypes.c_int),
+        "moe_permute": ([vp, sp, vp, vp, vp, vp, vp, vp, vp, sz, vp], ctypes.c_int),
+        "moe_grouped_gemm_swiglu": ([vp, vp, vp, vp, vp, sp, vp, vp], ctypes.c_int),
+        "moe_grouped_gemm_down": ([vp, vp, vp, vp, sp, vp, vp], ctypes.c_int),
+        "moe_finalize": ([vp, vp, vp, sp, vp, vp], ctypes.c_int),
+        "moe_forward": ([vp, vp, vp, vp, vp, vp, sp, vp, vp, sz, vp], ctypes.c_int),
+        "moe_forward_host": ([vp, vp, vp, vp, vp, vp, sp, vp, vp, sz, vp], ctypes.c_int),
+        "moe_dequant_int4": ([vp, vp, i32, i32, vp, vp], ctypes.c_int),
+        "moe_permute_noalloc": ([vp, sp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
+        "moe_get_device_error": ([ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
+        "moe_selftest_bounded_wait": ([ctypes.c_int64, vp], ctypes.c_int),
+        "moe_forward_kernel_count": ([sp], ctypes.c_int32),
+        "moe_forward_gathers_in_gemm": ([sp], ctypes.c_int32),
+        "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    }
+    for name, (args, res) in sigs.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    return L
 
 
 # ---- marshalling helpers ---------------------------------------------------

@@ -157,7 +157,7 @@ moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const
         e = moe::launch_grouped_gemm(gu, st);
     } else {
         auto *hperm = reinterpret_cast<uint16_t *>(ws + L.hperm);
-        if ((e = moe::launch_gather(hidden, perm, P, H, k, hperm, st)) != cudaSuccess) return cuda_status(e);
+        if ((e = moe::launch_gather(hidden, perm, P, H, k, hperm, error_flag_ptr(), st)) != cudaSuccess) return cuda_status(e);
         e = moe::launch_grouped_gemm(gemm_args(s, hperm, nullptr, offsets, w_gu, w_gu_scales, true, act), st);
     }
     if (e != cudaSuccess) return cuda_status(e);
@@ -226,7 +226,7 @@ moe_status_t moe_permute(const int32_t *topk_ids, const moe_shape_t *shape, int3
     cudaError_t e = moe::launch_permute(topk_ids, static_cast<int>(P), shape->E, counts, offsets, perm, inv_perm, ws,
                                         error_flag_ptr(), s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    if (hidden) e = moe::launch_gather(hidden, perm, static_cast<int>(P), shape->H, shape->top_k, hidden_perm, s);
+    if (hidden) e = moe::launch_gather(hidden, perm, static_cast<int>(P), shape->H, shape->top_k, hidden_perm, error_flag_ptr(), s);
     return cuda_status(e);
 }
 

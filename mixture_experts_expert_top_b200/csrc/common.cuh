@@ -11,7 +11,17 @@
 namespace moe {
 
 // Device error codes (the flag word moe_get_device_error reads).
-enum : int { kErrBadExpertId = 1, kErrTimeout = 2, kErrBadRow = 3 };
+enum : int { kErrBadExpertId = 1, kErrTimeout = 2, kErrBadRow = 3, kErrBounds = 4 };
+
+// Built with -DMOE_DEBUG_BOUNDS (libmoe_b200_debug.so): every row index read
+// from perm and every expert offset is range-checked before it addresses
+// memory or a TMA load; a bad one raises kErrBounds and is replaced by an
+// in-range value, so the access is skipped rather than made.
+#ifdef MOE_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
 
 // A pipeline wait that has not completed after this long gives up, raises
 // kErrTimeout and lets the kernel unwind instead of hanging the GPU.

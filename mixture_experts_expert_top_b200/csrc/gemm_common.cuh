@@ -71,20 +71,40 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int *pre, const 
 // gather mode (rows past P read row 0; they are never stored), else r.
 __device__ __forceinline__ int token_row(const Params &p, int r) {
     if (!p.perm) return r;
-    return r < p.P ? __ldg(p.perm + r) / p.top_k : 0;
+    if (r >= p.P) return 0;
+    int v = __ldg(p.perm + r);
+    if (kDebugBounds && (v < 0 || v >= p.P)) {
+        raise_error(p.err, kErrBounds);
+        v = 0;
+    }
+    return v / p.top_k;
 }
 
 // Copies offsets into shared memory and builds pre[e] = number of tiles of
 // experts 0..e-1 (a block-wide scan). All threads of the CTA call it.
 template <int NT>
 __device__ __forceinline__ void build_tile_prefix(const int32_t *offsets, int E, int MB, int BN, int *off_s,
-                                                  int *pre_s) {
+                                                  int *pre_s, int P = 0, int *err = nullptr) {
     __shared__ int wsum[NT / 32];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // L2 reads (no L1 line can be stale): a kernel launched with an early
     // start may read offsets before griddepcontrol.wait (kGemmHintOffsetsReady)
     for (int i = threadIdx.x; i <= E; i += NT) off_s[i] = __ldcg(offsets + i);
     __syncthreads();
+    if (kDebugBounds && threadIdx.x == 0) {
+        // offsets must start at 0, never decrease and end at P
+        bool bad = off_s[0] != 0 || off_s[E] != P;
+        int prev = 0;
+        for (int i = 0; i <= E; ++i) {
+            const int v = min(max(off_s[i], prev), P);
+            bad |= v != off_s[i];
+            off_s[i] = v;
+            prev = v;
+        }
+        off_s[0] = 0;
+        if (bad) raise_error(err, kErrBounds);
+    }
+    if (kDebugBounds) __syncthreads();
     const int seg = (E + NT - 1) / NT;
     const int b0 = threadIdx.x * seg;
     int local = 0;

@@ -142,7 +142,7 @@ grouped_gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
     // tiles of expert e: ceil(rows / 128) token blocks x NB feature blocks
     // barriers, tensor maps and TMEM are set up while the previous kernel drains
     griddep_wait();
-    build_tile_prefix<192>(p.offsets, E, NB, kTokM, off_s, pre_s);
+    build_tile_prefix<192>(p.offsets, E, NB, kTokM, off_s, pre_s, p.P, p.err);
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
@@ -326,7 +326,7 @@ grouped_gemm_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmA, const 
     }
     // barriers, tensor maps and TMEM are set up while the previous kernel drains
     griddep_wait();
-    build_tile_prefix<192>(p.offsets, E, NB, kPairRows, off_s, pre_s);
+    build_tile_prefix<192>(p.offsets, E, NB, kPairRows, off_s, pre_s, p.P, p.err);
     tc_fence_before_sync();
     __syncthreads();
     cluster_sync();                                          // barriers of both CTAs initialised
@@ -483,6 +483,9 @@ cudaError_t run_prefill(const GemmArgs &g, cudaStream_t s) {
 
 cudaError_t launch_grouped_gemm_prefill(const GemmArgs &g, cudaStream_t s) {
     if (g.P == 0) return cudaSuccess;
+    // rows already permuted: weights on M across CTA pairs, runtime token N
+    // (gemm_wm_pair_sm100.cu)
+    if (!g.perm) return launch_grouped_gemm_wm_pair(g, s);
     // CTA pairs when the token blocks are long enough for 256-row tiles to pay
     // (few rows lost to the last tile of each expert); single CTAs otherwise.
     const bool pairs = !g.perm && static_cast<long long>(g.P) >= kPairMinRowsPerExpert * g.E;

@@ -158,7 +158,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
         griddep_wait();
     }
-    build_tile_prefix<C::kThreads>(p.offsets, E, MB, BN, off_s, pre_s);
+    build_tile_prefix<C::kThreads>(p.offsets, E, MB, BN, off_s, pre_s, p.P, p.err);
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
@@ -394,7 +394,7 @@ grouped_gemm_int4_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_c
     }
     // barriers, tensor maps and TMEM are set up while the previous kernel drains
     griddep_wait();
-    build_tile_prefix<C::kThreads>(p.offsets, E, MB, BN, off_s, pre_s);
+    build_tile_prefix<C::kThreads>(p.offsets, E, MB, BN, off_s, pre_s, p.P, p.err);
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();

@@ -53,7 +53,7 @@ int permute_kernel_count(long long P, int E);
 cudaError_t launch_permute(const int32_t *ids, int P, int E, int32_t *counts, int32_t *offsets, int32_t *perm,
                            int32_t *inv_perm, void *scratch, int *err, cudaStream_t s);
 cudaError_t launch_gather(const uint16_t *hidden, const int32_t *perm, int P, int H, int k, uint16_t *hidden_perm,
-                          cudaStream_t s);
+                          int *err, cudaStream_t s);
 
 // ---- finalize.cu
 cudaError_t launch_finalize(const uint16_t *y, const float *w, const int32_t *inv_perm, int T, int H, int k,

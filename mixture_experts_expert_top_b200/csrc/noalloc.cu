@@ -74,6 +74,6 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t *topk_ids, const moe_s
     cudaError_t e = moe::launch_permute(topk_ids, static_cast<int>(P), shape->E, counts, offsets, perm, inv_perm,
                                         scratch, moe::device_error_flag(), s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    if (hidden) e = moe::launch_gather(hidden, perm, static_cast<int>(P), shape->H, shape->top_k, hidden_perm, s);
+    if (hidden) e = moe::launch_gather(hidden, perm, static_cast<int>(P), shape->H, shape->top_k, hidden_perm, moe::device_error_flag(), s);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -200,13 +200,17 @@ permute_scatter_kernel(const int32_t *__restrict__ ids, int P, int E, const int3
 // hidden_perm[r] = hidden[perm[r] / k]: one warp per row, 16-byte vectors.
 __global__ void __launch_bounds__(256)
 gather_rows_kernel(const uint4 *__restrict__ hidden, const int32_t *__restrict__ perm, int P, int vecs_per_row,
-                   int k, uint4 *__restrict__ out) {
+                   int k, uint4 *__restrict__ out, int *err) {
     griddep_launch_dependents();
     griddep_wait();
     const int lane = threadIdx.x & 31;
     const int warps = gridDim.x * (blockDim.x >> 5);
     for (int r = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); r < P; r += warps) {
-        const int p = __ldg(perm + r);
+        int p = __ldg(perm + r);
+        if (kDebugBounds && (p < 0 || p >= P)) {
+            raise_error(err, kErrBounds);
+            p = 0;
+        }
         const uint4 *src = hidden + static_cast<size_t>(p / k) * vecs_per_row;
         uint4 *dst = out + static_cast<size_t>(r) * vecs_per_row;
         // all loads of a 4 KB slice are in flight before its stores; the copy is
@@ -277,13 +281,14 @@ cudaError_t launch_permute(const int32_t *ids, int P, int E, int32_t *counts, in
 }
 
 cudaError_t launch_gather(const uint16_t *hidden, const int32_t *perm, int P, int H, int k, uint16_t *hidden_perm,
-                          cudaStream_t s) {
+                          int *err, cudaStream_t s) {
     if (P == 0) return cudaSuccess;
     const int rows_per_block = 8;
     int blocks = (P + rows_per_block - 1) / rows_per_block;
     if (blocks > 148 * 16) blocks = 148 * 16;
     return launch_pdl(gather_rows_kernel, dim3(blocks), dim3(32 * rows_per_block), 0, s,
-                      reinterpret_cast<const uint4 *>(hidden), perm, P, H / 8, k, reinterpret_cast<uint4 *>(hidden_perm));
+                      reinterpret_cast<const uint4 *>(hidden), perm, P, H / 8, k, reinterpret_cast<uint4 *>(hidden_perm),
+                      err);
 }
 
 }  // namespace moe

@@ -41,6 +41,21 @@ def test_library_exports_every_declared_symbol():
         assert hasattr(lib, n), n
 
 
+def test_debug_bounds_library_builds_and_exports_every_declared_symbol():
+    # the -DMOE_DEBUG_BOUNDS build of the same sources (range checks in the
+    # kernels, device error 4) is a drop-in replacement for the release library
+    path = moe_build.build(debug_bounds=True)
+    assert path != moe.library_path
+    lib = ctypes.CDLL(path)
+    for n in declared_entry_points():
+        assert hasattr(lib, n), n
+    with moe.debug_bounds_library() as L:
+        assert moe.lib() is L
+        assert moe.moe_workspace_size(moe.Shape.of(64, 2048, 768, 128, 8)) == \
+            ctypes.CDLL(moe.library_path).moe_workspace_size(ctypes.byref(moe.Shape.of(64, 2048, 768, 128, 8)))
+    assert moe.lib() is not L
+
+
 def test_binding_names_match_the_header():
     for n in declared_entry_points():
         assert callable(getattr(moe, n)), n
