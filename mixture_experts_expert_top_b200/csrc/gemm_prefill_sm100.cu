@@ -1,4 +1,6 @@
-// gemm_prefill_sm100.cu -- grouped GEMMs for many tokens per expert (bf16).
+// gemm_prefill_sm100.cu -- grouped GEMMs for many tokens per expert (bf16)
+// whose token rows are read through perm (TMA gather4) rather than from a
+// permuted copy; permuted copies go to gemm_wm_pair_sm100.cu.
 //
 // Same results as the kernels of gemm_sm100.cu (InfiniLM PR #500 Qwen3-MoE
 // report, §2.2 step 2: gate/up with SwiGLU, then down, over every expert's
@@ -31,7 +33,6 @@ constexpr int kTileA = kTokM * kBK * 2;             // 16 KB
 constexpr int kTileB = kRowsB * kBK * 2;            // 32 KB
 constexpr int kStageBytes = kTileA + kTileB;        // 48 KB
 constexpr int kAccCols = kRowsB;                    // fp32 accumulator columns per buffer
-constexpr long long kPairMinRowsPerExpert = 256;    // average rows per expert for the CTA-pair kernel
 
 // Reads this thread's accumulator row (kFeat output features) from TMEM and
 // packs it to bf16 pairs: SwiGLU over columns c (gate) and 128 + c (up), or
@@ -257,206 +258,6 @@ grouped_gemm_prefill_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
     }
 }
 
-// ---------------------------------------------------------------------------
-// CTA-pair variant: a cluster of two CTAs computes a 256-token x 256 tile with
-// M = 256 tcgen05.mma.cta_group::2. Each CTA loads its own 128 token rows and
-// half of the 256 weight rows (gate rows in the leading CTA and up rows in
-// the other for gate/up; two 128-feature halves for down), so per SM the
-// shared-memory traffic per FLOP is half that of the single-CTA kernel. Only
-// the leading CTA issues MMAs; its commits arrive on both CTAs' barriers.
-constexpr int kPairRows = 2 * kTokM;                 // token rows per pair tile
-constexpr int kHalfB = 128 * kBK * 2;                // 16 KB: this CTA's half of B
-constexpr int kPairStage = kTileA + kHalfB;          // 32 KB
-
-template <int STAGES>
-struct PairCfg {
-    static constexpr int kRingBytes = STAGES * kPairStage;
-    static constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1;
-    static constexpr int kSmemBytes = 1024 + kRingBytes + 8 * kNumBars + 64 + 2 * (kMaxExperts + 1) * 4;
-    static_assert(kSmemBytes + 64 <= kSmemLimit, "shared memory");
-};
-
-template <bool SWIGLU, int STAGES>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
-grouped_gemm_prefill_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                                 const Params p) {
-    using C = PairCfg<STAGES>;
-    constexpr int kFeat = SWIGLU ? 128 : 256;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    uint8_t *ring = smem;                                    // STAGES x [A own tokens | B own half]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + C::kRingBytes);
-    uint64_t *full_bar = bars;                               // used in the leading CTA: both CTAs' bytes
-    uint64_t *empty_bar = full_bar + STAGES;                 // each CTA's own (MMA commit to both)
-    uint64_t *tfull_bar = empty_bar + STAGES;                // each CTA's own (MMA commit to both)
-    uint64_t *tempty_bar = tfull_bar + 2;                    // used in the leading CTA: 8 warp arrivals
-    uint64_t *drain_bar = tempty_bar + 2;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain_bar + 1);
-    volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
-    int *off_s = reinterpret_cast<int *>(tmem_holder + 16);
-    int *pre_s = off_s + (kMaxExperts + 1);
-
-    const int warp = threadIdx.x >> 5;
-    const int lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_ctarank();                 // 0 = leading CTA of the pair
-    const int E = p.E;
-    const int NB = (p.m_out + kFeat - 1) / kFeat;
-    const int KB = (p.K + kBK - 1) / kBK;
-
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full_bar[s], 1);
-            mbar_init(&empty_bar[s], 1);
-        }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&tfull_bar[b], 1);
-            mbar_init(&tempty_bar[b], 8);      // 4 epilogue warps in each of the two CTAs
-        }
-        mbar_init(drain_bar, 1);
-        *abort_flag = 0;
-        fence_mbar_init();
-    }
-    if (warp == 0 && lane == 0) {
-        prefetch_tmap(&tmA);
-        prefetch_tmap(&tmB);
-    }
-    if (warp == 1) {
-        tmem_alloc_pair(tmem_holder, 2 * kAccCols);
-        tmem_relinquish_pair();
-    }
-    // barriers, tensor maps and TMEM are set up while the previous kernel drains
-    griddep_wait();
-    build_tile_prefix<192>(p.offsets, E, NB, kPairRows, off_s, pre_s, p.P, p.err);
-    tc_fence_before_sync();
-    __syncthreads();
-    cluster_sync();                                          // barriers of both CTAs initialised
-    tc_fence_after_sync();
-    const uint32_t tmem_base = *tmem_holder;
-    const int total_tiles = pre_s[E];
-    const int first_tile = static_cast<int>(cluster_id_x());
-    const int tile_step = static_cast<int>(cluster_count_x());
-
-    if (warp == 0) {
-        // ============================ TMA producer (both CTAs) ==================
-        if (lane == 0) {
-            const uint64_t pol = l2_policy_evict_last();
-            int stage = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            for (int tile = first_tile; tile < total_tiles && ok; tile += tile_step) {
-                const TileInfo ti = decode_tile(tile, pre_s, off_s, E, NB, kPairRows);
-                const int f0 = ti.mb * kFeat;
-                const int a_row = ti.row0 + static_cast<int>(rank) * kTokM;
-                const int b_row = ti.e * p.w_rows + f0 + static_cast<int>(rank) * (SWIGLU ? p.m_out : 128);
-                for (int kb = 0; kb < KB; ++kb) {
-                    ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.err, 256);
-                    if (!ok) break;
-                    const uint32_t full_leader = cluster_map(smem_u32(&full_bar[stage]), 0);
-                    if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], 2 * kPairStage);
-                    uint8_t *st = ring + stage * kPairStage;
-                    tma_load_2d_pair(st, &tmA, full_leader, kb * kBK, a_row, pol);
-                    tma_load_2d_pair(st + kTileA, &tmB, full_leader, kb * kBK, b_row, pol);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                }
-            }
-        }
-    } else if (warp == 1) {
-        // ============================ MMA issuer (leading CTA) ==================
-        if (lane == 0 && rank == 0) {
-            const uint32_t idesc = idesc_bf16_f32(kPairRows, kRowsB);
-            int stage = 0;
-            uint32_t phase = 0;
-            int buf = 0;
-            uint32_t bphase = 0;
-            bool ok = true;
-            for (int tile = first_tile; tile < total_tiles && ok; tile += tile_step) {
-                ok = mbar_wait(&tempty_bar[buf], bphase ^ 1, abort_flag, p.err);
-                if (!ok) break;
-                tc_fence_after_sync();
-                const uint32_t d = tmem_base + buf * kAccCols;
-                for (int kb = 0; kb < KB; ++kb) {
-                    ok = mbar_wait(&full_bar[stage], phase, abort_flag, p.err, 0);
-                    if (!ok) break;
-                    tc_fence_after_sync();
-                    const uint32_t st = smem_u32(ring + stage * kPairStage);
-                    const uint64_t da = sw128_kmajor_desc(st);
-                    const uint64_t db = sw128_kmajor_desc(st + kTileA);
-#pragma unroll
-                    for (int k = 0; k < kBK / 16; ++k)
-                        umma_bf16_ss_pair(d, da + 2 * k, db + 2 * k, idesc, (kb | k) != 0);
-                    umma_commit_pair(&empty_bar[stage], 0x3);
-                    if (++stage == STAGES) { stage = 0; phase ^= 1; }
-                }
-                if (!ok) break;
-                umma_commit_pair(&tfull_bar[buf], 0x3);
-                if (++buf == 2) { buf = 0; bphase ^= 1; }
-            }
-            umma_commit_pair(drain_bar, 0x1);
-            volatile int never = 0;
-            mbar_wait(drain_bar, 0, &never, p.err);
-        }
-    } else {
-        // ====================== warps 2-5: epilogue (both CTAs) =================
-        const int q = warp & 3;
-        const int tr = q * 32 + lane;                       // this CTA's token row owned by this thread
-        int buf = 0;
-        uint32_t bphase = 0;
-        for (int tile = first_tile; tile < total_tiles; tile += tile_step) {
-            const TileInfo ti = decode_tile(tile, pre_s, off_s, E, NB, kPairRows);
-            if (!mbar_wait(&tfull_bar[buf], bphase, abort_flag, p.err, 512)) break;
-            tc_fence_after_sync();
-            const int f0 = ti.mb * kFeat;
-            const int my_row0 = ti.row0 + static_cast<int>(rank) * kTokM;
-            const bool row_ok = static_cast<int>(rank) * kTokM + tr < ti.valid;
-            uint16_t *orow = p.out + static_cast<size_t>(my_row0 + (row_ok ? tr : 0)) * p.m_out;
-            const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * kAccCols;
-            uint32_t packed[kFeat / 2];
-            load_acc_row<SWIGLU>(tb, packed);
-            tc_fence_before_sync();
-            __syncwarp();
-            // buffer free before the stores go out (the release then covers
-            // only the previous tile's stores, long since drained)
-            if (lane == 0) mbar_arrive_cluster(cluster_map(smem_u32(&tempty_bar[buf]), 0));
-            if (row_ok) store_row<kFeat>(orow, f0, p.m_out, packed);
-            if (++buf == 2) { buf = 0; bphase ^= 1; }
-        }
-    }
-
-    // every role is done: the next kernel may start its set-up now
-    griddep_launch_dependents();
-    __syncthreads();
-    if (*abort_flag) {
-        for (int i = 0; i < 1000; ++i) __nanosleep(1000);
-    }
-    cluster_sync();                                          // no remote arrival or MMA left in flight
-    if (warp == 1) {
-        tc_fence_after_sync();
-        tmem_dealloc_pair(tmem_base, 2 * kAccCols);
-    }
-}
-
-template <bool SWIGLU>
-cudaError_t run_prefill_pair(const GemmArgs &g, cudaStream_t s) {
-    constexpr int STAGES = 6;
-    using C = PairCfg<STAGES>;
-    CUtensorMap ta, tb;
-    const uint64_t b_rows = static_cast<uint64_t>(g.E) * g.w_rows;
-    bool ok = make_token_map(&ta, g, kTokM) &&
-              make_map(&tb, g.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.K, b_rows, kBK, 128,
-                       CU_TENSOR_MAP_SWIZZLE_128B);
-    if (!ok || g.perm) return cudaErrorInvalidValue;
-    auto kern = grouped_gemm_prefill_pair_kernel<SWIGLU, STAGES>;
-    cudaError_t st = ensure_dynamic_smem(kern, C::kSmemBytes);
-    if (st != cudaSuccess) return st;
-    constexpr int kFeat = SWIGLU ? 128 : 256;
-    const long long NB = (g.m_out + kFeat - 1) / kFeat;
-    const long long max_tiles = ((static_cast<long long>(g.P) + kPairRows - 1) / kPairRows + std::min(g.E, g.P)) * NB;
-    const int pairs = static_cast<int>(std::min<long long>(num_sms() / 2, max_tiles));
-    if (pairs <= 0) return cudaSuccess;
-    Params p = make_params(g, kPairRows);
-    return launch_pdl(kern, dim3(2 * pairs), dim3(192), C::kSmemBytes, s, ta, tb, p);
-}
-
 template <bool SWIGLU>
 cudaError_t run_prefill(const GemmArgs &g, cudaStream_t s) {
     constexpr int STAGES = 4;
@@ -484,12 +285,8 @@ cudaError_t run_prefill(const GemmArgs &g, cudaStream_t s) {
 cudaError_t launch_grouped_gemm_prefill(const GemmArgs &g, cudaStream_t s) {
     if (g.P == 0) return cudaSuccess;
     // rows already permuted: weights on M across CTA pairs, runtime token N
-    // (gemm_wm_pair_sm100.cu)
+    // (gemm_wm_pair_sm100.cu); rows read through perm: this file's kernel
     if (!g.perm) return launch_grouped_gemm_wm_pair(g, s);
-    // CTA pairs when the token blocks are long enough for 256-row tiles to pay
-    // (few rows lost to the last tile of each expert); single CTAs otherwise.
-    const bool pairs = !g.perm && static_cast<long long>(g.P) >= kPairMinRowsPerExpert * g.E;
-    if (pairs) return g.swiglu ? run_prefill_pair<true>(g, s) : run_prefill_pair<false>(g, s);
     return g.swiglu ? run_prefill<true>(g, s) : run_prefill<false>(g, s);
 }
 

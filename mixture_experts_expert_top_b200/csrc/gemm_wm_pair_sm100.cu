@@ -25,9 +25,10 @@
 //  - Epilogue threads own one feature each; a warp stores 32 consecutive
 //    features (64 bytes) of each token row.
 // Warp roles: warp 0 TMA (both CTAs), warp 1 MMA (leading CTA) and TMEM
-// owner, warps 2-5 epilogue over a double-buffered 2 x 256-column fp32
-// accumulator; each epilogue warp loads the next 32 accumulator columns while
-// it stores the current ones and hands the buffer back after its last load.
+// owner, warps 2-9 epilogue over a double-buffered 2 x 256-column fp32
+// accumulator: two sets of 4 warps split a tile's columns, each warp loads the
+// next 32 columns while it stores the current ones and hands the buffer back
+// right after its last tcgen05.ld of the tile.
 // Every mbarrier wait is bounded; the named-barrier hand-off between epilogue
 // warps is entered only after a bounded wait succeeded, and both warps of a
 // pair take the same number of steps.
@@ -41,17 +42,24 @@ using namespace gemm;
 
 constexpr int kPairM = 256;                          // weight rows per pair tile (MMA M)
 constexpr int kTokBlock = 256;                       // token rows per tile at most (MMA N)
-constexpr int kABox = 64;                            // weight rows per TMA box
-constexpr int kBBox = 32;                            // token rows per TMA box
+constexpr int kABox = 64;                            // weight rows per TMA box (gate/up: gate and up halves)
+constexpr int kBBox = 128;                           // token rows per TMA box: one box per stage
 constexpr int kTileA = 128 * kBK * 2;                // 16 KB: this CTA's 128 weight rows
 constexpr int kTileB = (kTokBlock / 2) * kBK * 2;    // 16 KB: up to 128 token rows of this CTA
-constexpr int kBBoxBytes = kBBox * kBK * 2;          // 4 KB
+constexpr int kBBoxBytes = kBBox * kBK * 2;          // 16 KB
 constexpr int kStage = kTileA + kTileB;              // 32 KB
 constexpr int kAccCols = kTokBlock;                  // fp32 accumulator columns per buffer
-constexpr int kXchgBytes = 2 * 2 * 2 * 16 * 32 * 4;  // gate/up hand-off: 2 warp pairs x 2 buffers x 2 x 16 x 32 fp32
+constexpr int kPairXchgBytes = 2 * 2 * 16 * 32 * 4;  // one warp pair's gate/up hand-off: 2 buffers x 2 x 16 x 32 fp32
 
-template <int STAGES>
+// 8 epilogue warps: two sets of 4 (one per TMEM lane quarter), each set
+// covering half of a tile's 32-column chunks, so that a tile's accumulator is
+// read and handed back in half the time; for gate/up the 8 form 4 gate/up
+// warp pairs.
+template <bool SWIGLU, int STAGES>
 struct WmPairCfg {
+    static constexpr int kEpiWarps = 8;
+    static constexpr int kThreads = 64 + 32 * kEpiWarps;
+    static constexpr int kXchgBytes = SWIGLU ? 4 * kPairXchgBytes : 0;
     static constexpr int kRingBytes = STAGES * kStage;
     static constexpr int kNumBars = 2 * STAGES + 2 + 2 + 1;
     static constexpr int kSmemBytes =
@@ -60,11 +68,10 @@ struct WmPairCfg {
 };
 
 // Named barriers of the gate/up epilogue (barrier 0 is __syncthreads): per
-// warp pair q (gate warp q, up warp q + 2), "go" carries the gate warp's
-// decision for the tile, "xchg" separates the writes and reads of one chunk's
-// hand-off buffer.
-__device__ __forceinline__ int bar_go(int q) { return 1 + q; }
-__device__ __forceinline__ int bar_xchg(int q) { return 3 + q; }
+// warp pair pq (0-3), "go" carries the gate warp's decision for the tile,
+// "xchg" separates the writes and reads of one chunk's hand-off buffer.
+__device__ __forceinline__ int bar_go(int pq) { return 1 + pq; }
+__device__ __forceinline__ int bar_xchg(int pq) { return 5 + pq; }
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -75,16 +82,16 @@ __device__ __forceinline__ uint16_t bf16_rn_bits(float v) {
 }
 
 template <bool SWIGLU, int STAGES>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(320, 1)
 grouped_gemm_wm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                             const Params p) {
-    using C = WmPairCfg<STAGES>;
+    using C = WmPairCfg<SWIGLU, STAGES>;
     constexpr int kFeatPerTile = SWIGLU ? 128 : 256;         // output features per pair tile
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint8_t *ring = smem;                                    // STAGES x [A own 128 rows | B own rows]
     float *xchg = reinterpret_cast<float *>(ring + C::kRingBytes);   // gate/up hand-off buffers
-    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + C::kRingBytes + kXchgBytes);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(ring + C::kRingBytes + C::kXchgBytes);
     uint64_t *full_bar = bars;                               // used in the leading CTA: both CTAs' bytes
     uint64_t *empty_bar = full_bar + STAGES;                 // each CTA's own (MMA commit to both)
     uint64_t *tfull_bar = empty_bar + STAGES;                // each CTA's own (MMA commit to both)
@@ -92,7 +99,7 @@ grouped_gemm_wm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
     uint64_t *drain_bar = tempty_bar + 2;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
-    volatile int *go_flag = reinterpret_cast<volatile int *>(tmem_holder + 2);     // [2]
+    volatile int *go_flag = reinterpret_cast<volatile int *>(tmem_holder + 2);     // [4]
     int *off_s = reinterpret_cast<int *>(tmem_holder + 16);
     int *pre_s = off_s + (kMaxExperts + 1);
 
@@ -110,7 +117,7 @@ grouped_gemm_wm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull_bar[b], 1);
-            mbar_init(&tempty_bar[b], 8);      // 4 epilogue warps in each of the two CTAs
+            mbar_init(&tempty_bar[b], 2 * C::kEpiWarps);      // every epilogue warp of both CTAs
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -129,7 +136,7 @@ grouped_gemm_wm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
     // stages need not wait for it (only the token rows do).
     const bool early = (p.hints & kGemmHintOffsetsReady) != 0;
     if (!early) griddep_wait();
-    build_tile_prefix<192>(p.offsets, E, MB, kTokBlock, off_s, pre_s, p.P, p.err);
+    build_tile_prefix<C::kThreads>(p.offsets, E, MB, kTokBlock, off_s, pre_s, p.P, p.err);
     tc_fence_before_sync();
     __syncthreads();
     cluster_sync();                                          // barriers of both CTAs initialised
@@ -153,8 +160,8 @@ grouped_gemm_wm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
                     r0 = ti.e * p.w_rows + ti.mb * 128 + 64 * rank;     // gate rows
                     r1 = r0 + p.m_out;                                  // the matching up rows
                 } else {
-                    r0 = ti.e * p.w_rows + ti.mb * 256 + 128 * rank;
-                    r1 = r0 + kABox;
+                    r0 = ti.e * p.w_rows + ti.mb * 256 + 128 * rank;   // one 128-row box
+                    r1 = -1;
                 }
             };
             int preloaded = 0;
@@ -170,7 +177,7 @@ grouped_gemm_wm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
                         if (rank == 0) mbar_arrive_expect_tx(&full_bar[preloaded], tx);
                         uint8_t *st = ring + preloaded * kStage;
                         tma_load_2d_pair(st, &tmA, full_leader, kb * kBK, r0, pol_w);
-                        tma_load_2d_pair(st + kTileA / 2, &tmA, full_leader, kb * kBK, r1, pol_w);
+                        if (SWIGLU) tma_load_2d_pair(st + kTileA / 2, &tmA, full_leader, kb * kBK, r1, pol_w);
                     }
                 }
                 griddep_wait();
@@ -192,7 +199,7 @@ grouped_gemm_wm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
                     if (it >= preloaded) {
                         if (rank == 0) mbar_arrive_expect_tx(&full_bar[stage], tx);
                         tma_load_2d_pair(st, &tmA, full_leader, kb * kBK, r0, pol_w);
-                        tma_load_2d_pair(st + kTileA / 2, &tmA, full_leader, kb * kBK, r1, pol_w);
+                        if (SWIGLU) tma_load_2d_pair(st + kTileA / 2, &tmA, full_leader, kb * kBK, r1, pol_w);
                     }
                     for (int b = 0; b < nbox; ++b)
                         tma_load_2d_pair(st + kTileA + b * kBBoxBytes, &tmB, full_leader, kb * kBK,
@@ -239,7 +246,7 @@ grouped_gemm_wm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
             mbar_wait(drain_bar, 0, &never, p.err);
         }
     } else {
-        // ====================== warps 2-5: epilogue (both CTAs) =================
+        // ====================== warps 2+: epilogue (both CTAs) ==================
         if (early) griddep_wait();
         const int q = warp & 3;                              // TMEM lane quarter of this warp
         const uint32_t tempty_leader0 = cluster_map(smem_u32(&tempty_bar[0]), 0);
@@ -254,33 +261,49 @@ grouped_gemm_wm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
             if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
         };
         if (!SWIGLU) {
+            // warps 2-5 store the first half of a tile's 32-column chunks,
+            // warps 6-9 the second half, each warp its 32 features
+            const int h = (warp - 2) >> 2;
             const int f_in_tile = 128 * rank + 32 * q + lane;
             for (int tile = first_tile; tile < total_tiles; tile += tile_step) {
                 const TileInfo ti = decode_tile(tile, pre_s, off_s, E, MB, kTokBlock);
                 if (!__shfl_sync(0xffffffffu, mbar_wait(&tfull_bar[buf], bphase, abort_flag, p.err, 512), 0)) break;
                 tc_fence_after_sync();
+                const int nch = (ti.valid + 31) >> 5;
+                const int split = (nch + 1) >> 1;
+                const int c_lo = h ? split : 0, c_hi = h ? nch : split;
+                if (c_lo >= c_hi) {
+                    release();
+                    if (++buf == 2) { buf = 0; bphase ^= 1; }
+                    continue;
+                }
                 const int f = ti.mb * kFeatPerTile + f_in_tile;
                 const bool f_ok = f < p.m_out;
                 const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * kAccCols;
                 uint16_t *col = p.out + static_cast<size_t>(ti.row0) * p.m_out + f;
+                const size_t row_stride = static_cast<size_t>(p.m_out);
                 auto store = [&](const uint32_t (&v)[32], int c0) {
                     if (!f_ok) return;
+                    uint16_t *dst = col + static_cast<size_t>(c0) * row_stride;
+                    const int n = min(32, ti.valid - c0);
 #pragma unroll
-                    for (int j = 0; j < 32; ++j)
-                        if (c0 + j < ti.valid)
-                            col[static_cast<size_t>(c0 + j) * p.m_out] = bf16_rn_bits(__uint_as_float(v[j]));
+                    for (int j = 0; j < 32; ++j) {
+                        if (j < n) *dst = bf16_rn_bits(__uint_as_float(v[j]));
+                        dst += row_stride;
+                    }
                 };
                 // two register sets: the next 32 columns load while this set is stored
+                const int c_end = 32 * c_hi;
                 uint32_t va[32], vb[32];
-                tmem_ld_32x32b_x32(tb, va);
+                tmem_ld_32x32b_x32(tb + 32 * c_lo, va);
                 tmem_wait_ld();
-                for (int c0 = 0;; c0 += 64) {
-                    const bool more_a = c0 + 32 < ti.valid;
+                for (int c0 = 32 * c_lo;; c0 += 64) {
+                    const bool more_a = c0 + 32 < c_end;
                     if (more_a) tmem_ld_32x32b_x32(tb + c0 + 32, vb); else release();
                     store(va, c0);
                     if (!more_a) break;
                     tmem_wait_ld();
-                    const bool more_b = c0 + 64 < ti.valid;
+                    const bool more_b = c0 + 64 < c_end;
                     if (more_b) tmem_ld_32x32b_x32(tb + c0 + 64, va); else release();
                     store(vb, c0 + 32);
                     if (!more_b) break;
@@ -289,16 +312,18 @@ grouped_gemm_wm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
                 if (++buf == 2) { buf = 0; bphase ^= 1; }
             }
         } else {
-            // Warp pair (gate warp q < 2, up warp q + 2) shares 32 features of
-            // each 32-token chunk: the gate warp hands g of tokens 16-31 to the
-            // up warp, the up warp hands u of tokens 0-15 to the gate warp, and
-            // each forms act for its 16 tokens. Two hand-off buffers alternate,
-            // so one barrier per chunk orders every write after the partner's
-            // read of the same buffer two chunks earlier.
+            // Warp pair (gate warp q < 2, up warp q + 2, same column half h)
+            // shares 32 features of each 32-token chunk of its half of the
+            // tile: the gate warp hands g of tokens 16-31 to the up warp, the
+            // up warp hands u of tokens 0-15 to the gate warp, and each forms
+            // act for its 16 tokens. Two hand-off buffers alternate, so one
+            // barrier per chunk orders every write after the partner's read
+            // of the same buffer two chunks earlier.
+            const int h = (warp - 2) >> 2;                   // column half: warps 2-5 first, 6-9 second
             const bool gate_warp = q < 2;
-            const int pq = q & 1;                            // warp pair index
-            float *xb = xchg + pq * (2 * 2 * 16 * 32);       // [buffer][giver: gate, up][16 tokens][32 lanes]
-            const int f_in_tile = 64 * rank + 32 * pq + lane;
+            const int pq = (q & 1) + 2 * h;                  // warp pair index
+            float *xb = xchg + pq * (kPairXchgBytes / 4);    // [buffer][giver: gate, up][16 tokens][32 lanes]
+            const int f_in_tile = 64 * rank + 32 * (q & 1) + lane;
             uint32_t xbuf = 0;
             for (int tile = first_tile; tile < total_tiles; tile += tile_step) {
                 const TileInfo ti = decode_tile(tile, pre_s, off_s, E, MB, kTokBlock);
@@ -315,6 +340,15 @@ grouped_gemm_wm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
                 // once and orders this warp's TMEM reads after the MMAs
                 if (!gate_warp) mbar_wait(&tfull_bar[buf], bphase, abort_flag, p.err, 512);
                 tc_fence_after_sync();
+                // this half's columns: chunks [c_lo, c_hi) of 32
+                const int nch = (ti.valid + 31) >> 5;
+                const int split = (nch + 1) >> 1;
+                const int c_lo = h ? split : 0, c_hi = h ? nch : split;
+                if (c_lo >= c_hi) {
+                    release();
+                    if (++buf == 2) { buf = 0; bphase ^= 1; }
+                    continue;
+                }
                 const int f = ti.mb * kFeatPerTile + f_in_tile;
                 const bool f_ok = f < p.m_out;
                 // this warp's 16 tokens of each chunk: 0-15 (gate warp) or 16-31 (up warp)
@@ -341,16 +375,17 @@ grouped_gemm_wm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
                     }
                     xbuf ^= 1;
                 };
+                const int c_end = 32 * c_hi;
                 uint32_t va[32], vb[32];
-                tmem_ld_32x32b_x32(tb, va);
+                tmem_ld_32x32b_x32(tb + 32 * c_lo, va);
                 tmem_wait_ld();
-                for (int c0 = 0;; c0 += 64) {
-                    const bool more_a = c0 + 32 < ti.valid;
+                for (int c0 = 32 * c_lo;; c0 += 64) {
+                    const bool more_a = c0 + 32 < c_end;
                     if (more_a) tmem_ld_32x32b_x32(tb + c0 + 32, vb); else release();
                     chunk(va, c0);
                     if (!more_a) break;
                     tmem_wait_ld();
-                    const bool more_b = c0 + 64 < ti.valid;
+                    const bool more_b = c0 + 64 < c_end;
                     if (more_b) tmem_ld_32x32b_x32(tb + c0 + 64, va); else release();
                     chunk(vb, c0 + 32);
                     if (!more_b) break;
@@ -376,11 +411,11 @@ grouped_gemm_wm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
 
 template <bool SWIGLU>
 cudaError_t run_wm_pair(const GemmArgs &g, cudaStream_t s) {
-    constexpr int STAGES = 6;
-    using C = WmPairCfg<STAGES>;
+    constexpr int STAGES = SWIGLU ? 5 : 6;
+    using C = WmPairCfg<SWIGLU, STAGES>;
     CUtensorMap ta, tb;
     const uint64_t a_rows = static_cast<uint64_t>(g.E) * g.w_rows;
-    bool ok = make_map(&ta, g.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.K, a_rows, kBK, kABox,
+    bool ok = make_map(&ta, g.w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.K, a_rows, kBK, SWIGLU ? kABox : 128,
                        CU_TENSOR_MAP_SWIZZLE_128B) &&
               make_map(&tb, g.a, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, g.K, static_cast<uint64_t>(g.P), kBK, kBBox,
                        CU_TENSOR_MAP_SWIZZLE_128B);
@@ -396,7 +431,7 @@ cudaError_t run_wm_pair(const GemmArgs &g, cudaStream_t s) {
     if (pairs <= 0) return cudaSuccess;
     Params p = make_params(g, kTokBlock);
     p.evict_first_weights = 0;
-    return launch_pdl(kern, dim3(2 * pairs), dim3(192), C::kSmemBytes, s, ta, tb, p);
+    return launch_pdl(kern, dim3(2 * pairs), dim3(C::kThreads), C::kSmemBytes, s, ta, tb, p);
 }
 
 }  // namespace
