@@ -299,6 +299,44 @@ def test_grouped_gemm_swiglu_gathers_through_perm(cfg):
     gemm_rows_close(bf16_bits(act_g), r["act"], "act (gathered)")
 
 
+RAGGED_EXPERTS = [
+    # (rows per expert, H, I): tails of 1, 15, 17 rows, one row past a 256-row
+    # block, empty experts, and H / I that are not multiples of 64 or 128
+    ([1, 15, 17, 255, 257, 0, 512, 16, 256, 33], 512, 384),
+    ([257, 1, 0, 17, 255, 100], 264, 200),
+    ([300, 700, 3, 0, 0, 129], 1024, 768),
+]
+
+
+@pytest.mark.parametrize("counts,H,I", RAGGED_EXPERTS, ids=lambda x: str(x))
+def test_grouped_gemms_on_ragged_experts_match_oracle(counts, H, I):
+    """Many rows per expert (weights on M across a CTA pair, token N set per
+    tile at run time): every row of every expert against the oracle's FFN of
+    that row, with experts whose row counts end anywhere in a 256-row block."""
+    E = len(counts)
+    P = sum(counts)
+    assert P >= 64 * E            # the shapes that take the many-rows-per-expert kernels
+    g = torch.Generator().manual_seed(P + H + I)
+    a = (torch.randn(P, H, generator=g)).to(torch.bfloat16)
+    w_gu = (torch.randn(E, 2 * I, H, generator=g) * 0.02).to(torch.bfloat16)
+    w_d = (torch.randn(E, H, I, generator=g) * 0.02).to(torch.bfloat16)
+    offsets = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    ref_act = np.zeros((P, I), np.uint16)
+    ref_y = np.zeros((P, H), np.uint16)
+    for e in range(E):
+        for r in range(offsets[e], offsets[e + 1]):
+            ref_act[r], ref_y[r] = oracle.expert_ffn(a[r], w_gu[e], w_d[e], H, I)
+    sh = moe.Shape.of(P, H, I, E, 1)
+    d_off = dev(offsets)
+    act = torch.empty(P, I, dtype=torch.bfloat16, device=DEV)
+    moe.moe_grouped_gemm_swiglu(dev(a), None, d_off, dev(w_gu), None, sh, act)
+    y = torch.empty(P, H, dtype=torch.bfloat16, device=DEV)
+    moe.moe_grouped_gemm_down(dev(bits_to_bf16(ref_act)), d_off, dev(w_d), None, sh, y)
+    torch.cuda.synchronize()
+    gemm_rows_close(bf16_bits(act), ref_act, "act")
+    gemm_rows_close(bf16_bits(y), ref_y, "y")
+
+
 def test_grouped_gemm_int4_matches_oracle():
     cfg = moe_synth.MoeConfig("int4_mid", T=48, H=1024, I=384, E=12, k=4, fmt="int4_g128")
     test_grouped_gemm_swiglu_and_down_match_oracle(cfg)
