@@ -26,8 +26,11 @@
  *    H and I multiples of 8 (multiples of 128 for MOE_W_INT4_G128).
  *    Device pointers must be 16-byte aligned (4-byte for logits/topk_w and
  *    the int32 arrays).
- *  - Pair ids: p = t*top_k + j for token t and slot j. Slot order is
- *    descending logit; equal logits go to the lower expert id.
+ *  - Pair ids: p = t*K + j for token t and slot j, with K = top_k +
+ *    n_shared slots per token. Routed slot order is descending logit; equal
+ *    logits go to the lower expert id; shared slots follow.
+ *  - Below, "T*top_k" and "E" in array sizes of permute, the GEMMs and
+ *    finalize mean T*(top_k + n_shared) and E + n_shared.
  *  - No C++ exception crosses this interface. Entry points are reentrant
  *    given distinct workspaces and outputs.
  *  - The library keeps, per device, the device address of its error flag
@@ -66,10 +69,22 @@ typedef enum {
     MOE_W_INT4_G128 = 1    /* W4A16: int4 weights, one bf16 scale per 128 K */
 } moe_weight_fmt_t;
 
-/* Layer shape. T tokens, hidden size H, expert intermediate size I, E experts,
- * top_k experts per token, fmt a moe_weight_fmt_t. */
+/* Layer shape. T tokens, hidden size H, expert intermediate size I, E routed
+ * experts, top_k routed experts per token, fmt a moe_weight_fmt_t, n_shared
+ * shared experts (set it to 0 when there are none).
+ *
+ * Shared experts (GC-MoE abstract: MoE layers with shared experts next to the
+ * routed ones): every token also goes through experts E .. E+n_shared-1 of
+ * the weight arrays, whose outputs are added with weight 1:
+ *   out[t] = sum_{j<top_k} w_j FFN_{e_j}(x_t) + sum_{s<n_shared} FFN_{E+s}(x_t)
+ * They are carried as extra slots of each token: the routing arrays are
+ * [T, top_k + n_shared], slot top_k + s holds expert E + s with weight 1.0,
+ * and permute, the grouped GEMMs and finalize see E + n_shared experts and
+ * top_k + n_shared slots. The finalize sum therefore adds the shared
+ * experts after the routed slots, in slot order.
+ * Limits: top_k + n_shared <= 32 and E + n_shared <= 1024. */
 typedef struct {
-    int32_t T, H, I, E, top_k, fmt;
+    int32_t T, H, I, E, top_k, fmt, n_shared;
 } moe_shape_t;
 
 typedef uint16_t moe_bf16_t;   /* bit pattern of a bfloat16 value */
@@ -88,10 +103,13 @@ MOE_API size_t moe_permute_workspace_size(const moe_shape_t *shape);
 
 /* Route. InfiniLM PR #500 report §2.1/§2.4 (top-k softmax routing) with
  * renormalisation over the selected experts.
- *   logits   [T,E] fp32 (finite values; NaN is treated as -inf)
- *   topk_ids [T,top_k] int32 out: expert ids in slot order
- *   topk_w   [T,top_k] fp32 out: w_j = exp(l_j - l_0) / sum_i exp(l_i - l_0),
- *            sums to one; one warp per token, expf, fp32 sum in slot order. */
+ *   logits   [T,E] fp32 (NaN ranks as -inf; -0 equals +0)
+ *   topk_ids [T,top_k+n_shared] int32 out: expert ids in slot order, then
+ *            E .. E+n_shared-1
+ *   topk_w   [T,top_k+n_shared] fp32 out: w_j = exp(l_j - l_0) /
+ *            sum_i exp(l_i - l_0) over the routed slots (they sum to one;
+ *            one warp per token, expf, fp32 sum in slot order), then 1.0 for
+ *            each shared slot. */
 MOE_API moe_status_t moe_route(const float *logits, const moe_shape_t *shape,
                        int32_t *topk_ids, float *topk_w, moe_stream_t stream);
 

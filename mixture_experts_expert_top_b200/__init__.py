@@ -45,14 +45,26 @@ class MoeError(RuntimeError):
 
 
 class Shape(ctypes.Structure):
+    """moe_shape_t: E routed experts and top_k routed slots per token, plus
+    n_shared shared experts (experts E.. of the weight arrays, one extra slot
+    each with weight 1)."""
     _fields_ = [("T", ctypes.c_int32), ("H", ctypes.c_int32), ("I", ctypes.c_int32),
-                ("E", ctypes.c_int32), ("top_k", ctypes.c_int32), ("fmt", ctypes.c_int32)]
+                ("E", ctypes.c_int32), ("top_k", ctypes.c_int32), ("fmt", ctypes.c_int32),
+                ("n_shared", ctypes.c_int32)]
 
     @classmethod
-    def of(cls, T, H, I, E, top_k, fmt=FMT_BF16) -> "Shape":
+    def of(cls, T, H, I, E, top_k, fmt=FMT_BF16, n_shared=0) -> "Shape":
         if isinstance(fmt, str):
             fmt = {"bf16": FMT_BF16, "int4_g128": FMT_INT4_G128}[fmt]
-        return cls(int(T), int(H), int(I), int(E), int(top_k), int(fmt))
+        return cls(int(T), int(H), int(I), int(E), int(top_k), int(fmt), int(n_shared))
+
+    @property
+    def slots(self) -> int:
+        return self.top_k + self.n_shared
+
+    @property
+    def experts(self) -> int:
+        return self.E + self.n_shared
 
 
 _lib: Optional[ctypes.CDLL] = None
@@ -279,12 +291,14 @@ def forward(hidden: torch.Tensor, logits: torch.Tensor, w_gu: torch.Tensor, w_d:
             out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """moe_forward on device tensors; allocates out and the workspace with
     torch when they are not given. hidden [T,H] bf16, logits [T,E] fp32,
-    w_gu [E,2I,H] bf16 (or uint8 [E,2I,H/2] + scales), w_d [E,H,I] (or uint8)."""
+    w_gu [E+S,2I,H] bf16 (or uint8 [E+S,2I,H/2] + scales), w_d [E+S,H,I] (or
+    uint8): weight arrays with more experts than logits columns hold S shared
+    experts after the E routed ones."""
     T, H = hidden.shape
     E = logits.shape[1]
     fmt = FMT_INT4_G128 if w_gu.dtype == torch.uint8 else FMT_BF16
     I = w_d.shape[2] * (2 if fmt == FMT_INT4_G128 else 1)
-    shape = Shape.of(T, H, I, E, top_k, fmt)
+    shape = Shape.of(T, H, I, E, top_k, fmt, n_shared=w_gu.shape[0] - E)
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=hidden.device)
     if ws is None:

@@ -37,16 +37,22 @@ int *error_flag_ptr() {
 
 inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Slots per token (routed, then shared) and experts in the weight arrays.
+inline int slots(const moe_shape_t *s) { return s->top_k + s->n_shared; }
+inline int experts(const moe_shape_t *s) { return s->E + s->n_shared; }
+
 moe_status_t check_shape(const moe_shape_t *s) {
     if (!s) return MOE_ERR_INVALID_ARG;
-    if (s->T < 0 || s->H <= 0 || s->I <= 0 || s->E < 1 || s->top_k < 1 || s->top_k > s->E)
+    if (s->T < 0 || s->H <= 0 || s->I <= 0 || s->E < 1 || s->top_k < 1 || s->top_k > s->E || s->n_shared < 0)
         return MOE_ERR_INVALID_ARG;
     if (s->fmt != MOE_W_BF16 && s->fmt != MOE_W_INT4_G128) return MOE_ERR_INVALID_ARG;
-    if (s->E > 1024 || s->top_k > 32) return MOE_ERR_UNSUPPORTED;
+    if (static_cast<long long>(s->E) + s->n_shared > 1024 || static_cast<long long>(s->top_k) + s->n_shared > 32)
+        return MOE_ERR_UNSUPPORTED;
     if (s->H % 8 || s->I % 8) return MOE_ERR_UNSUPPORTED;
     if (s->fmt == MOE_W_INT4_G128 && (s->H % 128 || s->I % 128)) return MOE_ERR_UNSUPPORTED;
-    if (static_cast<long long>(s->T) * s->top_k >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
-    if (static_cast<long long>(s->E) * 2 * s->I >= (1LL << 31) || static_cast<long long>(s->E) * s->H >= (1LL << 31))
+    if (static_cast<long long>(s->T) * slots(s) >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
+    if (static_cast<long long>(experts(s)) * 2 * s->I >= (1LL << 31) ||
+        static_cast<long long>(experts(s)) * s->H >= (1LL << 31))
         return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
@@ -63,7 +69,8 @@ struct Layout {
 };
 
 Layout layout(const moe_shape_t *s, bool host) {
-    const size_t P = static_cast<size_t>(s->T) * s->top_k;
+    const size_t P = static_cast<size_t>(s->T) * slots(s);
+    const int E = experts(s);
     Layout L;
     size_t o = 0;
     auto take = [&](size_t bytes) {
@@ -73,12 +80,12 @@ Layout layout(const moe_shape_t *s, bool host) {
     };
     L.ids = take(P * 4);
     L.w = take(P * 4);
-    L.counts = take(static_cast<size_t>(s->E) * 4);
-    L.offsets = take(static_cast<size_t>(s->E + 1) * 4);
+    L.counts = take(static_cast<size_t>(E) * 4);
+    L.offsets = take(static_cast<size_t>(E + 1) * 4);
     L.perm = take(P * 4);
     L.inv = take(P * 4);
-    L.scratch = take(moe::permute_scratch_bytes(static_cast<long long>(P), s->E));
-    L.hperm = moe::gemm_gathers_in_kernel(static_cast<int>(P), s->E, s->fmt) ? o : take(P * s->H * 2);
+    L.scratch = take(moe::permute_scratch_bytes(static_cast<long long>(P), E));
+    L.hperm = moe::gemm_gathers_in_kernel(static_cast<int>(P), E, s->fmt) ? o : take(P * s->H * 2);
     L.act = take(P * s->I * 2);
     L.y = take(P * s->H * 2);
     L.hidden_in = L.logits_in = L.out_st = 0;
@@ -97,12 +104,12 @@ moe::GemmArgs gemm_args(const moe_shape_t *s, const void *a, const int32_t *perm
     g.a = a;
     g.perm = perm;
     g.T = s->T;
-    g.top_k = s->top_k;
+    g.top_k = slots(s);
     g.offsets = offsets;
     g.w = w;
     g.w_scales = scales;
-    g.P = s->T * s->top_k;
-    g.E = s->E;
+    g.P = s->T * slots(s);
+    g.E = experts(s);
     g.K = swiglu ? s->H : s->I;
     g.m_out = swiglu ? s->I : s->H;
     g.w_rows = swiglu ? 2 * s->I : s->H;
@@ -127,7 +134,10 @@ moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const
                             const moe_bf16_t *w_gu_scales, const void *w_d, const moe_bf16_t *w_d_scales,
                             const moe_shape_t *s, moe_bf16_t *out, uint8_t *ws, const Layout &L,
                             cudaStream_t st) {
-    const int T = s->T, k = s->top_k, E = s->E, H = s->H;
+    // routing: top_k of the E routed experts, then the shared slots; every
+    // later step sees K = top_k + n_shared slots over E + n_shared experts
+    const int T = s->T, kr = s->top_k, Er = s->E, S = s->n_shared, H = s->H;
+    const int k = slots(s), E = experts(s);
     const int P = T * k;
     auto *ids = reinterpret_cast<int32_t *>(ws + L.ids);
     auto *w = reinterpret_cast<float *>(ws + L.w);
@@ -139,10 +149,10 @@ moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const
     auto *y = reinterpret_cast<uint16_t *>(ws + L.y);
     cudaError_t e;
     if (moe::route_permute_fusable(T, E, k)) {
-        e = moe::launch_route_permute(logits, T, E, k, ids, w, counts, offsets, perm, inv, error_flag_ptr(), st);
+        e = moe::launch_route_permute(logits, T, Er, kr, S, ids, w, counts, offsets, perm, inv, error_flag_ptr(), st);
         if (e != cudaSuccess) return cuda_status(e);
     } else {
-        if ((e = moe::launch_route(logits, T, E, k, ids, w, st)) != cudaSuccess) return cuda_status(e);
+        if ((e = moe::launch_route(logits, T, Er, kr, S, ids, w, st)) != cudaSuccess) return cuda_status(e);
         if ((e = moe::launch_permute(ids, P, E, counts, offsets, perm, inv, ws + L.scratch, error_flag_ptr(), st)) !=
             cudaSuccess)
             return cuda_status(e);
@@ -173,6 +183,8 @@ moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const
 
 namespace moe {
 moe_status_t validate_shape(const moe_shape_t *shape) { return check_shape(shape); }
+int shape_slots(const moe_shape_t *shape) { return slots(shape); }
+int shape_experts(const moe_shape_t *shape) { return experts(shape); }
 int *device_error_flag() { return error_flag_ptr(); }
 }  // namespace moe
 
@@ -190,7 +202,7 @@ size_t moe_forward_host_workspace_size(const moe_shape_t *shape) {
 
 size_t moe_permute_workspace_size(const moe_shape_t *shape) {
     if (check_shape(shape) != MOE_OK) return 0;
-    return moe::permute_scratch_bytes(static_cast<long long>(shape->T) * shape->top_k, shape->E);
+    return moe::permute_scratch_bytes(static_cast<long long>(shape->T) * slots(shape), experts(shape));
 }
 
 moe_status_t moe_route(const float *logits, const moe_shape_t *shape, int32_t *topk_ids, float *topk_w,
@@ -201,8 +213,8 @@ moe_status_t moe_route(const float *logits, const moe_shape_t *shape, int32_t *t
     if (shape->T == 0) return MOE_OK;
     if (!logits || !topk_ids || !topk_w || !aligned(logits, 4) || !aligned(topk_ids, 4) || !aligned(topk_w, 4))
         return MOE_ERR_INVALID_ARG;
-    return cuda_status(moe::launch_route(logits, shape->T, shape->E, shape->top_k, topk_ids, topk_w,
-                                         static_cast<cudaStream_t>(stream)));
+    return cuda_status(moe::launch_route(logits, shape->T, shape->E, shape->top_k, shape->n_shared, topk_ids,
+                                         topk_w, static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_permute(const int32_t *topk_ids, const moe_shape_t *shape, int32_t *counts, int32_t *offsets,
@@ -212,21 +224,24 @@ moe_status_t moe_permute(const int32_t *topk_ids, const moe_shape_t *shape, int3
     moe_status_t st = check_shape(shape);
     if (st != MOE_OK) return st;
     if (shape->T == 0) return MOE_OK;
-    const long long P = static_cast<long long>(shape->T) * shape->top_k;
+    const long long P = static_cast<long long>(shape->T) * slots(shape);
+    const int E = experts(shape);
     if (!counts || !offsets || !aligned(counts, 4) || !aligned(offsets, 4)) return MOE_ERR_INVALID_ARG;
     if (P > 0 && (!topk_ids || !perm || !inv_perm || !aligned(topk_ids, 4) || !aligned(perm, 4) ||
                   !aligned(inv_perm, 4)))
         return MOE_ERR_INVALID_ARG;
     if ((hidden == nullptr) != (hidden_perm == nullptr)) return MOE_ERR_INVALID_ARG;
     if (hidden && (!aligned(hidden, 16) || !aligned(hidden_perm, 16))) return MOE_ERR_INVALID_ARG;
-    const size_t need = moe::permute_scratch_bytes(P, shape->E);
+    const size_t need = moe::permute_scratch_bytes(P, E);
     if (need > 0 && (!ws || ws_bytes < need)) return MOE_ERR_WORKSPACE_TOO_SMALL;
     if (ws && !aligned(ws, 16)) return MOE_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = moe::launch_permute(topk_ids, static_cast<int>(P), shape->E, counts, offsets, perm, inv_perm, ws,
+    cudaError_t e = moe::launch_permute(topk_ids, static_cast<int>(P), E, counts, offsets, perm, inv_perm, ws,
                                         error_flag_ptr(), s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    if (hidden) e = moe::launch_gather(hidden, perm, static_cast<int>(P), shape->H, shape->top_k, hidden_perm, error_flag_ptr(), s);
+    if (hidden)
+        e = moe::launch_gather(hidden, perm, static_cast<int>(P), shape->H, slots(shape), hidden_perm,
+                               error_flag_ptr(), s);
     return cuda_status(e);
 }
 
@@ -268,14 +283,14 @@ moe_status_t moe_finalize(const moe_bf16_t *y, const float *topk_w, const int32_
     if (!y || !topk_w || !inv_perm || !out || !aligned(y, 16) || !aligned(out, 16) || !aligned(topk_w, 4) ||
         !aligned(inv_perm, 4))
         return MOE_ERR_INVALID_ARG;
-    return cuda_status(moe::launch_finalize(y, topk_w, inv_perm, shape->T, shape->H, shape->top_k, out,
+    return cuda_status(moe::launch_finalize(y, topk_w, inv_perm, shape->T, shape->H, slots(shape), out,
                                             error_flag_ptr(), static_cast<cudaStream_t>(stream)));
 }
 
 int32_t moe_forward_kernel_count(const moe_shape_t *shape) {
     if (check_shape(shape) != MOE_OK) return -1;
     if (shape->T == 0) return 0;
-    const int T = shape->T, k = shape->top_k, E = shape->E;
+    const int T = shape->T, k = slots(shape), E = experts(shape);
     const long long P = static_cast<long long>(T) * k;
     int32_t n = 0;
     if (moe::route_permute_fusable(T, E, k))
@@ -288,7 +303,7 @@ int32_t moe_forward_kernel_count(const moe_shape_t *shape) {
 
 int32_t moe_forward_gathers_in_gemm(const moe_shape_t *shape) {
     if (check_shape(shape) != MOE_OK) return -1;
-    return moe::gemm_gathers_in_kernel(shape->T * shape->top_k, shape->E, shape->fmt) ? 1 : 0;
+    return moe::gemm_gathers_in_kernel(shape->T * slots(shape), experts(shape), shape->fmt) ? 1 : 0;
 }
 
 moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits, const void *w_gu,

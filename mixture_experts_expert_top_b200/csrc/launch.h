@@ -26,6 +26,10 @@ struct NvtxRange {
 // ---- capi.cu
 // The shape rules every entry point applies (MOE_OK or the status to return).
 moe_status_t validate_shape(const moe_shape_t *shape);
+// Slots per token (top_k routed + n_shared shared) and experts in the weight
+// arrays (E routed + n_shared shared): what permute, the GEMMs and finalize see.
+int shape_slots(const moe_shape_t *shape);
+int shape_experts(const moe_shape_t *shape);
 // Device address of the library's error flag word on the current device.
 int *device_error_flag();
 
@@ -35,14 +39,20 @@ int *device_error_flag();
 cudaError_t launch_bounded_wait_selftest(unsigned long long limit_ns, int *err, cudaStream_t s);
 
 // ---- route.cu
-cudaError_t launch_route(const float *logits, int T, int E, int k, int32_t *ids, float *w, cudaStream_t s);
+// ids/w rows hold k routed slots, then n_shared slots of experts E.. with
+// weight 1 (row stride k + n_shared).
+cudaError_t launch_route(const float *logits, int T, int E, int k, int n_shared, int32_t *ids, float *w,
+                         cudaStream_t s);
 
 // ---- route_permute.cu
 // Routing and bucketing of a small batch by one CTA (same outputs as
 // launch_route followed by launch_permute).
+// E and k here count all experts and slots (shared included).
 bool route_permute_fusable(int T, int E, int k);
-cudaError_t launch_route_permute(const float *logits, int T, int E, int k, int32_t *ids, float *w, int32_t *counts,
-                                 int32_t *offsets, int32_t *perm, int32_t *inv_perm, int *err, cudaStream_t s);
+// E routed experts, k routed slots, n_shared shared experts / slots.
+cudaError_t launch_route_permute(const float *logits, int T, int E, int k, int n_shared, int32_t *ids, float *w,
+                                 int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv_perm, int *err,
+                                 cudaStream_t s);
 
 // ---- permute.cu
 // Scratch bytes the permute needs for P pairs over E experts (0 when a

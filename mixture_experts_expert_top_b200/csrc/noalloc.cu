@@ -59,21 +59,24 @@ extern "C" moe_status_t moe_permute_noalloc(const int32_t *topk_ids, const moe_s
     const moe_status_t st = moe::validate_shape(shape);
     if (st != MOE_OK) return st;
     if (shape->T == 0) return MOE_OK;
-    const long long P = static_cast<long long>(shape->T) * shape->top_k;
+    const long long P = static_cast<long long>(shape->T) * moe::shape_slots(shape);
+    const int E = moe::shape_experts(shape);
     if (!counts || !offsets || !topk_ids || !perm || !inv_perm || !aligned(counts, 4) || !aligned(offsets, 4) ||
         !aligned(topk_ids, 4) || !aligned(perm, 4) || !aligned(inv_perm, 4))
         return MOE_ERR_INVALID_ARG;
     if ((hidden == nullptr) != (hidden_perm == nullptr)) return MOE_ERR_INVALID_ARG;
     if (hidden && (!aligned(hidden, 16) || !aligned(hidden_perm, 16))) return MOE_ERR_INVALID_ARG;
     // the chunk histogram must fit the built-in array
-    if (moe::permute_scratch_bytes(P, shape->E) > sizeof(int32_t) * static_cast<size_t>(kScratchInts))
+    if (moe::permute_scratch_bytes(P, E) > sizeof(int32_t) * static_cast<size_t>(kScratchInts))
         return MOE_ERR_UNSUPPORTED;
     int32_t *scratch = scratch_ptr();
     if (!scratch) return MOE_ERR_CUDA;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    cudaError_t e = moe::launch_permute(topk_ids, static_cast<int>(P), shape->E, counts, offsets, perm, inv_perm,
+    cudaError_t e = moe::launch_permute(topk_ids, static_cast<int>(P), E, counts, offsets, perm, inv_perm,
                                         scratch, moe::device_error_flag(), s);
     if (e != cudaSuccess) return MOE_ERR_CUDA;
-    if (hidden) e = moe::launch_gather(hidden, perm, static_cast<int>(P), shape->H, shape->top_k, hidden_perm, moe::device_error_flag(), s);
+    if (hidden)
+        e = moe::launch_gather(hidden, perm, static_cast<int>(P), shape->H, moe::shape_slots(shape), hidden_perm,
+                               moe::device_error_flag(), s);
     return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -72,4 +72,13 @@ __device__ __forceinline__ void route_token(const float *row, int E, int k, int 
     my_w = __fdiv_rn(ej, sum);
 }
 
+// Lane j >= k of a routed token takes shared slot j - k: expert E + j - k,
+// weight 1 (the shared experts' outputs are added unweighted).
+__device__ __forceinline__ void shared_slot(int lane, int k, int E, int &id, float &w) {
+    if (lane >= k) {
+        id = E + lane - k;
+        w = 1.0f;
+    }
+}
+
 }  // namespace moe

@@ -24,12 +24,15 @@ constexpr int kMaxExperts = 256;    // at most 8 logits per lane
 
 template <int PER_LANE>
 __global__ void __launch_bounds__(kThreads, 1)
-route_permute_kernel(const float *__restrict__ logits, int T, int E, int k, int32_t *__restrict__ ids,
+route_permute_kernel(const float *__restrict__ logits, int T, int E, int k, int n_shared, int32_t *__restrict__ ids,
                      float *__restrict__ w, int32_t *__restrict__ counts, int32_t *__restrict__ offsets,
                      int32_t *__restrict__ perm, int32_t *__restrict__ inv_perm, int *err) {
+    // E routed experts and k routed slots; the bucketing sees E + n_shared
+    // experts and K = k + n_shared slots per token
+    const int K = k + n_shared, Et = E + n_shared;
     extern __shared__ int smem[];
-    int *bucket_smem = smem;                                   // [(32 + 2) * E]
-    int32_t *ids_s = smem + (kThreads / 32 + 2) * E;           // [T * k]
+    int *bucket_smem = smem;                                   // [(32 + 2) * Et]
+    int32_t *ids_s = smem + (kThreads / 32 + 2) * Et;          // [T * K]
     griddep_launch_dependents();
     griddep_wait();
     const int lane = threadIdx.x & 31;
@@ -37,24 +40,26 @@ route_permute_kernel(const float *__restrict__ logits, int T, int E, int k, int3
         int id;
         float wt;
         route_token<PER_LANE>(logits + static_cast<size_t>(t) * E, E, k, id, wt);
-        if (lane < k) {
-            ids[static_cast<size_t>(t) * k + lane] = id;
-            w[static_cast<size_t>(t) * k + lane] = wt;
-            ids_s[t * k + lane] = id;
+        shared_slot(lane, k, E, id, wt);
+        if (lane < K) {
+            ids[static_cast<size_t>(t) * K + lane] = id;
+            w[static_cast<size_t>(t) * K + lane] = wt;
+            ids_s[t * K + lane] = id;
         }
     }
     __syncthreads();
-    bucket_single_cta<kThreads>(ids_s, T * k, E, counts, offsets, perm, inv_perm, bucket_smem, err);
+    bucket_single_cta<kThreads>(ids_s, T * K, Et, counts, offsets, perm, inv_perm, bucket_smem, err);
 }
 
 template <int PER_LANE>
-cudaError_t launch_t(const float *logits, int T, int E, int k, int32_t *ids, float *w, int32_t *counts,
+cudaError_t launch_t(const float *logits, int T, int E, int k, int n_shared, int32_t *ids, float *w, int32_t *counts,
                      int32_t *offsets, int32_t *perm, int32_t *inv_perm, int *err, cudaStream_t s) {
-    const size_t sm = (static_cast<size_t>(kThreads / 32 + 2) * E + static_cast<size_t>(T) * k) * sizeof(int);
+    const int K = k + n_shared, Et = E + n_shared;
+    const size_t sm = (static_cast<size_t>(kThreads / 32 + 2) * Et + static_cast<size_t>(T) * K) * sizeof(int);
     const cudaError_t st = ensure_dynamic_smem(route_permute_kernel<PER_LANE>, sm);
     if (st != cudaSuccess) return st;
-    return launch_pdl(route_permute_kernel<PER_LANE>, dim3(1), dim3(kThreads), sm, s, logits, T, E, k, ids, w,
-                      counts, offsets, perm, inv_perm, err);
+    return launch_pdl(route_permute_kernel<PER_LANE>, dim3(1), dim3(kThreads), sm, s, logits, T, E, k, n_shared,
+                      ids, w, counts, offsets, perm, inv_perm, err);
 }
 
 }  // namespace
@@ -63,14 +68,15 @@ bool route_permute_fusable(int T, int E, int k) {
     return T > 0 && T <= kMaxTokens && static_cast<long long>(T) * k <= kMaxPairs && E <= kMaxExperts;
 }
 
-cudaError_t launch_route_permute(const float *logits, int T, int E, int k, int32_t *ids, float *w, int32_t *counts,
-                                 int32_t *offsets, int32_t *perm, int32_t *inv_perm, int *err, cudaStream_t s) {
-    if (!route_permute_fusable(T, E, k)) return cudaErrorInvalidValue;
+cudaError_t launch_route_permute(const float *logits, int T, int E, int k, int n_shared, int32_t *ids, float *w,
+                                 int32_t *counts, int32_t *offsets, int32_t *perm, int32_t *inv_perm, int *err,
+                                 cudaStream_t s) {
+    if (!route_permute_fusable(T, E + n_shared, k + n_shared)) return cudaErrorInvalidValue;
     const int per_lane = (E + 31) / 32;
-    if (per_lane <= 1) return launch_t<1>(logits, T, E, k, ids, w, counts, offsets, perm, inv_perm, err, s);
-    if (per_lane <= 2) return launch_t<2>(logits, T, E, k, ids, w, counts, offsets, perm, inv_perm, err, s);
-    if (per_lane <= 4) return launch_t<4>(logits, T, E, k, ids, w, counts, offsets, perm, inv_perm, err, s);
-    return launch_t<8>(logits, T, E, k, ids, w, counts, offsets, perm, inv_perm, err, s);
+    if (per_lane <= 1) return launch_t<1>(logits, T, E, k, n_shared, ids, w, counts, offsets, perm, inv_perm, err, s);
+    if (per_lane <= 2) return launch_t<2>(logits, T, E, k, n_shared, ids, w, counts, offsets, perm, inv_perm, err, s);
+    if (per_lane <= 4) return launch_t<4>(logits, T, E, k, n_shared, ids, w, counts, offsets, perm, inv_perm, err, s);
+    return launch_t<8>(logits, T, E, k, n_shared, ids, w, counts, offsets, perm, inv_perm, err, s);
 }
 
 }  // namespace moe

@@ -61,17 +61,20 @@ class MoeConfig:
     fmt: str = "bf16"          # "bf16" or "int4_g128"
     logit_extra: str = "none"  # "none", "bias0.5" or "zipf1.2"
     weight_std: float = 0.02
+    n_shared: int = 0          # shared experts: weight arrays hold E + n_shared experts
 
     def with_(self, **kw) -> "MoeConfig":
         return dataclasses.replace(self, **kw)
 
     @property
     def P(self) -> int:
-        return self.T * self.k
+        """(token, expert) pairs: k routed slots plus n_shared shared slots per token."""
+        return self.T * (self.k + self.n_shared)
 
     def describe(self) -> str:
+        shared = f" n_shared={self.n_shared}" if self.n_shared else ""
         return (f"{self.name}: T={self.T} H={self.H} I={self.I} E={self.E} "
-                f"top_k={self.k} fmt={self.fmt} logits+={self.logit_extra}")
+                f"top_k={self.k}{shared} fmt={self.fmt} logits+={self.logit_extra}")
 
 
 CONFIGS: Dict[str, MoeConfig] = {
@@ -155,13 +158,15 @@ def gen_inputs(cfg: MoeConfig, seed: int = 0, experts: Optional[Iterable[int]] =
     """All inputs of one layer call as CPU tensors.
 
     Weights are stacked over experts: w_gu [E,2I,H] (or packed [E,2I,H/2] with
-    scales [E,2I,H/128]) and w_d [E,H,I] (or [E,H,I/2] with [E,H,I/128]).
+    scales [E,2I,H/128]) and w_d [E,H,I] (or [E,H,I/2] with [E,H,I/128]); with
+    n_shared shared experts the arrays hold E + n_shared experts, the shared
+    ones last (expert e's weights always come from streams 16+2e, 17+2e).
     If `experts` is given, only those experts' weights are drawn and the rest
     are left zero (used to keep tests of large configs cheap).
     """
     hidden = gen_hidden(cfg, seed)
     logits = gen_logits(cfg, seed)
-    E, H, I = cfg.E, cfg.H, cfg.I
+    E, H, I = cfg.E + cfg.n_shared, cfg.H, cfg.I       # routed experts, then the shared ones
     if cfg.fmt == "bf16":
         shapes = {"w_gu": ((E, 2 * I, H), torch.bfloat16), "w_d": ((E, H, I), torch.bfloat16)}
     else:

@@ -42,11 +42,13 @@ def lib() -> ctypes.CDLL:
         L.oracle_finalize.argtypes = [vp, vp, vp, i32, i32, i32, vp]
         L.oracle_forward.argtypes = [i32, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                      vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.oracle_forward_shared.argtypes = [i32, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                            vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.oracle_forward_tokens.argtypes = [i32, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                             vp, i32, vp, vp, vp]
         L.oracle_set_num_threads.argtypes = [i32]
-        for f in ("oracle_route", "oracle_permute", "oracle_forward", "oracle_forward_tokens",
-                  "oracle_num_threads"):
+        for f in ("oracle_route", "oracle_permute", "oracle_forward", "oracle_forward_shared",
+                  "oracle_forward_tokens", "oracle_num_threads"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -187,12 +189,14 @@ def _weights(inputs: Dict[str, torch.Tensor], fmt: str):
     return f, gu, sg, d, sd
 
 
-def forward(inputs: Dict[str, torch.Tensor], k: int, fmt: str = "bf16") -> Dict[str, np.ndarray]:
+def forward(inputs: Dict[str, torch.Tensor], k: int, fmt: str = "bf16", n_shared: int = 0) -> Dict[str, np.ndarray]:
     """The whole layer with every intermediate.
 
     inputs: hidden [T,H] bf16, logits [T,E] fp32, w_gu, w_d (+ scales for int4),
-    as produced by moe_synth.gen_inputs. Returns numpy arrays: ids, w, counts,
-    offsets, perm, inv_perm (int32 / fp32) and act, y, out (bf16 bit patterns).
+    as produced by moe_synth.gen_inputs; with n_shared > 0 the weight arrays
+    hold E + n_shared experts, the last n_shared shared. Returns numpy arrays:
+    ids, w ([T, k + n_shared]), counts, offsets (over E + n_shared experts),
+    perm, inv_perm (int32 / fp32) and act, y, out (bf16 bit patterns).
     """
     f, gu, sg, d, sd = _weights(inputs, fmt)
     h = _np(inputs["hidden"], np.uint16)
@@ -200,17 +204,18 @@ def forward(inputs: Dict[str, torch.Tensor], k: int, fmt: str = "bf16") -> Dict[
     T, H = h.shape
     E = lg.shape[1]
     I = d.shape[2] if f == 0 else d.shape[2] * 2
-    P = T * k
+    K, Et = k + n_shared, E + n_shared
+    P = T * K
     r = {
-        "ids": np.zeros((T, k), np.int32), "w": np.zeros((T, k), np.float32),
-        "counts": np.zeros(E, np.int32), "offsets": np.zeros(E + 1, np.int32),
+        "ids": np.zeros((T, K), np.int32), "w": np.zeros((T, K), np.float32),
+        "counts": np.zeros(Et, np.int32), "offsets": np.zeros(Et + 1, np.int32),
         "perm": np.zeros(P, np.int32), "inv_perm": np.zeros(P, np.int32),
         "act": np.zeros((P, I), np.uint16), "y": np.zeros((P, H), np.uint16),
         "out": np.zeros((T, H), np.uint16),
     }
-    rc = lib().oracle_forward(f, _p(h), _p(lg), _p(gu), _p(sg), _p(d), _p(sd), T, H, I, E, k,
-                              *[_p(r[n]) for n in ("ids", "w", "counts", "offsets", "perm",
-                                                   "inv_perm", "act", "y", "out")])
+    rc = lib().oracle_forward_shared(f, _p(h), _p(lg), _p(gu), _p(sg), _p(d), _p(sd), T, H, I, E, k, n_shared,
+                                     *[_p(r[n]) for n in ("ids", "w", "counts", "offsets", "perm",
+                                                          "inv_perm", "act", "y", "out")])
     if rc:
         raise ValueError("oracle_forward: bad arguments")
     return r

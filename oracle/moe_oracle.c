@@ -302,6 +302,27 @@ void oracle_finalize(const uint16_t *y, const float *w, const int32_t *inv_perm,
  * weights [E,2I,H] and [E,H,I]; fmt 1: int4 [E,2I,H/2], [E,H,I/2] with bf16
  * scales [E,2I,H/128], [E,H,I/128].
  */
+/* Every permuted row r through its expert's FFN: row r of expert e's segment
+ * [offsets[e], offsets[e+1]) is token perm[r] / K through expert e; rows are
+ * independent. */
+static void ffn_rows(int fmt, const uint16_t *hidden, const void *w_gu, const uint16_t *w_gu_s, const void *w_d,
+                     const uint16_t *w_d_s, int H, int I, int K, int P, const int32_t *ids, const int32_t *perm,
+                     uint16_t *act, uint16_t *y) {
+    size_t gu_elems = fmt == 0 ? (size_t)2 * I * H : (size_t)2 * I * (H / 2);
+    size_t d_elems = fmt == 0 ? (size_t)H * I : (size_t)H * (I / 2);
+    size_t esz = fmt == 0 ? 2 : 1;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < P; ++r) {
+        int p = perm[r], t = p / K, e = ids[p];
+        const char *wgu_e = (const char *)w_gu + (size_t)e * gu_elems * esz;
+        const char *wd_e = (const char *)w_d + (size_t)e * d_elems * esz;
+        const uint16_t *sgu_e = fmt == 1 ? w_gu_s + (size_t)e * 2 * I * (H / 128) : NULL;
+        const uint16_t *sd_e = fmt == 1 ? w_d_s + (size_t)e * H * (I / 128) : NULL;
+        oracle_expert_ffn(fmt, hidden + (size_t)t * H, wgu_e, sgu_e, wd_e, sd_e, H, I,
+                          act + (size_t)r * I, y + (size_t)r * H);
+    }
+}
+
 int oracle_forward(int fmt, const uint16_t *hidden, const float *logits,
                    const void *w_gu, const uint16_t *w_gu_s, const void *w_d, const uint16_t *w_d_s,
                    int T, int H, int I, int E, int k,
@@ -312,22 +333,51 @@ int oracle_forward(int fmt, const uint16_t *hidden, const float *logits,
     int P = T * k;
     if (oracle_route(logits, T, E, k, ids, w)) return -1;
     if (oracle_permute(ids, P, E, counts, offsets, perm, inv_perm)) return -1;
-    size_t gu_elems = fmt == 0 ? (size_t)2 * I * H : (size_t)2 * I * (H / 2);
-    size_t d_elems = fmt == 0 ? (size_t)H * I : (size_t)H * (I / 2);
-    size_t esz = fmt == 0 ? 2 : 1;
-    /* every row r of expert e's segment [offsets[e], offsets[e+1]) is one
-       token through that expert's FFN; rows are independent */
-#pragma omp parallel for schedule(dynamic, 1)
-    for (int r = 0; r < P; ++r) {
-        int p = perm[r], t = p / k, e = ids[p];
-        const char *wgu_e = (const char *)w_gu + (size_t)e * gu_elems * esz;
-        const char *wd_e = (const char *)w_d + (size_t)e * d_elems * esz;
-        const uint16_t *sgu_e = fmt == 1 ? w_gu_s + (size_t)e * 2 * I * (H / 128) : NULL;
-        const uint16_t *sd_e = fmt == 1 ? w_d_s + (size_t)e * H * (I / 128) : NULL;
-        oracle_expert_ffn(fmt, hidden + (size_t)t * H, wgu_e, sgu_e, wd_e, sd_e, H, I,
-                          act + (size_t)r * I, y + (size_t)r * H);
-    }
+    ffn_rows(fmt, hidden, w_gu, w_gu_s, w_d, w_d_s, H, I, k, P, ids, perm, act, y);
     oracle_finalize(y, w, inv_perm, T, H, k, out);
+    return 0;
+}
+
+/* ---- shared experts -----------------------------------------------------------
+ * GC-MoE abstract (MoE layers with shared experts beside the routed ones):
+ *   out[t] = sum_{j<k} w_j FFN_{e_j}(x_t) + sum_{s<S} FFN_{E+s}(x_t)
+ * The S shared experts are experts E..E+S-1 of the weight arrays; every
+ * token takes them as extra slots k..k+S-1 with weight 1, after its routed
+ * slots, and the layer proceeds over E+S experts and k+S slots, so the
+ * finalize sum adds them after the routed slots (fma with weight 1 is an
+ * add rounded once). ids, w are [T, k+S]; counts, offsets are over E+S.
+ */
+int oracle_forward_shared(int fmt, const uint16_t *hidden, const float *logits,
+                          const void *w_gu, const uint16_t *w_gu_s, const void *w_d, const uint16_t *w_d_s,
+                          int T, int H, int I, int E, int k, int S,
+                          int32_t *ids, float *w, int32_t *counts, int32_t *offsets,
+                          int32_t *perm, int32_t *inv_perm, uint16_t *act, uint16_t *y, uint16_t *out) {
+    if (S < 0) return -1;
+    if (S == 0) return oracle_forward(fmt, hidden, logits, w_gu, w_gu_s, w_d, w_d_s, T, H, I, E, k,
+                                      ids, w, counts, offsets, perm, inv_perm, act, y, out);
+    if (T < 0 || H < 1 || I < 1 || k < 1 || k > E) return -1;
+    if (fmt == 1 && (H % 128 || I % 128)) return -1;
+    int K = k + S, P = T * K;
+    int32_t *ids_k = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T > 0 ? T : 1) * k);
+    float *w_k = (float *)malloc(sizeof(float) * (size_t)(T > 0 ? T : 1) * k);
+    if (!ids_k || !w_k) { free(ids_k); free(w_k); return -1; }
+    int rc = oracle_route(logits, T, E, k, ids_k, w_k);
+    for (int t = 0; rc == 0 && t < T; ++t) {
+        for (int j = 0; j < k; ++j) {
+            ids[(size_t)t * K + j] = ids_k[(size_t)t * k + j];
+            w[(size_t)t * K + j] = w_k[(size_t)t * k + j];
+        }
+        for (int s2 = 0; s2 < S; ++s2) {
+            ids[(size_t)t * K + k + s2] = E + s2;
+            w[(size_t)t * K + k + s2] = 1.0f;
+        }
+    }
+    free(ids_k);
+    free(w_k);
+    if (rc) return -1;
+    if (oracle_permute(ids, P, E + S, counts, offsets, perm, inv_perm)) return -1;
+    ffn_rows(fmt, hidden, w_gu, w_gu_s, w_d, w_d_s, H, I, K, P, ids, perm, act, y);
+    oracle_finalize(y, w, inv_perm, T, H, K, out);
     return 0;
 }
 

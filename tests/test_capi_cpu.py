@@ -173,7 +173,7 @@ C_CLIENT = r"""
 
 int main(void) {
     moe_shape_t s;
-    s.T = 64; s.H = 2048; s.I = 768; s.E = 128; s.top_k = 8; s.fmt = MOE_W_BF16;
+    s.T = 64; s.H = 2048; s.I = 768; s.E = 128; s.top_k = 8; s.fmt = MOE_W_BF16; s.n_shared = 0;
     size_t ws = moe_workspace_size(&s);
     moe_shape_t bad = s;
     bad.top_k = 129;

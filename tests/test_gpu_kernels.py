@@ -36,11 +36,11 @@ def dev(x, dtype=None):
     return t.contiguous().to(DEV)
 
 
-def run_route(logits, k):
+def run_route(logits, k, n_shared=0):
     T, E = logits.shape
-    ids = torch.empty(T, k, dtype=torch.int32, device=DEV)
-    w = torch.empty(T, k, dtype=torch.float32, device=DEV)
-    moe.moe_route(dev(logits), moe.Shape.of(T, 8, 8, E, k), ids, w)
+    ids = torch.empty(T, k + n_shared, dtype=torch.int32, device=DEV)
+    w = torch.empty(T, k + n_shared, dtype=torch.float32, device=DEV)
+    moe.moe_route(dev(logits), moe.Shape.of(T, 8, 8, E, k, n_shared=n_shared), ids, w)
     torch.cuda.synchronize()
     return ids.cpu().numpy(), w.cpu().numpy()
 
@@ -128,6 +128,18 @@ def test_route_orders_by_logit_where_probabilities_tie(E):
         assert np.array_equal(gi, oi), (row, gi, oi)
         assert gi[0].tolist() == expect
         assert np.allclose(gw, ow, rtol=2 ** -20, atol=0)
+
+
+@pytest.mark.parametrize("T,E,k,S", [(37, 64, 6, 2), (5, 8, 2, 1), (300, 256, 8, 4), (9, 30, 1, 31)])
+def test_route_appends_shared_expert_slots(T, E, k, S):
+    """Shared experts: slots k..k+S-1 of every token hold experts E..E+S-1 with
+    weight exactly 1; the routed slots are the routing without them."""
+    logits = torch.randn(T, E, generator=torch.Generator().manual_seed(T + S))
+    gi, gw = run_route(logits, k, S)
+    oi, ow = run_route(logits, k)
+    assert np.array_equal(gi[:, :k], oi) and np.array_equal(gw[:, :k], ow)
+    assert np.array_equal(gi[:, k:], np.tile(np.arange(E, E + S, dtype=np.int32), (T, 1)))
+    assert np.all(gw[:, k:] == 1.0)
 
 
 # ---------------------------------------------------------------- permute --

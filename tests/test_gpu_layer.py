@@ -32,7 +32,7 @@ class Layer:
         self.cfg = cfg
         self.inp = moe_synth.gen_inputs(cfg, seed=seed)
         self.d = {n: t.to(DEV) for n, t in self.inp.items()}
-        self.shape = moe.Shape.of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.fmt)
+        self.shape = moe.Shape.of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.fmt, n_shared=cfg.n_shared)
         self.ws = torch.empty(moe.moe_workspace_size(self.shape), dtype=torch.uint8, device=DEV)
 
     def forward(self):
@@ -45,9 +45,10 @@ class Layer:
     def steps(self):
         c, d = self.cfg, self.d
         P = c.P
+        K, Et = c.k + c.n_shared, c.E + c.n_shared        # slots per token, experts in the weights
         i32 = dict(dtype=torch.int32, device=DEV)
-        s = {"ids": torch.empty(c.T, c.k, **i32), "w": torch.empty(c.T, c.k, dtype=torch.float32, device=DEV),
-             "counts": torch.empty(c.E, **i32), "offsets": torch.empty(c.E + 1, **i32),
+        s = {"ids": torch.empty(c.T, K, **i32), "w": torch.empty(c.T, K, dtype=torch.float32, device=DEV),
+             "counts": torch.empty(Et, **i32), "offsets": torch.empty(Et + 1, **i32),
              "perm": torch.empty(P, **i32), "inv_perm": torch.empty(P, **i32),
              "hp": torch.empty(P, c.H, dtype=torch.bfloat16, device=DEV),
              "act": torch.empty(P, c.I, dtype=torch.bfloat16, device=DEV),
@@ -66,36 +67,43 @@ class Layer:
 
 
 WORKLOADS = ["tiny", "qwen3_decode", "qwen3_prefill", "skewed", "w4a16_decode"]
+# shared experts beside the routed ones (GC-MoE abstract): 2 shared experts
+# on a decode batch and on a prefill batch (the shared experts then take
+# every token: 2048-row segments)
+SHARED = [moe_synth.MoeConfig("shared_decode", T=64, H=2048, I=768, E=64, k=6, n_shared=2),
+          moe_synth.MoeConfig("shared_prefill", T=2048, H=2048, I=768, E=64, k=6, n_shared=2,
+                              logit_extra="bias0.5")]
 
 
-@pytest.mark.parametrize("name", WORKLOADS)
-def test_layer_matches_oracle_on_every_element(name):
+@pytest.mark.parametrize("cfg", [moe_synth.get_config(n) for n in WORKLOADS] + SHARED, ids=lambda c: c.name)
+def test_layer_matches_oracle_on_every_element(cfg):
     """Each workload at its full size, every element of every step:
     routing ids, counts, offsets, perm, inv_perm and the gather bit-exact;
     act on every row; y on every row, from the down GEMM fed the oracle's act
     so that it is checked alone; finalize of the GPU's own y bit-exact; and
     the layer output on every token within the layer's tolerance."""
-    cfg = moe_synth.get_config(name)
+    name = cfg.name
     L = Layer(cfg)
     out = L.forward()
     s = L.steps()
     # moe_forward and the step-by-step calls run the same arithmetic
     assert torch.equal(out.view(torch.int16), s["out"].view(torch.int16))
-    r = oracle.forward(L.inp, cfg.k, fmt=cfg.fmt)
+    r = oracle.forward(L.inp, cfg.k, fmt=cfg.fmt, n_shared=cfg.n_shared)
     for n in ("ids", "counts", "offsets", "perm", "inv_perm"):
         assert np.array_equal(s[n].cpu().numpy().reshape(-1), r[n].reshape(-1)), n
     if cfg.name == "skewed":
         assert (r["counts"] == 0).any()          # empty experts are exercised
-    assert np.array_equal(bf16_bits(s["hp"]), oracle.gather(L.inp["hidden"], r["perm"], cfg.k))
+    assert np.array_equal(bf16_bits(s["hp"]), oracle.gather(L.inp["hidden"], r["perm"], cfg.k + cfg.n_shared))
     gemm_rows_close(bf16_bits(s["act"]), r["act"], "act")
     y = torch.empty_like(s["y"])
     moe.moe_grouped_gemm_down(bits_to_bf16(r["act"]).to(DEV), s["offsets"], L.d["w_d"], L.d.get("w_d_scales"),
                               L.shape, y)
     torch.cuda.synchronize()
     gemm_rows_close(bf16_bits(y), r["y"], "y")
-    fin = oracle.finalize(bf16_bits(s["y"]), s["w"].cpu().numpy(), s["inv_perm"].cpu().numpy(), cfg.T, cfg.H, cfg.k)
+    K = cfg.k + cfg.n_shared
+    fin = oracle.finalize(bf16_bits(s["y"]), s["w"].cpu().numpy(), s["inv_perm"].cpu().numpy(), cfg.T, cfg.H, K)
     assert np.array_equal(bf16_bits(s["out"]), fin)
-    y_abs = weighted_abs_y(bf16_bits(s["y"]), s["w"].cpu().numpy(), s["inv_perm"].cpu().numpy(), cfg.T, cfg.H, cfg.k)
+    y_abs = weighted_abs_y(bf16_bits(s["y"]), s["w"].cpu().numpy(), s["inv_perm"].cpu().numpy(), cfg.T, cfg.H, K)
     layer_output_close(bf16_bits(out), r["out"], name, scale_abs_by_rms=cfg.fmt == "int4_g128", y_abs=y_abs)
 
 

@@ -267,30 +267,34 @@ def test_finalize_metamorphic_scaling():
 
 # ------------------------------------------------- FFN / the whole layer --
 
-def dense_brute_force(inp, k, fmt="bf16"):
+def dense_brute_force(inp, k, fmt="bf16", n_shared=0):
     """Every token through every expert in float64 (torch matmul), combined
     with weight 0 for unselected experts; routing from torch softmax/sort.
-    Rounding points as in the layer: fp32 accumulators, bf16 act and y."""
+    Shared experts (the last n_shared of the weight arrays) get weight 1
+    for every token. Rounding points as in the layer: fp32 accumulators,
+    bf16 act and y."""
     x = inp["hidden"].double()
     logits = inp["logits"]
     T, H = x.shape
     E = logits.shape[1]
+    Et = E + n_shared
     if fmt == "bf16":
         Wgu = inp["w_gu"].double()
         Wd = inp["w_d"].double()
     else:
         Wgu = torch.stack([bits_to_bf16(oracle.dequant_int4(inp["w_gu"][e], inp["w_gu_scales"][e]))
-                           for e in range(E)]).double()
+                           for e in range(Et)]).double()
         Wd = torch.stack([bits_to_bf16(oracle.dequant_int4(inp["w_d"][e], inp["w_d_scales"][e]))
-                          for e in range(E)]).double()
+                          for e in range(Et)]).double()
     I = Wd.shape[2]
     p = torch.softmax(logits.double(), 1)
     order = torch.sort(logits, dim=1, descending=True, stable=True).indices[:, :k]
     sel = torch.gather(p, 1, order)
     wsel = sel / sel.sum(1, keepdim=True)
-    wfull = torch.zeros(T, E, dtype=torch.float64).scatter_(1, order, wsel)
+    wfull = torch.zeros(T, Et, dtype=torch.float64).scatter_(1, order, wsel)
+    wfull[:, E:] = 1.0
     out = torch.zeros(T, H, dtype=torch.float64)
-    for e in range(E):
+    for e in range(Et):
         g = (x @ Wgu[e, :I].T).float().double()
         u = (x @ Wgu[e, I:].T).float().double()
         act = (g / (1 + torch.exp(-g)) * u).float().to(torch.bfloat16).double()
@@ -321,6 +325,41 @@ def test_forward_matches_dense_brute_force(cfg):
     # oracle: fp32 slot-ordered combine then bf16; brute force: float64 sum.
     assert torch.all(err <= ref.abs() * 2.0 ** -8 + 1e-6), float(err.max())
     assert np.array_equal(r["counts"].sum(), cfg.T * cfg.k)
+
+
+@pytest.mark.parametrize("cfg", [moe_synth.get_config("tiny", n_shared=1),
+                                 moe_synth.get_config("tiny", T=33, H=72, I=40, E=5, k=3, n_shared=2),
+                                 moe_synth.get_config("skewed", T=24, H=96, I=48, E=16, k=3, n_shared=1)],
+                         ids=lambda c: c.describe())
+def test_forward_with_shared_experts_matches_dense_brute_force(cfg):
+    # GC-MoE abstract: shared experts beside the routed ones, added with weight 1
+    inp = moe_synth.gen_inputs(cfg, seed=17)
+    r = oracle.forward(inp, cfg.k, n_shared=cfg.n_shared)
+    ref = dense_brute_force(inp, cfg.k, n_shared=cfg.n_shared)
+    out = bits_to_bf16(r["out"]).double()
+    assert torch.all((out - ref).abs() <= ref.abs() * 2.0 ** -8 + 1e-6), float((out - ref).abs().max())
+    # every token has its k routed slots, then experts E.. with weight exactly 1
+    assert np.array_equal(r["ids"][:, cfg.k:], np.tile(np.arange(cfg.E, cfg.E + cfg.n_shared), (cfg.T, 1)))
+    assert np.all(r["w"][:, cfg.k:] == 1.0)
+    assert np.array_equal(r["counts"][cfg.E:], np.full(cfg.n_shared, cfg.T))
+    # the routed slots are those of the layer without shared experts
+    r0 = oracle.forward(dict(inp, w_gu=inp["w_gu"][:cfg.E], w_d=inp["w_d"][:cfg.E]), cfg.k)
+    assert np.array_equal(r["ids"][:, :cfg.k], r0["ids"])
+    assert np.array_equal(r["w"][:, :cfg.k], r0["w"])
+
+
+def test_shared_expert_alone_when_routed_outputs_vanish():
+    # routed W_down = 0 makes every routed y exactly +0, so the combine is
+    # 0*w_0 (+) ... (+) 1*y_shared = y_shared: the output is the shared expert's
+    # own bf16 output, bit for bit, for every token
+    cfg = moe_synth.get_config("tiny", n_shared=1)
+    inp = moe_synth.gen_inputs(cfg, seed=18)
+    wd = inp["w_d"].clone()
+    wd[:cfg.E] = 0
+    r = oracle.forward(dict(inp, w_d=wd), cfg.k, n_shared=1)
+    for t in range(cfg.T):
+        _, y = oracle.expert_ffn(inp["hidden"][t], inp["w_gu"][cfg.E], wd[cfg.E], cfg.H, cfg.I)
+        assert np.array_equal(bits_to_bf16(r["out"][t]).float().numpy(), bits_to_bf16(y).float().numpy())
 
 
 def test_forward_int4_matches_dense_brute_force():
