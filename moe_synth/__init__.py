@@ -27,7 +27,9 @@ bf16 weights are N(0,0.02) fp32 draws rounded to bf16. int4 weights are
 uniform bytes (each nibble uniform on [0,15], read as two's complement
 [-8,7]; the low nibble holds the even K index) followed, from the same
 generator, by scales U(0.002,0.02) fp32 rounded to bf16, one per 128
-consecutive K elements of a row.
+consecutive K elements of a row. MXFP8 weights are E4M3 codes with a uniform
+sign, an exponent field uniform on 4..7 and a uniform mantissa, followed by
+E8M0 scale codes uniform on 120..122, one per 32 consecutive K elements.
 """
 
 from __future__ import annotations
@@ -58,7 +60,7 @@ class MoeConfig:
     I: int
     E: int
     k: int
-    fmt: str = "bf16"          # "bf16" or "int4_g128"
+    fmt: str = "bf16"          # "bf16", "int4_g128" or "mxfp8"
     logit_extra: str = "none"  # "none", "bias0.5" or "zipf1.2"
     weight_std: float = 0.02
     n_shared: int = 0          # shared experts: weight arrays hold E + n_shared experts
@@ -150,6 +152,19 @@ def gen_expert_weights(cfg: MoeConfig, e: int, seed: int = 0) -> Dict[str, torch
             out[name] = q
             out[name + "_scales"] = s.to(torch.bfloat16)
         return out
+    if cfg.fmt == "mxfp8":
+        if H % 32 or I % 32:
+            raise ValueError("mxfp8 needs H and I multiples of 32")
+        out = {}
+        for name, g, rows, K in (("w_gu", g_gu, 2 * I, H), ("w_d", g_d, H, I)):
+            # E4M3 codes: sign, exponent field uniform on 4..7, mantissa uniform;
+            # E8M0 scale codes uniform on 120..122 (2^-7 .. 2^-5)
+            sign = torch.randint(0, 2, (rows, K), generator=g, dtype=torch.int32) << 7
+            expo = torch.randint(4, 8, (rows, K), generator=g, dtype=torch.int32) << 3
+            mant = torch.randint(0, 8, (rows, K), generator=g, dtype=torch.int32)
+            out[name] = (sign | expo | mant).to(torch.uint8)
+            out[name + "_scales"] = torch.randint(120, 123, (rows, K // 32), generator=g, dtype=torch.int32).to(torch.uint8)
+        return out
     raise ValueError(f"unknown weight format {cfg.fmt!r}")
 
 
@@ -169,6 +184,13 @@ def gen_inputs(cfg: MoeConfig, seed: int = 0, experts: Optional[Iterable[int]] =
     E, H, I = cfg.E + cfg.n_shared, cfg.H, cfg.I       # routed experts, then the shared ones
     if cfg.fmt == "bf16":
         shapes = {"w_gu": ((E, 2 * I, H), torch.bfloat16), "w_d": ((E, H, I), torch.bfloat16)}
+    elif cfg.fmt == "mxfp8":
+        shapes = {
+            "w_gu": ((E, 2 * I, H), torch.uint8),
+            "w_gu_scales": ((E, 2 * I, H // 32), torch.uint8),
+            "w_d": ((E, H, I), torch.uint8),
+            "w_d_scales": ((E, H, I // 32), torch.uint8),
+        }
     else:
         shapes = {
             "w_gu": ((E, 2 * I, H // 2), torch.uint8),

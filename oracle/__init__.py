@@ -47,6 +47,8 @@ def lib() -> ctypes.CDLL:
         L.oracle_forward_tokens.argtypes = [i32, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
                                             vp, i32, vp, vp, vp]
         L.oracle_set_num_threads.argtypes = [i32]
+        L.oracle_mx_quantize.argtypes = [vp, i32, i32, vp, vp]
+        L.oracle_mx_dequantize.argtypes = [vp, vp, i32, i32, vp]
         for f in ("oracle_route", "oracle_permute", "oracle_forward", "oracle_forward_shared",
                   "oracle_forward_tokens", "oracle_num_threads"):
             getattr(L, f).restype = ctypes.c_int
@@ -95,7 +97,30 @@ def _fmt_code(fmt: str) -> int:
         return 0
     if fmt == "int4_g128":
         return 1
+    if fmt == "mxfp8":
+        return 2
     raise ValueError(fmt)
+
+
+def mx_quantize(x):
+    """MXFP8 quantisation (OCP MX v1.0) of bf16 rows [rows, K], K % 32 == 0:
+    (E4M3 codes [rows, K] uint8, E8M0 scale codes [rows, K/32] uint8)."""
+    xa = _np(x, np.uint16)
+    rows, K = xa.shape
+    q = np.zeros((rows, K), np.uint8)
+    sc = np.zeros((rows, K // 32), np.uint8)
+    lib().oracle_mx_quantize(_p(xa), rows, K, _p(q), _p(sc))
+    return q, sc
+
+
+def mx_dequantize(q, scales) -> np.ndarray:
+    """Decoded values (float64 [rows, K]) of MXFP8 codes and scales."""
+    qa = _np(q, np.uint8)
+    sa = _np(scales, np.uint8)
+    rows, K = qa.shape
+    out = np.zeros((rows, K), np.float64)
+    lib().oracle_mx_dequantize(_p(qa), _p(sa), rows, K, _p(out))
+    return out
 
 
 # ---- steps -----------------------------------------------------------------
@@ -149,8 +174,9 @@ def expert_ffn(x, w_gu, w_d, H: int, I: int, fmt: str = "bf16", w_gu_scales=None
     xa = _np(x, np.uint16).reshape(-1)
     gu = _np(w_gu, wdt)
     d = _np(w_d, wdt)
-    sg = None if f == 0 else _np(w_gu_scales, np.uint16)
-    sd = None if f == 0 else _np(w_d_scales, np.uint16)
+    sdt = np.uint16 if f == 1 else np.uint8
+    sg = None if f == 0 else _np(w_gu_scales, sdt)
+    sd = None if f == 0 else _np(w_d_scales, sdt)
     act = np.zeros(I, np.uint16)
     y = np.zeros(H, np.uint16)
     lib().oracle_expert_ffn(f, _p(xa), _p(gu), _p(sg), _p(d), _p(sd), H, I, _p(act), _p(y))
@@ -163,7 +189,7 @@ def expert_down(act, w_d, H: int, I: int, fmt: str = "bf16", w_d_scales=None):
     wdt = np.uint16 if f == 0 else np.uint8
     aa = _np(act, np.uint16).reshape(-1)
     d = _np(w_d, wdt)
-    sd = None if f == 0 else _np(w_d_scales, np.uint16)
+    sd = None if f == 0 else _np(w_d_scales, np.uint16 if f == 1 else np.uint8)
     y = np.zeros(H, np.uint16)
     lib().oracle_expert_down(f, _p(aa), _p(d), _p(sd), H, I, _p(y))
     return y
@@ -182,11 +208,17 @@ def finalize(y, w, inv_perm, T: int, H: int, k: int) -> np.ndarray:
 def _weights(inputs: Dict[str, torch.Tensor], fmt: str):
     f = _fmt_code(fmt)
     wdt = np.uint16 if f == 0 else np.uint8
+    sdt = np.uint16 if f == 1 else np.uint8
     gu = _np(inputs["w_gu"], wdt)
     d = _np(inputs["w_d"], wdt)
-    sg = None if f == 0 else _np(inputs["w_gu_scales"], np.uint16)
-    sd = None if f == 0 else _np(inputs["w_d_scales"], np.uint16)
+    sg = None if f == 0 else _np(inputs["w_gu_scales"], sdt)
+    sd = None if f == 0 else _np(inputs["w_d_scales"], sdt)
     return f, gu, sg, d, sd
+
+
+def _inner(d: np.ndarray, f: int) -> int:
+    """I from the down weights [E, H, I] (int4: packed, I/2 bytes per row)."""
+    return d.shape[2] * 2 if f == 1 else d.shape[2]
 
 
 def forward(inputs: Dict[str, torch.Tensor], k: int, fmt: str = "bf16", n_shared: int = 0) -> Dict[str, np.ndarray]:
@@ -203,7 +235,7 @@ def forward(inputs: Dict[str, torch.Tensor], k: int, fmt: str = "bf16", n_shared
     lg = _np(inputs["logits"], np.float32)
     T, H = h.shape
     E = lg.shape[1]
-    I = d.shape[2] if f == 0 else d.shape[2] * 2
+    I = _inner(d, f)
     K, Et = k + n_shared, E + n_shared
     P = T * K
     r = {
@@ -228,7 +260,7 @@ def forward_tokens(inputs: Dict[str, torch.Tensor], k: int, tokens: Sequence[int
     lg = _np(inputs["logits"], np.float32)
     T, H = h.shape
     E = lg.shape[1]
-    I = d.shape[2] if f == 0 else d.shape[2] * 2
+    I = _inner(d, f)
     tk = np.ascontiguousarray(np.asarray(tokens, np.int32))
     n = tk.size
     ids = np.zeros((n, k), np.int32)

@@ -95,6 +95,99 @@ static uint16_t dequant_one(const uint8_t *row_q, const uint16_t *row_s, int kid
     return f32_to_bf16(q * s);
 }
 
+/* ---- MXFP8 (OCP Microscaling Formats (MX) v1.0: E4M3 elements, one E8M0
+ * scale per 32 consecutive elements) ----------------------------------------
+ * E4M3 ("fn" variant): sign, 4-bit exponent with bias 7, 3-bit mantissa; no
+ * infinities; 0x7F / 0xFF are NaN; the largest finite magnitude is 448 =
+ * 1.75 * 2^8; subnormals are m * 2^-9. E8M0: 2^(code - 127), code 255 NaN.
+ */
+static double e4m3_value(uint8_t b) {
+    int sign = b >> 7, ex = (b >> 3) & 15, m = b & 7;
+    double v;
+    if (ex == 15 && m == 7) return NAN;
+    if (ex == 0) v = ldexp((double)m, -9);
+    else v = ldexp(1.0 + m / 8.0, ex - 7);
+    return sign ? -v : v;
+}
+
+static double e8m0_value(uint8_t c) { return c == 255 ? NAN : ldexp(1.0, (int)c - 127); }
+
+/* Round-to-nearest-even conversion to E4M3 with saturation to +-448 (every
+ * magnitude >= 448 gives 448; NaN gives 0x7F). */
+static uint8_t e4m3_rne_satfinite(float x) {
+    if (x != x) return 0x7F;
+    uint8_t sign = signbit(x) ? 0x80 : 0;
+    double a = fabs((double)x);
+    if (a >= 448.0) return sign | 0x7E;
+    if (a == 0.0) return sign;
+    int ex;
+    frexp(a, &ex);                       /* a = fr * 2^ex, fr in [0.5, 1) */
+    int E = ex - 1;                      /* a = (2 fr) * 2^E, 2 fr in [1, 2) */
+    double units;                        /* a in units of the spacing at a */
+    int field;
+    if (E < -6) {                        /* subnormal range: spacing 2^-9 */
+        units = ldexp(a, 9);
+        field = 0;
+    } else {
+        units = ldexp(a, 3 - E);         /* in [8, 16): 8 + mantissa */
+        field = E + 7;
+    }
+    double r = nearbyint(units);         /* round half to even (default mode) */
+    int q = (int)r;
+    if (field == 0) {
+        if (q >= 8) return sign | (1 << 3);          /* rounds up to 2^-6 */
+        return sign | (uint8_t)q;
+    }
+    if (q >= 16) { q = 8; ++field; }                 /* mantissa carry */
+    if (field > 15 || (field == 15 && q - 8 == 7)) return sign | 0x7E;
+    return sign | (uint8_t)((field << 3) | (q - 8));
+}
+
+/* MX quantisation of a row of K bf16 values (K a multiple of 32), OCP MX
+ * v1.0 §6.3: per block of 32, shared exponent e = floor(log2(max |x|)) - 8
+ * (8 = the largest E4M3 exponent), clamped to [-127, 127] (0 for an
+ * all-zero block gives code 0), then each element x / 2^e converted to E4M3
+ * with round-to-nearest-even and saturation. The division by 2^e is exact
+ * in fp32 for these operands, so it is done in fp32. */
+void oracle_mx_quantize(const uint16_t *x, int rows, int K, uint8_t *q, uint8_t *scales) {
+    no_ftz_daz();
+    for (int r = 0; r < rows; ++r) {
+        for (int b = 0; b < K / 32; ++b) {
+            const uint16_t *xb = x + (size_t)r * K + (size_t)b * 32;
+            float amax = 0.0f;
+            for (int i = 0; i < 32; ++i) {
+                float v = fabsf(bf16_to_f32(xb[i]));
+                if (v > amax) amax = v;
+            }
+            int e;
+            if (amax == 0.0f) {
+                e = -127;
+            } else {
+                int ex;
+                frexp((double)amax, &ex);
+                e = (ex - 1) - 8;
+                if (e < -127) e = -127;
+                if (e > 127) e = 127;
+            }
+            scales[(size_t)r * (K / 32) + b] = (uint8_t)(e + 127);
+            float inv = (float)ldexp(1.0, -e);
+            for (int i = 0; i < 32; ++i)
+                q[(size_t)r * K + (size_t)b * 32 + i] = e4m3_rne_satfinite(bf16_to_f32(xb[i]) * inv);
+        }
+    }
+}
+
+/* Decoded value of element k of an MX row: E4M3 element times its block's E8M0 scale. */
+static double mx_value(const uint8_t *row_q, const uint8_t *row_s, int k) {
+    return e4m3_value(row_q[k]) * e8m0_value(row_s[k / 32]);
+}
+
+void oracle_mx_dequantize(const uint8_t *q, const uint8_t *scales, int rows, int K, double *out) {
+    for (int r = 0; r < rows; ++r)
+        for (int k = 0; k < K; ++k)
+            out[(size_t)r * K + k] = mx_value(q + (size_t)r * K, scales + (size_t)r * (K / 32), k);
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();
@@ -223,42 +316,67 @@ void oracle_dequant_int4(const uint8_t *q, const uint16_t *scales, int rows, int
  * act[i] = bf16(silu(g_i) * u_i),  g = W_g x, u = W_u x  (R3), InfiniLM PR
  * #500 §2.2 (gate/up grouped GEMM, then SwiGLU);
  * y[h] = bf16(sum_i act[i] * W_d[h][i]) (R6), the down grouped GEMM.
- * Weights are bf16 (fmt 0) or int4 + scales (fmt 1, decoded per element).
+ * Weights are bf16 (fmt 0), int4 + bf16 scales (fmt 1, decoded per element)
+ * or MXFP8 (fmt 2: E4M3 + one E8M0 scale per 32 K, decoded per element; the
+ * activation row x, and act before the down projection, are MX-quantised
+ * first, since the block-scaled MMA takes both operands in MXFP8).
  */
-static float weight_at(int fmt, const void *w, const uint16_t *s, int K, int row, int col) {
-    if (fmt == 0) return bf16_to_f32(((const uint16_t *)w)[(size_t)row * K + col]);
-    return bf16_to_f32(dequant_one((const uint8_t *)w + (size_t)row * (K / 2), s + (size_t)row * (K / 128), col));
+static double weight_at(int fmt, const void *w, const void *s, int K, int row, int col) {
+    if (fmt == 0) return (double)bf16_to_f32(((const uint16_t *)w)[(size_t)row * K + col]);
+    if (fmt == 1)
+        return (double)bf16_to_f32(dequant_one((const uint8_t *)w + (size_t)row * (K / 2),
+                                               (const uint16_t *)s + (size_t)row * (K / 128), col));
+    return mx_value((const uint8_t *)w + (size_t)row * K, (const uint8_t *)s + (size_t)row * (K / 32), col);
 }
 
-void oracle_expert_gate_up(int fmt, const uint16_t *x, const void *w_gu, const uint16_t *w_gu_s, int H, int I,
+/* The activation row as the MMA sees it: bf16 values, or for fmt 2 the
+ * decoded MX quantisation of the row. xv has K entries. */
+static void activation_values(int fmt, const uint16_t *x, int K, double *xv) {
+    if (fmt != 2) {
+        for (int k = 0; k < K; ++k) xv[k] = (double)bf16_to_f32(x[k]);
+        return;
+    }
+    uint8_t *q = (uint8_t *)malloc((size_t)K);
+    uint8_t *sc = (uint8_t *)malloc((size_t)K / 32);
+    oracle_mx_quantize(x, 1, K, q, sc);
+    for (int k = 0; k < K; ++k) xv[k] = mx_value(q, sc, k);
+    free(q);
+    free(sc);
+}
+
+void oracle_expert_gate_up(int fmt, const uint16_t *x, const void *w_gu, const void *w_gu_s, int H, int I,
                            uint16_t *act) {
     no_ftz_daz();
+    double *xv = (double *)malloc(sizeof(double) * (size_t)H);
+    activation_values(fmt, x, H, xv);
     for (int i = 0; i < I; ++i) {
         double g = 0.0, u = 0.0;
         for (int h = 0; h < H; ++h) {
-            double xv = (double)bf16_to_f32(x[h]);
-            g += xv * (double)weight_at(fmt, w_gu, w_gu_s, H, i, h);
-            u += xv * (double)weight_at(fmt, w_gu, w_gu_s, H, I + i, h);
+            g += xv[h] * weight_at(fmt, w_gu, w_gu_s, H, i, h);
+            u += xv[h] * weight_at(fmt, w_gu, w_gu_s, H, I + i, h);
         }
         float gf = (float)g, uf = (float)u;
         double silu = (double)gf / (1.0 + exp(-(double)gf));
         act[i] = f32_to_bf16((float)(silu * (double)uf));
     }
+    free(xv);
 }
 
-void oracle_expert_down(int fmt, const uint16_t *act, const void *w_d, const uint16_t *w_d_s, int H, int I,
+void oracle_expert_down(int fmt, const uint16_t *act, const void *w_d, const void *w_d_s, int H, int I,
                         uint16_t *y) {
     no_ftz_daz();
+    double *av = (double *)malloc(sizeof(double) * (size_t)I);
+    activation_values(fmt, act, I, av);
     for (int h = 0; h < H; ++h) {
         double acc = 0.0;
-        for (int i = 0; i < I; ++i)
-            acc += (double)bf16_to_f32(act[i]) * (double)weight_at(fmt, w_d, w_d_s, I, h, i);
+        for (int i = 0; i < I; ++i) acc += av[i] * weight_at(fmt, w_d, w_d_s, I, h, i);
         y[h] = f32_to_bf16((float)acc);
     }
+    free(av);
 }
 
-void oracle_expert_ffn(int fmt, const uint16_t *x, const void *w_gu, const uint16_t *w_gu_s,
-                       const void *w_d, const uint16_t *w_d_s, int H, int I,
+void oracle_expert_ffn(int fmt, const uint16_t *x, const void *w_gu, const void *w_gu_s,
+                       const void *w_d, const void *w_d_s, int H, int I,
                        uint16_t *act, uint16_t *y) {
     oracle_expert_gate_up(fmt, x, w_gu, w_gu_s, H, I, act);
     oracle_expert_down(fmt, act, w_d, w_d_s, H, I, y);
@@ -305,31 +423,36 @@ void oracle_finalize(const uint16_t *y, const float *w, const int32_t *inv_perm,
 /* Every permuted row r through its expert's FFN: row r of expert e's segment
  * [offsets[e], offsets[e+1]) is token perm[r] / K through expert e; rows are
  * independent. */
-static void ffn_rows(int fmt, const uint16_t *hidden, const void *w_gu, const uint16_t *w_gu_s, const void *w_d,
-                     const uint16_t *w_d_s, int H, int I, int K, int P, const int32_t *ids, const int32_t *perm,
+/* Bytes of one expert's weight matrix [rows, K] and of its scales in format fmt. */
+static size_t weight_bytes(int fmt, int rows, int K) {
+    return fmt == 0 ? (size_t)rows * K * 2 : fmt == 1 ? (size_t)rows * (K / 2) : (size_t)rows * K;
+}
+static size_t scale_bytes(int fmt, int rows, int K) {
+    return fmt == 1 ? (size_t)rows * (K / 128) * 2 : fmt == 2 ? (size_t)rows * (K / 32) : 0;
+}
+
+static void ffn_rows(int fmt, const uint16_t *hidden, const void *w_gu, const void *w_gu_s, const void *w_d,
+                     const void *w_d_s, int H, int I, int K, int P, const int32_t *ids, const int32_t *perm,
                      uint16_t *act, uint16_t *y) {
-    size_t gu_elems = fmt == 0 ? (size_t)2 * I * H : (size_t)2 * I * (H / 2);
-    size_t d_elems = fmt == 0 ? (size_t)H * I : (size_t)H * (I / 2);
-    size_t esz = fmt == 0 ? 2 : 1;
 #pragma omp parallel for schedule(dynamic, 1)
     for (int r = 0; r < P; ++r) {
         int p = perm[r], t = p / K, e = ids[p];
-        const char *wgu_e = (const char *)w_gu + (size_t)e * gu_elems * esz;
-        const char *wd_e = (const char *)w_d + (size_t)e * d_elems * esz;
-        const uint16_t *sgu_e = fmt == 1 ? w_gu_s + (size_t)e * 2 * I * (H / 128) : NULL;
-        const uint16_t *sd_e = fmt == 1 ? w_d_s + (size_t)e * H * (I / 128) : NULL;
+        const char *wgu_e = (const char *)w_gu + (size_t)e * weight_bytes(fmt, 2 * I, H);
+        const char *wd_e = (const char *)w_d + (size_t)e * weight_bytes(fmt, H, I);
+        const char *sgu_e = fmt ? (const char *)w_gu_s + (size_t)e * scale_bytes(fmt, 2 * I, H) : NULL;
+        const char *sd_e = fmt ? (const char *)w_d_s + (size_t)e * scale_bytes(fmt, H, I) : NULL;
         oracle_expert_ffn(fmt, hidden + (size_t)t * H, wgu_e, sgu_e, wd_e, sd_e, H, I,
                           act + (size_t)r * I, y + (size_t)r * H);
     }
 }
 
 int oracle_forward(int fmt, const uint16_t *hidden, const float *logits,
-                   const void *w_gu, const uint16_t *w_gu_s, const void *w_d, const uint16_t *w_d_s,
+                   const void *w_gu, const void *w_gu_s, const void *w_d, const void *w_d_s,
                    int T, int H, int I, int E, int k,
                    int32_t *ids, float *w, int32_t *counts, int32_t *offsets,
                    int32_t *perm, int32_t *inv_perm, uint16_t *act, uint16_t *y, uint16_t *out) {
     if (T < 0 || H < 1 || I < 1 || k < 1 || k > E) return -1;
-    if (fmt == 1 && (H % 128 || I % 128)) return -1;
+    if ((fmt == 1 && (H % 128 || I % 128)) || (fmt == 2 && (H % 32 || I % 32)) || fmt < 0 || fmt > 2) return -1;
     int P = T * k;
     if (oracle_route(logits, T, E, k, ids, w)) return -1;
     if (oracle_permute(ids, P, E, counts, offsets, perm, inv_perm)) return -1;
@@ -348,7 +471,7 @@ int oracle_forward(int fmt, const uint16_t *hidden, const float *logits,
  * add rounded once). ids, w are [T, k+S]; counts, offsets are over E+S.
  */
 int oracle_forward_shared(int fmt, const uint16_t *hidden, const float *logits,
-                          const void *w_gu, const uint16_t *w_gu_s, const void *w_d, const uint16_t *w_d_s,
+                          const void *w_gu, const void *w_gu_s, const void *w_d, const void *w_d_s,
                           int T, int H, int I, int E, int k, int S,
                           int32_t *ids, float *w, int32_t *counts, int32_t *offsets,
                           int32_t *perm, int32_t *inv_perm, uint16_t *act, uint16_t *y, uint16_t *out) {
@@ -356,7 +479,7 @@ int oracle_forward_shared(int fmt, const uint16_t *hidden, const float *logits,
     if (S == 0) return oracle_forward(fmt, hidden, logits, w_gu, w_gu_s, w_d, w_d_s, T, H, I, E, k,
                                       ids, w, counts, offsets, perm, inv_perm, act, y, out);
     if (T < 0 || H < 1 || I < 1 || k < 1 || k > E) return -1;
-    if (fmt == 1 && (H % 128 || I % 128)) return -1;
+    if ((fmt == 1 && (H % 128 || I % 128)) || (fmt == 2 && (H % 32 || I % 32)) || fmt < 0 || fmt > 2) return -1;
     int K = k + S, P = T * K;
     int32_t *ids_k = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T > 0 ? T : 1) * k);
     float *w_k = (float *)malloc(sizeof(float) * (size_t)(T > 0 ? T : 1) * k);
@@ -388,19 +511,16 @@ int oracle_forward_shared(int fmt, const uint16_t *hidden, const float *logits,
  * [n_tokens, k].
  */
 int oracle_forward_tokens(int fmt, const uint16_t *hidden, const float *logits,
-                          const void *w_gu, const uint16_t *w_gu_s, const void *w_d, const uint16_t *w_d_s,
+                          const void *w_gu, const void *w_gu_s, const void *w_d, const void *w_d_s,
                           int T, int H, int I, int E, int k, const int32_t *tokens, int n_tokens,
                           int32_t *ids_out, float *w_out, uint16_t *out_rows) {
     if (T < 0 || H < 1 || I < 1 || k < 1 || k > E || n_tokens < 0) return -1;
-    if (fmt == 1 && (H % 128 || I % 128)) return -1;
+    if ((fmt == 1 && (H % 128 || I % 128)) || (fmt == 2 && (H % 32 || I % 32)) || fmt < 0 || fmt > 2) return -1;
     for (int n = 0; n < n_tokens; ++n) {
         if (tokens[n] < 0 || tokens[n] >= T) return -1;
         if (oracle_route(logits + (size_t)tokens[n] * E, 1, E, k, ids_out + (size_t)n * k, w_out + (size_t)n * k))
             return -1;
     }
-    size_t gu_elems = fmt == 0 ? (size_t)2 * I * H : (size_t)2 * I * (H / 2);
-    size_t d_elems = fmt == 0 ? (size_t)H * I : (size_t)H * (I / 2);
-    size_t esz = fmt == 0 ? 2 : 1;
     int npairs = n_tokens * k;
     uint16_t *ybuf = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(npairs > 0 ? npairs : 1) * H);
     if (!ybuf) return -1;
@@ -414,10 +534,10 @@ int oracle_forward_tokens(int fmt, const uint16_t *hidden, const float *logits,
             if (!abuf) continue;
             int n = q / k;
             int e = ids_out[q];
-            const char *wgu_e = (const char *)w_gu + (size_t)e * gu_elems * esz;
-            const char *wd_e = (const char *)w_d + (size_t)e * d_elems * esz;
-            const uint16_t *sgu_e = fmt == 1 ? w_gu_s + (size_t)e * 2 * I * (H / 128) : NULL;
-            const uint16_t *sd_e = fmt == 1 ? w_d_s + (size_t)e * H * (I / 128) : NULL;
+            const char *wgu_e = (const char *)w_gu + (size_t)e * weight_bytes(fmt, 2 * I, H);
+            const char *wd_e = (const char *)w_d + (size_t)e * weight_bytes(fmt, H, I);
+            const char *sgu_e = fmt ? (const char *)w_gu_s + (size_t)e * scale_bytes(fmt, 2 * I, H) : NULL;
+            const char *sd_e = fmt ? (const char *)w_d_s + (size_t)e * scale_bytes(fmt, H, I) : NULL;
             oracle_expert_ffn(fmt, hidden + (size_t)tokens[n] * H, wgu_e, sgu_e, wd_e, sd_e, H, I,
                               abuf, ybuf + (size_t)q * H);
         }

@@ -466,3 +466,70 @@ def test_expert_ffn_is_gate_up_then_down():
     inp = moe_synth.gen_inputs(cfg, seed=17)
     act, y = oracle.expert_ffn(inp["hidden"][3], inp["w_gu"][2], inp["w_d"][2], cfg.H, cfg.I)
     assert np.array_equal(oracle.expert_down(act, inp["w_d"][2], cfg.H, cfg.I), y)
+
+
+# ------------------------------------------------------------------ MXFP8 --
+# OCP Microscaling Formats (MX) v1.0: E4M3 elements, one E8M0 scale (2^(c-127))
+# per 32 consecutive elements; the block exponent is floor(log2 max|x|) - 8,
+# elements are x / 2^e rounded to nearest even and saturated to +-448.
+
+def _torch_e4m3_codes(v: torch.Tensor) -> np.ndarray:
+    return v.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_mx_quantize_matches_the_definition_and_torch_e4m3():
+    g = torch.Generator().manual_seed(31)
+    x = (torch.randn(64, 256, generator=g) * torch.exp(torch.randn(64, 1, generator=g) * 4)).to(torch.bfloat16)
+    x[0, :32] = 0                                   # all-zero block: code 0, zero elements
+    x[1, 5] = 2.0 ** -100                           # tiny next to the block's max
+    q, sc = oracle.mx_quantize(x)
+    xf = x.float()
+    for r in range(x.shape[0]):
+        for b in range(x.shape[1] // 32):
+            blk = xf[r, 32 * b:32 * b + 32]
+            amax = float(blk.abs().max())
+            e = -127 if amax == 0 else max(-127, min(127, math.frexp(amax)[1] - 1 - 8))
+            assert sc[r, b] == e + 127
+            scaled = blk * 2.0 ** -e                 # exact in fp32 here
+            assert float(scaled.abs().max()) < 512
+            ref = _torch_e4m3_codes(scaled.clamp(-448, 448))   # torch: round to nearest even
+            assert np.array_equal(q[r, 32 * b:32 * b + 32], ref), (r, b)
+
+
+def test_e4m3_codes_decode_as_torch_and_saturate():
+    # every finite code decodes to torch's float8_e4m3fn value (scale 2^0)
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], np.uint8)
+    q = codes.reshape(-1, 1).repeat(32, 1)[:, :32]
+    dec = oracle.mx_dequantize(q, np.full((q.shape[0], 1), 127, np.uint8))
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(dec[:, 0], ref)
+    # saturation: a block whose max scales into [448, 512) keeps 448
+    x = torch.zeros(1, 32, dtype=torch.bfloat16)
+    x[0, 0] = 255.0 * 2 ** -7                     # 1.9921875: e = -8, scaled 510
+    x[0, 1] = -1.0
+    q, sc = oracle.mx_quantize(x)
+    assert sc[0, 0] == 127 - 8 and q[0, 0] == 0x7E and q[0, 1] == 0xF8   # 448; -256 = -(1.0 * 2^8)
+    # subnormal elements: 2^-9 steps below 2^-6 (scale 2^0 block with max 256)
+    x = torch.zeros(1, 32, dtype=torch.bfloat16)
+    x[0, 0], x[0, 1], x[0, 2] = 256.0, 3 * 2.0 ** -9, 2.0 ** -10
+    q, sc = oracle.mx_quantize(x)
+    assert sc[0, 0] == 127 and q[0, 1] == 3 and q[0, 2] == 0      # 2^-10 ties to even 0
+
+
+def test_mxfp8_ffn_matches_dense_double_of_the_decoded_operands():
+    cfg = moe_synth.MoeConfig("mx_small", T=6, H=128, I=64, E=3, k=2, fmt="mxfp8")
+    inp = moe_synth.gen_inputs(cfg, seed=32)
+    for e in range(cfg.E):
+        wgu = oracle.mx_dequantize(inp["w_gu"][e], inp["w_gu_scales"][e])
+        wd = oracle.mx_dequantize(inp["w_d"][e], inp["w_d_scales"][e])
+        for t in range(cfg.T):
+            act, y = oracle.expert_ffn(inp["hidden"][t], inp["w_gu"][e], inp["w_d"][e], cfg.H, cfg.I, fmt="mxfp8",
+                                       w_gu_scales=inp["w_gu_scales"][e], w_d_scales=inp["w_d_scales"][e])
+            xq = oracle.mx_dequantize(*oracle.mx_quantize(inp["hidden"][t:t + 1]))[0]
+            g = np.float32(wgu[:cfg.I] @ xq).astype(np.float64)
+            u = np.float32(wgu[cfg.I:] @ xq).astype(np.float64)
+            a_ref = torch.from_numpy((g / (1 + np.exp(-g)) * u).astype(np.float32)).to(torch.bfloat16)
+            assert np.array_equal(act, bf16_bits(a_ref))
+            aq = oracle.mx_dequantize(*oracle.mx_quantize(a_ref[None]))[0]
+            y_ref = torch.from_numpy(np.float32(wd @ aq)).to(torch.bfloat16)
+            assert np.array_equal(y, bf16_bits(y_ref))
