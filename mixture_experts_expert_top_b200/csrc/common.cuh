@@ -141,6 +141,14 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 
+// The same arrive without release semantics: it does not wait for this
+// thread's earlier memory writes (for example its global stores) to become
+// visible. For hand-offs that order only completed tcgen05 loads (after
+// tcgen05.wait::ld and tcgen05.fence::before_thread_sync), not memory.
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // ---------------------------------------------------------------------- TMA --
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap *m) {
@@ -377,6 +385,52 @@ __host__ __device__ __forceinline__ uint32_t idesc_bf16_f32(int M, int N) {
            | (1u << 10)                                     // B format: bf16
            | (static_cast<uint32_t>(N >> 3) << 17)          // N >> 3
            | (static_cast<uint32_t>(M >> 4) << 24);         // M >> 4
+}
+
+// --- block-scaled MXFP8 (kind::mxf8f6f4, E4M3 operands, E8M0 scales) ----------
+
+// tcgen05.cp 32x128b.warpx4: a 32-row x 16-byte matrix in shared memory
+// (rows 16 bytes apart) into TMEM lanes 0-31 x 4 columns, replicated into
+// the other three lane quarters. Issued by one thread; ordered before later
+// tcgen05.mma of the same thread.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor of such a 32 x 16-byte matrix: K-major, no
+// swizzle, 8-row core matrices 128 bytes apart (stride byte offset), version
+// 1. The leading byte offset is not used by a 16-byte-wide matrix.
+__device__ __forceinline__ uint64_t sf_smem_desc(uint32_t smem_addr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(1u) << 16;
+    d |= static_cast<uint64_t>(128u >> 4) << 32;
+    d |= static_cast<uint64_t>(1u) << 46;
+    return d;
+}
+
+// Instruction descriptor of kind::mxf8f6f4 with block scaling: E4M3 A and B
+// (K-major), E8M0 scale factors, fp32 D, shape M x N; sf ids select the byte
+// of each 32-bit TMEM scale-factor word (the K block of 32 within 128).
+__host__ __device__ __forceinline__ uint32_t idesc_mxf8_e4m3(int M, int N, uint32_t a_sf_id, uint32_t b_sf_id) {
+    return (b_sf_id << 4)                                   // B scale factor id
+           | (0u << 7) | (0u << 10)                         // A, B format: E4M3
+           | (static_cast<uint32_t>(N >> 3) << 17)          // N >> 3
+           | (1u << 23)                                     // scale format: E8M0
+           | (static_cast<uint32_t>(M >> 4) << 24)          // M >> 4
+           | (a_sf_id << 29);                               // A scale factor id
+}
+
+// D[tmem] (+)= (A .* SFA)[smem] * (B .* SFB)[smem]^T, K = 32 per instruction,
+// scale factors read from TMEM (addresses carry the sf id in bits 30-31).
+__device__ __forceinline__ void umma_mxf8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %6, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%4], [%5], p;\n\t}\n" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(sfa_tmem), "r"(sfb_tmem), "r"(accumulate)
+        : "memory");
 }
 
 // ----------------------------------------------------------------- numerics --

@@ -254,11 +254,14 @@ grouped_gemm_wm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __gri
         int buf = 0;
         uint32_t bphase = 0;
         // TMEM accumulator buffer handed back to the MMA issuer once this
-        // warp's last tcgen05.ld of the tile has completed
+        // warp's last tcgen05.ld of the tile has completed (every lane has
+        // passed tcgen05.wait::ld). The arrive orders only those completed
+        // loads, so it is relaxed: a release would first wait for the warp's
+        // outstanding global stores.
         auto release = [&]() {
             tc_fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(buf ? tempty_leader1 : tempty_leader0);
+            if (lane == 0) mbar_arrive_cluster_relaxed(buf ? tempty_leader1 : tempty_leader0);
         };
         if (!SWIGLU) {
             // warps 2-5 store the first half of a tile's 32-column chunks,
