@@ -57,6 +57,8 @@ PROFILE_DIR = os.path.join(ROOT, "profiles")
 # the grouped-GEMM kernels' sources: a change to any of them invalidates stored counters
 KERNEL_SOURCES = ["mixture_experts_expert_top_b200/csrc/gemm_sm100.cu",
                   "mixture_experts_expert_top_b200/csrc/gemm_prefill_sm100.cu",
+                  "mixture_experts_expert_top_b200/csrc/gemm_wm_pair_sm100.cu",
+                  "mixture_experts_expert_top_b200/csrc/gemm_mxfp8_sm100.cu",
                   "mixture_experts_expert_top_b200/csrc/gemm_common.cuh",
                   "mixture_experts_expert_top_b200/csrc/common.cuh",
                   "mixture_experts_expert_top_b200/csrc/launch_util.cuh"]

@@ -23,7 +23,10 @@
  *  - Arguments are validated before anything is enqueued; a non-OK status
  *    means nothing was launched. T = 0 is valid and enqueues nothing.
  *  - Shape limits: 1 <= E <= 1024, 1 <= top_k <= min(E, 32), T*top_k < 2^31;
- *    H and I multiples of 8 (multiples of 128 for MOE_W_INT4_G128).
+ *    H and I multiples of 8 (multiples of 128 for MOE_W_INT4_G128 and
+ *    MOE_W_MXFP8).
+ *  - Weight scales are passed as untyped pointers: bf16 [rows, K/128] for
+ *    MOE_W_INT4_G128, E8M0 bytes [rows, K/32] for MOE_W_MXFP8, NULL for bf16.
  *    Device pointers must be 16-byte aligned (4-byte for logits/topk_w and
  *    the int32 arrays).
  *  - Pair ids: p = t*K + j for token t and slot j, with K = top_k +
@@ -66,7 +69,9 @@ typedef enum {
 
 typedef enum {
     MOE_W_BF16 = 0,        /* bf16 weights */
-    MOE_W_INT4_G128 = 1    /* W4A16: int4 weights, one bf16 scale per 128 K */
+    MOE_W_INT4_G128 = 1,   /* W4A16: int4 weights, one bf16 scale per 128 K */
+    MOE_W_MXFP8 = 2        /* MXFP8 (OCP MX v1.0): E4M3 weights, one E8M0 scale per 32 K;
+                              the activations are MX-quantised by the layer */
 } moe_weight_fmt_t;
 
 /* Layer shape. T tokens, hidden size H, expert intermediate size I, E routed
@@ -149,7 +154,7 @@ MOE_API moe_status_t moe_permute(const int32_t *topk_ids, const moe_shape_t *sha
  *   act     [T*top_k,I] bf16 out: act = bf16(silu(g) * u), g/u fp32 accumulated.
  * Experts with no rows cost no tiles. */
 MOE_API moe_status_t moe_grouped_gemm_swiglu(const moe_bf16_t *a, const int32_t *perm, const int32_t *offsets,
-                                     const void *w_gu, const moe_bf16_t *w_gu_scales,
+                                     const void *w_gu, const void *w_gu_scales,
                                      const moe_shape_t *shape, moe_bf16_t *act, moe_stream_t stream);
 
 /* Grouped GEMM down. InfiniLM PR #500 report §2.2 step 2 (third grouped GEMM).
@@ -158,7 +163,7 @@ MOE_API moe_status_t moe_grouped_gemm_swiglu(const moe_bf16_t *a, const int32_t 
  *           w_d_scales [E,H,I/128] bf16.
  *   y       [T*top_k,H] bf16 out: unscaled down projection, permuted row order. */
 MOE_API moe_status_t moe_grouped_gemm_down(const moe_bf16_t *act, const int32_t *offsets,
-                                   const void *w_d, const moe_bf16_t *w_d_scales,
+                                   const void *w_d, const void *w_d_scales,
                                    const moe_shape_t *shape, moe_bf16_t *y, moe_stream_t stream);
 
 /* Finalize / unpermute. FlashInfer PR #7196 analysis §1 (moe_finalize):
@@ -194,8 +199,8 @@ MOE_API int32_t moe_forward_gathers_in_gemm(const moe_shape_t *shape);
  *   call overwrites it, so calls that overlap on the GPU need distinct
  *   workspaces. */
 MOE_API moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits,
-                         const void *w_gu, const moe_bf16_t *w_gu_scales,
-                         const void *w_d, const moe_bf16_t *w_d_scales,
+                         const void *w_gu, const void *w_gu_scales,
+                         const void *w_d, const void *w_d_scales,
                          const moe_shape_t *shape, moe_bf16_t *out,
                          void *ws, size_t ws_bytes, moe_stream_t stream);
 
@@ -206,10 +211,43 @@ MOE_API moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits,
  *   ws: at least moe_forward_host_workspace_size(shape) bytes. */
 MOE_API size_t moe_forward_host_workspace_size(const moe_shape_t *shape);
 MOE_API moe_status_t moe_forward_host(const moe_bf16_t *hidden_host, const float *logits_host,
-                              const void *w_gu, const moe_bf16_t *w_gu_scales,
-                              const void *w_d, const moe_bf16_t *w_d_scales,
+                              const void *w_gu, const void *w_gu_scales,
+                              const void *w_d, const void *w_d_scales,
                               const moe_shape_t *shape, moe_bf16_t *out_host,
                               void *ws, size_t ws_bytes, moe_stream_t stream);
+
+/* MXFP8 (OCP Microscaling Formats (MX) v1.0; the GC-MoE abstract runs its
+ * expert GEMMs in FP8 / FP4). The block-scaled tensor-core MMA
+ * (tcgen05.mma kind::mxf8f6f4) takes both operands in MX form, so with
+ * MOE_W_MXFP8 weights the layer MX-quantises its activations: hidden before
+ * gate/up, and act (after its bf16 rounding) before down. moe_forward does
+ * all of it; these are the steps on their own.
+ *
+ * Quantisation of x [rows, K] bf16 (K % 32 == 0) into q [rows, K] E4M3 and
+ * scales [rows, K/32] E8M0: per block of 32 consecutive elements, e =
+ * floor(log2 max|x|) - 8 clamped to [-127, 127] (-127 for an all-zero
+ * block; the scale byte is e + 127), then q = E4M3(x / 2^e), rounded to
+ * nearest even and saturated to +-448. Bit-exact. */
+MOE_API moe_status_t moe_mx_quantize(const moe_bf16_t *x, int32_t rows, int32_t K, uint8_t *q, uint8_t *scales,
+                                     moe_stream_t stream);
+
+/* Gate/up + SwiGLU with MXFP8 weights (shape->fmt = MOE_W_MXFP8):
+ *   a_q, a_scales  perm == NULL: permuted rows [T*top_k, H] / [T*top_k, H/32];
+ *                  perm != NULL: hidden's quantisation [T, H] / [T, H/32], rows
+ *                  read through perm (TMA gather4)
+ *   w_gu [E,2I,H] E4M3, w_gu_scales [E,2I,H/32] E8M0
+ *   act_q [T*top_k, I] E4M3 and act_scales [T*top_k, I/32] out: the MX
+ *   quantisation of act = bf16(silu(g) * u), fp32 accumulation. */
+MOE_API moe_status_t moe_grouped_gemm_swiglu_mx(const uint8_t *a_q, const uint8_t *a_scales, const int32_t *perm,
+                                                const int32_t *offsets, const void *w_gu, const void *w_gu_scales,
+                                                const moe_shape_t *shape, uint8_t *act_q, uint8_t *act_scales,
+                                                moe_stream_t stream);
+
+/* Down with MXFP8 weights: act_q [T*top_k, I] E4M3 + act_scales [T*top_k,
+ * I/32], w_d [E,H,I] E4M3 + w_d_scales [E,H,I/32] -> y [T*top_k, H] bf16. */
+MOE_API moe_status_t moe_grouped_gemm_down_mx(const uint8_t *act_q, const uint8_t *act_scales,
+                                              const int32_t *offsets, const void *w_d, const void *w_d_scales,
+                                              const moe_shape_t *shape, moe_bf16_t *y, moe_stream_t stream);
 
 /* W4A16 weight decoding on its own (the step the int4 GEMMs run on chip
  * before their MMAs). FlashInfer PR #7196 analysis §2-§3.

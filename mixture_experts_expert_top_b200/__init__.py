@@ -26,6 +26,7 @@ __all__ = [
     "moe_finalize", "moe_forward", "moe_forward_host", "moe_dequant_int4",
     "moe_get_device_error", "moe_status_string", "moe_permute_noalloc", "moe_selftest_bounded_wait",
     "moe_forward_kernel_count", "moe_forward_gathers_in_gemm", "forward", "debug_bounds_library",
+    "moe_mx_quantize", "moe_grouped_gemm_swiglu_mx", "moe_grouped_gemm_down_mx", "FMT_MXFP8",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -33,6 +34,7 @@ library_path = os.path.join(HERE, "libmoe_b200.so")
 
 FMT_BF16 = 0
 FMT_INT4_G128 = 1
+FMT_MXFP8 = 2
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
           3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_FLAG"}
@@ -55,7 +57,7 @@ class Shape(ctypes.Structure):
     @classmethod
     def of(cls, T, H, I, E, top_k, fmt=FMT_BF16, n_shared=0) -> "Shape":
         if isinstance(fmt, str):
-            fmt = {"bf16": FMT_BF16, "int4_g128": FMT_INT4_G128}[fmt]
+            fmt = {"bf16": FMT_BF16, "int4_g128": FMT_INT4_G128, "mxfp8": FMT_MXFP8}[fmt]
         return cls(int(T), int(H), int(I), int(E), int(top_k), int(fmt), int(n_shared))
 
     @property
@@ -127,6 +129,9 @@ def _load(debug_bounds: bool) -> ctypes.CDLL:
         "moe_forward": ([vp, vp, vp, vp, vp, vp, sp, vp, vp, sz, vp], ctypes.c_int),
         "moe_forward_host": ([vp, vp, vp, vp, vp, vp, sp, vp, vp, sz, vp], ctypes.c_int),
         "moe_dequant_int4": ([vp, vp, i32, i32, vp, vp], ctypes.c_int),
+        "moe_mx_quantize": ([vp, i32, i32, vp, vp, vp], ctypes.c_int),
+        "moe_grouped_gemm_swiglu_mx": ([vp, vp, vp, vp, vp, vp, sp, vp, vp, vp], ctypes.c_int),
+        "moe_grouped_gemm_down_mx": ([vp, vp, vp, vp, vp, sp, vp, vp], ctypes.c_int),
         "moe_permute_noalloc": ([vp, sp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
         "moe_get_device_error": ([ctypes.POINTER(ctypes.c_int32)], ctypes.c_int),
         "moe_selftest_bounded_wait": ([ctypes.c_int64, vp], ctypes.c_int),
@@ -220,13 +225,13 @@ def moe_permute_noalloc(topk_ids, shape, counts, offsets, perm, inv_perm, hidden
 
 def moe_grouped_gemm_swiglu(a, perm, offsets, w_gu, w_gu_scales, shape, act, stream=None) -> None:
     _check(lib().moe_grouped_gemm_swiglu(_p(a, BF16), _p(perm, I32), _p(offsets, I32), _p(w_gu, BF16, U8),
-                                         _p(w_gu_scales, BF16), ctypes.byref(_shape(shape)), _p(act, BF16),
+                                         _p(w_gu_scales, BF16, U8), ctypes.byref(_shape(shape)), _p(act, BF16),
                                          _s(stream)),
            "moe_grouped_gemm_swiglu")
 
 
 def moe_grouped_gemm_down(act, offsets, w_d, w_d_scales, shape, y, stream=None) -> None:
-    _check(lib().moe_grouped_gemm_down(_p(act, BF16), _p(offsets, I32), _p(w_d, BF16, U8), _p(w_d_scales, BF16),
+    _check(lib().moe_grouped_gemm_down(_p(act, BF16), _p(offsets, I32), _p(w_d, BF16, U8), _p(w_d_scales, BF16, U8),
                                        ctypes.byref(_shape(shape)), _p(y, BF16), _s(stream)),
            "moe_grouped_gemm_down")
 
@@ -239,8 +244,8 @@ def moe_finalize(y, topk_w, inv_perm, shape, out, stream=None) -> None:
 
 def moe_forward(hidden, logits, w_gu, w_gu_scales, w_d, w_d_scales, shape, out, ws, stream=None) -> None:
     nbytes = ws.numel() * ws.element_size()
-    _check(lib().moe_forward(_p(hidden, BF16), _p(logits, F32), _p(w_gu, BF16, U8), _p(w_gu_scales, BF16),
-                             _p(w_d, BF16, U8), _p(w_d_scales, BF16), ctypes.byref(_shape(shape)), _p(out, BF16),
+    _check(lib().moe_forward(_p(hidden, BF16), _p(logits, F32), _p(w_gu, BF16, U8), _p(w_gu_scales, BF16, U8),
+                             _p(w_d, BF16, U8), _p(w_d_scales, BF16, U8), ctypes.byref(_shape(shape)), _p(out, BF16),
                              _p(ws), nbytes, _s(stream)),
            "moe_forward")
 
@@ -249,9 +254,28 @@ def moe_forward_host(hidden_host, logits_host, w_gu, w_gu_scales, w_d, w_d_scale
                      stream=None) -> None:
     nbytes = ws.numel() * ws.element_size()
     _check(lib().moe_forward_host(_p(hidden_host, BF16), _p(logits_host, F32), _p(w_gu, BF16, U8),
-                                  _p(w_gu_scales, BF16), _p(w_d, BF16, U8), _p(w_d_scales, BF16),
+                                  _p(w_gu_scales, BF16, U8), _p(w_d, BF16, U8), _p(w_d_scales, BF16, U8),
                                   ctypes.byref(_shape(shape)), _p(out_host, BF16), _p(ws), nbytes, _s(stream)),
            "moe_forward_host")
+
+
+def moe_mx_quantize(x, rows: int, K: int, q, scales, stream=None) -> None:
+    _check(lib().moe_mx_quantize(_p(x, BF16), int(rows), int(K), _p(q, U8), _p(scales, U8), _s(stream)),
+           "moe_mx_quantize")
+
+
+def moe_grouped_gemm_swiglu_mx(a_q, a_scales, perm, offsets, w_gu, w_gu_scales, shape, act_q, act_scales,
+                               stream=None) -> None:
+    _check(lib().moe_grouped_gemm_swiglu_mx(_p(a_q, U8), _p(a_scales, U8), _p(perm, I32), _p(offsets, I32),
+                                            _p(w_gu, U8), _p(w_gu_scales, U8), ctypes.byref(_shape(shape)),
+                                            _p(act_q, U8), _p(act_scales, U8), _s(stream)),
+           "moe_grouped_gemm_swiglu_mx")
+
+
+def moe_grouped_gemm_down_mx(act_q, act_scales, offsets, w_d, w_d_scales, shape, y, stream=None) -> None:
+    _check(lib().moe_grouped_gemm_down_mx(_p(act_q, U8), _p(act_scales, U8), _p(offsets, I32), _p(w_d, U8),
+                                          _p(w_d_scales, U8), ctypes.byref(_shape(shape)), _p(y, BF16), _s(stream)),
+           "moe_grouped_gemm_down_mx")
 
 
 def moe_dequant_int4(q, scales, rows: int, K: int, out, stream=None) -> None:
@@ -296,7 +320,10 @@ def forward(hidden: torch.Tensor, logits: torch.Tensor, w_gu: torch.Tensor, w_d:
     experts after the E routed ones."""
     T, H = hidden.shape
     E = logits.shape[1]
-    fmt = FMT_INT4_G128 if w_gu.dtype == torch.uint8 else FMT_BF16
+    if w_gu.dtype != torch.uint8:
+        fmt = FMT_BF16
+    else:
+        fmt = FMT_MXFP8 if (w_gu_scales is not None and w_gu_scales.dtype == torch.uint8) else FMT_INT4_G128
     I = w_d.shape[2] * (2 if fmt == FMT_INT4_G128 else 1)
     shape = Shape.of(T, H, I, E, top_k, fmt, n_shared=w_gu.shape[0] - E)
     if out is None:

@@ -45,11 +45,11 @@ moe_status_t check_shape(const moe_shape_t *s) {
     if (!s) return MOE_ERR_INVALID_ARG;
     if (s->T < 0 || s->H <= 0 || s->I <= 0 || s->E < 1 || s->top_k < 1 || s->top_k > s->E || s->n_shared < 0)
         return MOE_ERR_INVALID_ARG;
-    if (s->fmt != MOE_W_BF16 && s->fmt != MOE_W_INT4_G128) return MOE_ERR_INVALID_ARG;
+    if (s->fmt != MOE_W_BF16 && s->fmt != MOE_W_INT4_G128 && s->fmt != MOE_W_MXFP8) return MOE_ERR_INVALID_ARG;
     if (static_cast<long long>(s->E) + s->n_shared > 1024 || static_cast<long long>(s->top_k) + s->n_shared > 32)
         return MOE_ERR_UNSUPPORTED;
     if (s->H % 8 || s->I % 8) return MOE_ERR_UNSUPPORTED;
-    if (s->fmt == MOE_W_INT4_G128 && (s->H % 128 || s->I % 128)) return MOE_ERR_UNSUPPORTED;
+    if (s->fmt != MOE_W_BF16 && (s->H % 128 || s->I % 128)) return MOE_ERR_UNSUPPORTED;
     if (static_cast<long long>(s->T) * slots(s) >= (1LL << 31)) return MOE_ERR_UNSUPPORTED;
     if (static_cast<long long>(experts(s)) * 2 * s->I >= (1LL << 31) ||
         static_cast<long long>(experts(s)) * s->H >= (1LL << 31))
@@ -64,6 +64,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // Byte offsets of moe_forward's intermediates inside the workspace.
 struct Layout {
     size_t ids, w, counts, offsets, perm, inv, scratch, hperm, act, y;
+    size_t hq, hs, aq, as;                 // MXFP8: hidden and act, E4M3 codes and E8M0 scales
     size_t hidden_in, logits_in, out_st;   // staging for moe_forward_host
     size_t total;
 };
@@ -86,8 +87,16 @@ Layout layout(const moe_shape_t *s, bool host) {
     L.inv = take(P * 4);
     L.scratch = take(moe::permute_scratch_bytes(static_cast<long long>(P), E));
     L.hperm = moe::gemm_gathers_in_kernel(static_cast<int>(P), E, s->fmt) ? o : take(P * s->H * 2);
-    L.act = take(P * s->I * 2);
+    const bool mx = s->fmt == MOE_W_MXFP8;
+    L.act = mx ? o : take(P * s->I * 2);
     L.y = take(P * s->H * 2);
+    L.hq = L.hs = L.aq = L.as = o;
+    if (mx) {
+        L.hq = take(static_cast<size_t>(s->T) * s->H);
+        L.hs = take(static_cast<size_t>(s->T) * s->H / 32);
+        L.aq = take(P * s->I);
+        L.as = take(P * s->I / 32);
+    }
     L.hidden_in = L.logits_in = L.out_st = 0;
     if (host) {
         L.hidden_in = take(static_cast<size_t>(s->T) * s->H * 2);
@@ -99,7 +108,7 @@ Layout layout(const moe_shape_t *s, bool host) {
 }
 
 moe::GemmArgs gemm_args(const moe_shape_t *s, const void *a, const int32_t *perm, const int32_t *offsets,
-                        const void *w, const moe_bf16_t *scales, bool swiglu, moe_bf16_t *out) {
+                        const void *w, const void *scales, bool swiglu, moe_bf16_t *out) {
     moe::GemmArgs g;
     g.a = a;
     g.perm = perm;
@@ -107,7 +116,7 @@ moe::GemmArgs gemm_args(const moe_shape_t *s, const void *a, const int32_t *perm
     g.top_k = slots(s);
     g.offsets = offsets;
     g.w = w;
-    g.w_scales = scales;
+    g.w_scales = s->fmt == MOE_W_INT4_G128 ? static_cast<const uint16_t *>(scales) : nullptr;
     g.P = s->T * slots(s);
     g.E = experts(s);
     g.K = swiglu ? s->H : s->I;
@@ -120,9 +129,9 @@ moe::GemmArgs gemm_args(const moe_shape_t *s, const void *a, const int32_t *perm
     return g;
 }
 
-moe_status_t check_weights(const moe_shape_t *s, const void *w, const moe_bf16_t *scales) {
+moe_status_t check_weights(const moe_shape_t *s, const void *w, const void *scales) {
     if (!w || !aligned(w, 16)) return MOE_ERR_INVALID_ARG;
-    if (s->fmt == MOE_W_INT4_G128) {
+    if (s->fmt != MOE_W_BF16) {
         if (!scales || !aligned(scales, 4)) return MOE_ERR_INVALID_ARG;
     } else if (scales) {
         return MOE_ERR_INVALID_ARG;
@@ -130,8 +139,22 @@ moe_status_t check_weights(const moe_shape_t *s, const void *w, const moe_bf16_t
     return MOE_OK;
 }
 
+// The MXFP8 GEMM arguments: token rows a_q (E4M3) with scales a_sf, weight
+// scales w_sf, gate/up output act_q / act_sf (E4M3 / E8M0) or down output y.
+moe::MxGemmArgs mx_args(const moe_shape_t *s, const uint8_t *a_q, const uint8_t *a_sf, const int32_t *perm,
+                        const int32_t *offsets, const void *w, const void *w_sf, bool swiglu, uint8_t *act_q,
+                        uint8_t *act_sf, moe_bf16_t *y) {
+    moe::MxGemmArgs m;
+    m.base = gemm_args(s, a_q, perm, offsets, w, nullptr, swiglu, y);
+    m.w_sf = static_cast<const uint8_t *>(w_sf);
+    m.x_sf = a_sf;
+    m.out_q = act_q;
+    m.out_sf = act_sf;
+    return m;
+}
+
 moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const void *w_gu,
-                            const moe_bf16_t *w_gu_scales, const void *w_d, const moe_bf16_t *w_d_scales,
+                            const void *w_gu_scales, const void *w_d, const void *w_d_scales,
                             const moe_shape_t *s, moe_bf16_t *out, uint8_t *ws, const Layout &L,
                             cudaStream_t st) {
     // routing: top_k of the E routed experts, then the shared slots; every
@@ -156,6 +179,19 @@ moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const
         if ((e = moe::launch_permute(ids, P, E, counts, offsets, perm, inv, ws + L.scratch, error_flag_ptr(), st)) !=
             cudaSuccess)
             return cuda_status(e);
+    }
+    if (s->fmt == MOE_W_MXFP8) {
+        // MXFP8: hidden quantised once per token; gate/up gathers its rows through
+        // perm and writes act quantised; down reads act's codes and scales
+        auto *hq = ws + L.hq, *hs = ws + L.hs, *aq = ws + L.aq, *as = ws + L.as;
+        if ((e = moe::launch_mx_quantize(hidden, T, H, hq, hs, st)) != cudaSuccess) return cuda_status(e);
+        e = moe::launch_grouped_gemm_mxfp8(mx_args(s, hq, hs, perm, offsets, w_gu, w_gu_scales, true, aq, as, nullptr),
+                                           st);
+        if (e != cudaSuccess) return cuda_status(e);
+        e = moe::launch_grouped_gemm_mxfp8(mx_args(s, aq, as, nullptr, offsets, w_d, w_d_scales, false, nullptr,
+                                                   nullptr, y), st);
+        if (e != cudaSuccess) return cuda_status(e);
+        return cuda_status(moe::launch_finalize(y, w, inv, T, H, k, out, error_flag_ptr(), st));
     }
     // Few rows per expert: the gate/up GEMM gathers the token rows itself (TMA
     // gather4 through perm). Many rows per expert: one gather kernel writes the
@@ -246,11 +282,12 @@ moe_status_t moe_permute(const int32_t *topk_ids, const moe_shape_t *shape, int3
 }
 
 moe_status_t moe_grouped_gemm_swiglu(const moe_bf16_t *a, const int32_t *perm, const int32_t *offsets,
-                                     const void *w_gu, const moe_bf16_t *w_gu_scales, const moe_shape_t *shape,
+                                     const void *w_gu, const void *w_gu_scales, const moe_shape_t *shape,
                                      moe_bf16_t *act, moe_stream_t stream) {
     const moe::NvtxRange nvtx("moe_grouped_gemm_swiglu");
     moe_status_t st = check_shape(shape);
     if (st != MOE_OK) return st;
+    if (shape->fmt == MOE_W_MXFP8) return MOE_ERR_UNSUPPORTED;     // moe_grouped_gemm_swiglu_mx
     if (shape->T == 0) return MOE_OK;
     if (!a || !offsets || !act || !aligned(a, 16) || !aligned(act, 16) || !aligned(offsets, 4))
         return MOE_ERR_INVALID_ARG;
@@ -261,11 +298,12 @@ moe_status_t moe_grouped_gemm_swiglu(const moe_bf16_t *a, const int32_t *perm, c
 }
 
 moe_status_t moe_grouped_gemm_down(const moe_bf16_t *act, const int32_t *offsets, const void *w_d,
-                                   const moe_bf16_t *w_d_scales, const moe_shape_t *shape, moe_bf16_t *y,
+                                   const void *w_d_scales, const moe_shape_t *shape, moe_bf16_t *y,
                                    moe_stream_t stream) {
     const moe::NvtxRange nvtx("moe_grouped_gemm_down");
     moe_status_t st = check_shape(shape);
     if (st != MOE_OK) return st;
+    if (shape->fmt == MOE_W_MXFP8) return MOE_ERR_UNSUPPORTED;     // moe_grouped_gemm_down_mx
     if (shape->T == 0) return MOE_OK;
     if (!act || !offsets || !y || !aligned(act, 16) || !aligned(y, 16) || !aligned(offsets, 4))
         return MOE_ERR_INVALID_ARG;
@@ -298,6 +336,7 @@ int32_t moe_forward_kernel_count(const moe_shape_t *shape) {
     else
         n += 1 + moe::permute_kernel_count(P, E);                     // route; permute in 1, 2 or 3 kernels
     if (!moe::gemm_gathers_in_kernel(static_cast<int>(P), E, shape->fmt)) n += 1;   // gather
+    if (shape->fmt == MOE_W_MXFP8) n += 1;                            // MX quantisation of hidden
     return n + 3;                                                     // gate/up, down, finalize
 }
 
@@ -307,7 +346,7 @@ int32_t moe_forward_gathers_in_gemm(const moe_shape_t *shape) {
 }
 
 moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits, const void *w_gu,
-                         const moe_bf16_t *w_gu_scales, const void *w_d, const moe_bf16_t *w_d_scales,
+                         const void *w_gu_scales, const void *w_d, const void *w_d_scales,
                          const moe_shape_t *shape, moe_bf16_t *out, void *ws, size_t ws_bytes,
                          moe_stream_t stream) {
     const moe::NvtxRange nvtx("moe_forward");
@@ -326,7 +365,7 @@ moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits, const vo
 }
 
 moe_status_t moe_forward_host(const moe_bf16_t *hidden_host, const float *logits_host, const void *w_gu,
-                              const moe_bf16_t *w_gu_scales, const void *w_d, const moe_bf16_t *w_d_scales,
+                              const void *w_gu_scales, const void *w_d, const void *w_d_scales,
                               const moe_shape_t *shape, moe_bf16_t *out_host, void *ws, size_t ws_bytes,
                               moe_stream_t stream) {
     const moe::NvtxRange nvtx("moe_forward_host");
@@ -354,6 +393,52 @@ moe_status_t moe_forward_host(const moe_bf16_t *hidden_host, const float *logits
     if (cudaMemcpyAsync(out_host, base + L.out_st, hb, cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     return cuda_status(cudaStreamSynchronize(s));
+}
+
+moe_status_t moe_mx_quantize(const moe_bf16_t *x, int32_t rows, int32_t K, uint8_t *q, uint8_t *scales,
+                             moe_stream_t stream) {
+    const moe::NvtxRange nvtx("moe_mx_quantize");
+    if (rows < 0 || K <= 0 || K % 32) return MOE_ERR_INVALID_ARG;
+    if (static_cast<long long>(rows) * K >= (1LL << 40)) return MOE_ERR_UNSUPPORTED;
+    if (rows == 0) return MOE_OK;
+    if (!x || !q || !scales || !aligned(x, 16) || !aligned(q, 8)) return MOE_ERR_INVALID_ARG;
+    return cuda_status(moe::launch_mx_quantize(x, rows, K, q, scales, static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_grouped_gemm_swiglu_mx(const uint8_t *a_q, const uint8_t *a_scales, const int32_t *perm,
+                                        const int32_t *offsets, const void *w_gu, const void *w_gu_scales,
+                                        const moe_shape_t *shape, uint8_t *act_q, uint8_t *act_scales,
+                                        moe_stream_t stream) {
+    const moe::NvtxRange nvtx("moe_grouped_gemm_swiglu_mx");
+    moe_status_t st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (shape->fmt != MOE_W_MXFP8) return MOE_ERR_INVALID_ARG;
+    if (shape->T == 0) return MOE_OK;
+    if (!a_q || !a_scales || !offsets || !act_q || !act_scales || !aligned(a_q, 16) || !aligned(a_scales, 4) ||
+        !aligned(act_q, 16) || !aligned(offsets, 4))
+        return MOE_ERR_INVALID_ARG;
+    if (perm && !aligned(perm, 4)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_weights(shape, w_gu, w_gu_scales)) != MOE_OK) return st;
+    return cuda_status(moe::launch_grouped_gemm_mxfp8(
+        mx_args(shape, a_q, a_scales, perm, offsets, w_gu, w_gu_scales, true, act_q, act_scales, nullptr),
+        static_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_grouped_gemm_down_mx(const uint8_t *act_q, const uint8_t *act_scales, const int32_t *offsets,
+                                      const void *w_d, const void *w_d_scales, const moe_shape_t *shape,
+                                      moe_bf16_t *y, moe_stream_t stream) {
+    const moe::NvtxRange nvtx("moe_grouped_gemm_down_mx");
+    moe_status_t st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (shape->fmt != MOE_W_MXFP8) return MOE_ERR_INVALID_ARG;
+    if (shape->T == 0) return MOE_OK;
+    if (!act_q || !act_scales || !offsets || !y || !aligned(act_q, 16) || !aligned(act_scales, 4) ||
+        !aligned(y, 16) || !aligned(offsets, 4))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_weights(shape, w_d, w_d_scales)) != MOE_OK) return st;
+    return cuda_status(moe::launch_grouped_gemm_mxfp8(
+        mx_args(shape, act_q, act_scales, nullptr, offsets, w_d, w_d_scales, false, nullptr, nullptr, y),
+        static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_dequant_int4(const uint8_t *q, const moe_bf16_t *scales, int32_t rows, int32_t K,

@@ -107,4 +107,17 @@ cudaError_t launch_grouped_gemm_wm_pair(const GemmArgs &g, cudaStream_t s);
 cudaError_t launch_dequant_int4(const uint8_t *q, const uint16_t *scales, int rows, int K, uint16_t *out,
                                 cudaStream_t s);
 
+// ---- gemm_mxfp8_sm100.cu: MXFP8 weights (E4M3 + one E8M0 scale per 32 K),
+// block-scaled tcgen05 MMA; the token operand is MX-quantised too.
+struct MxGemmArgs {
+    GemmArgs base;              // base.a: token rows as E4M3 bytes; base.out: y (down) as bf16
+    const uint8_t *w_sf;        // [E * w_rows, K/32] E8M0 weight scales
+    const uint8_t *x_sf;        // [rows of base.a, K/32] E8M0 token scales
+    uint8_t *out_q;             // gate/up: act E4M3 [P, I]
+    uint8_t *out_sf;            // gate/up: act E8M0 [P, I/32]
+};
+cudaError_t launch_grouped_gemm_mxfp8(const MxGemmArgs &g, cudaStream_t s);
+// bf16 rows [rows, K] -> E4M3 [rows, K] and E8M0 [rows, K/32] (K % 32 == 0).
+cudaError_t launch_mx_quantize(const uint16_t *x, int rows, int K, uint8_t *q, uint8_t *scales, cudaStream_t s);
+
 }  // namespace moe
