@@ -50,6 +50,9 @@ EXTRA = ["qwen3_decode", "skewed", "w4a16_decode"]
 # prefill-like layers against 2.25 PFLOP/s dense bf16
 TARGETS = {"qwen3_decode": ("hbm", 0.70), "w4a16_decode": ("hbm", 0.70),
            "qwen3_prefill": ("tensor", 0.60), "skewed": ("tensor", 0.60), "tiny": (None, None)}
+# measured beside the graded workloads (no target of their own): MXFP8
+# weights on the block-scaled MMA, and shared experts
+UNGRADED = ["mxfp8_decode", "shared_decode"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NORTH_STAR_HBM_GBS = 8000.0       # the roofline literals the layer's target is stated against
 NORTH_STAR_BF16_TFLOPS = 2250.0
@@ -94,7 +97,7 @@ def parse_args(argv=None):
 def extra_workloads(args):
     if args.set or args.extra == "none":
         return []
-    names = EXTRA if args.extra == "all" else [n for n in args.extra.split(",") if n]
+    names = EXTRA + UNGRADED if args.extra == "all" else [n for n in args.extra.split(",") if n]
     return [n for n in names if n != args.workload]
 
 
@@ -288,25 +291,36 @@ def free_port() -> int:
 
 # -------------------------------------------------------- workload accounting --
 
+def weight_row_bytes(fmt, K):
+    """Bytes of one weight row of K elements with its scales."""
+    if fmt == "bf16":
+        return 2 * K
+    if fmt == "int4_g128":
+        return K // 2 + (K // 128) * 2
+    return K + K // 32                          # mxfp8: E4M3 codes + E8M0 scales
+
+
 def work_per_step(cfg, counts):
     """Algorithmic bytes and FLOPs of each kernel for one step, from the real
-    per-expert counts (experts with no rows read no weights)."""
-    T, H, I, E, k = cfg.T, cfg.H, cfg.I, cfg.E, cfg.k
-    P = T * k
+    per-expert counts (experts with no rows read no weights; shared experts
+    count as experts, their slots as pairs)."""
+    T, H, I, k = cfg.T, cfg.H, cfg.I, cfg.k
+    S = getattr(cfg, "n_shared", 0)
+    E = cfg.E + S
+    P = T * (k + S)
     active = int(sum(1 for c in counts if c > 0))
-    if cfg.fmt == "bf16":
-        w_gu = active * 2 * I * H * 2
-        w_d = active * H * I * 2
-    else:
-        w_gu = active * 2 * I * (H // 2 + (H // 128) * 2)
-        w_d = active * H * (I // 2 + (I // 128) * 2)
+    w_gu = active * 2 * I * weight_row_bytes(cfg.fmt, H)
+    w_d = active * H * weight_row_bytes(cfg.fmt, I)
+    # token operand bytes per element: bf16, or MX codes + scales
+    xb = (lambda K: K + K // 32) if cfg.fmt == "mxfp8" else (lambda K: 2 * K)
     return {
         "active_experts": active,
         "weight_bytes": w_gu + w_d,
-        "gemm_swiglu": {"bytes": w_gu + P * H * 2 + P * I * 2 + (E + 1) * 4, "flops": 2 * P * 2 * I * H},
-        "gemm_down": {"bytes": w_d + P * I * 2 + P * H * 2 + (E + 1) * 4, "flops": 2 * P * H * I},
-        "route": {"bytes": T * E * 4 + P * 8, "flops": 0},
+        "gemm_swiglu": {"bytes": w_gu + P * xb(H) + P * xb(I) + (E + 1) * 4, "flops": 2 * P * 2 * I * H},
+        "gemm_down": {"bytes": w_d + P * xb(I) + P * H * 2 + (E + 1) * 4, "flops": 2 * P * H * I},
+        "route": {"bytes": T * cfg.E * 4 + P * 8, "flops": 0},
         "permute": {"bytes": P * 4 * 3 + (2 * E + 1) * 4 + T * H * 2 + P * H * 2, "flops": 0},
+        "quantize": {"bytes": T * H * 2 + T * xb(H), "flops": 0},
         "finalize": {"bytes": P * H * 2 + T * H * 2 + P * 8, "flops": 0},
         "layer_flops": 2 * P * 3 * H * I,
     }
@@ -315,7 +329,8 @@ def work_per_step(cfg, counts):
 def launches_per_step(cfg) -> int:
     """Kernels one moe_forward call enqueues for this workload (the library's own count)."""
     import mixture_experts_expert_top_b200 as moe
-    return moe.moe_forward_kernel_count(moe.Shape.of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.fmt))
+    return moe.moe_forward_kernel_count(moe.Shape.of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.fmt,
+                                                     n_shared=getattr(cfg, "n_shared", 0)))
 
 
 def get_workload(name, sets=()):
@@ -379,7 +394,8 @@ def measure(cfg, args, dev, world, rank, sampler, headline):
         inp["hidden"] = moe_synth.gen_hidden(cfg, seed=args.seed + rank)
         inp["logits"] = moe_synth.gen_logits(cfg, seed=args.seed + rank)
     d = {n: t.to(dev) for n, t in inp.items()}
-    shape = moe.Shape.of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.fmt)
+    S = cfg.n_shared
+    shape = moe.Shape.of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.fmt, n_shared=S)
     ws = torch.empty(moe.moe_workspace_size(shape), dtype=torch.uint8, device=dev)
     out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -444,11 +460,12 @@ def measure(cfg, args, dev, world, rank, sampler, headline):
 
     # ---- per-stage pass: one C-ABI call per stage, events between ------------
     P = cfg.P
+    Kslots, Et = cfg.k + S, cfg.E + S
     i32 = dict(dtype=torch.int32, device=dev)
-    ids = torch.empty(cfg.T, cfg.k, **i32)
-    wts = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device=dev)
-    counts = torch.empty(cfg.E, **i32)
-    offsets = torch.empty(cfg.E + 1, **i32)
+    ids = torch.empty(cfg.T, Kslots, **i32)
+    wts = torch.empty(cfg.T, Kslots, dtype=torch.float32, device=dev)
+    counts = torch.empty(Et, **i32)
+    offsets = torch.empty(Et + 1, **i32)
     perm = torch.empty(P, **i32)
     inv = torch.empty(P, **i32)
     # the same gate/up kernel as moe_forward: rows read through perm, or a gathered copy
@@ -457,17 +474,35 @@ def measure(cfg, args, dev, world, rank, sampler, headline):
     act = torch.empty(P, cfg.I, dtype=torch.bfloat16, device=dev)
     y = torch.empty(P, cfg.H, dtype=torch.bfloat16, device=dev)
     pws = torch.empty(max(1, moe.moe_permute_workspace_size(shape)), dtype=torch.uint8, device=dev)
-    stages = ["route", "permute", "gemm_swiglu", "gemm_down", "finalize"]
-    calls = [
-        lambda: moe.moe_route(d["logits"], shape, ids, wts, stream),
-        (lambda: moe.moe_permute(ids, shape, counts, offsets, perm, inv, None, None, pws, stream)) if in_gemm else
-        (lambda: moe.moe_permute(ids, shape, counts, offsets, perm, inv, d["hidden"], hp, pws, stream)),
-        (lambda: moe.moe_grouped_gemm_swiglu(d["hidden"], perm, offsets, d["w_gu"], scales[0], shape, act, stream))
-        if in_gemm else
-        (lambda: moe.moe_grouped_gemm_swiglu(hp, None, offsets, d["w_gu"], scales[0], shape, act, stream)),
-        lambda: moe.moe_grouped_gemm_down(act, offsets, d["w_d"], scales[1], shape, y, stream),
-        lambda: moe.moe_finalize(y, wts, inv, shape, out, stream),
-    ]
+    if cfg.fmt == "mxfp8":
+        # the MXFP8 layer: hidden quantised once per token, gate/up reads its
+        # rows through perm and writes act quantised, down reads act's codes
+        u8 = dict(dtype=torch.uint8, device=dev)
+        hq, hs = torch.empty(cfg.T, cfg.H, **u8), torch.empty(cfg.T, cfg.H // 32, **u8)
+        aq, as_ = torch.empty(P, cfg.I, **u8), torch.empty(P, cfg.I // 32, **u8)
+        stages = ["route", "permute", "quantize", "gemm_swiglu", "gemm_down", "finalize"]
+        calls = [
+            lambda: moe.moe_route(d["logits"], shape, ids, wts, stream),
+            lambda: moe.moe_permute(ids, shape, counts, offsets, perm, inv, None, None, pws, stream),
+            lambda: moe.moe_mx_quantize(d["hidden"], cfg.T, cfg.H, hq, hs, stream),
+            lambda: moe.moe_grouped_gemm_swiglu_mx(hq, hs, perm, offsets, d["w_gu"], scales[0], shape, aq, as_,
+                                                   stream),
+            lambda: moe.moe_grouped_gemm_down_mx(aq, as_, offsets, d["w_d"], scales[1], shape, y, stream),
+            lambda: moe.moe_finalize(y, wts, inv, shape, out, stream),
+        ]
+    else:
+        stages = ["route", "permute", "gemm_swiglu", "gemm_down", "finalize"]
+        calls = [
+            lambda: moe.moe_route(d["logits"], shape, ids, wts, stream),
+            (lambda: moe.moe_permute(ids, shape, counts, offsets, perm, inv, None, None, pws, stream)) if in_gemm else
+            (lambda: moe.moe_permute(ids, shape, counts, offsets, perm, inv, d["hidden"], hp, pws, stream)),
+            (lambda: moe.moe_grouped_gemm_swiglu(d["hidden"], perm, offsets, d["w_gu"], scales[0], shape, act,
+                                                 stream))
+            if in_gemm else
+            (lambda: moe.moe_grouped_gemm_swiglu(hp, None, offsets, d["w_gu"], scales[0], shape, act, stream)),
+            lambda: moe.moe_grouped_gemm_down(act, offsets, d["w_d"], scales[1], shape, y, stream),
+            lambda: moe.moe_finalize(y, wts, inv, shape, out, stream),
+        ]
     for _ in range(W):
         for c in calls:
             c()
@@ -519,15 +554,19 @@ def measure(cfg, args, dev, world, rank, sampler, headline):
     peaks, peak_src = read_peaks()
     dom = max(("gemm_swiglu", "gemm_down"), key=lambda s: stage_ms[s])
     wk = work[dom]
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    # an MXFP8 contraction's peak: the measured bf16 peak times the nominal
+    # fp8 / bf16 ratio of 2 (4.5 / 2.25 PFLOP/s dense)
+    fp8 = cfg.fmt == "mxfp8"
+    tensor_peak = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
+    ridge = tensor_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
     sec = stage_ms[dom] / 1e3
     if wk["flops"] / wk["bytes"] < ridge:
         roof = {"bound": "hbm", "achieved": wk["bytes"] / sec / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
         which = "hbm_gbs"
     else:
-        roof = {"bound": "tensor", "achieved": wk["flops"] / sec / 1e12, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s"}
-        which = "bf16_tflops (burst: the kernel is timed alone)"
+        roof = {"bound": "tensor", "achieved": wk["flops"] / sec / 1e12, "peak": tensor_peak, "unit": "TFLOP/s"}
+        which = ("bf16_tflops x 2 (fp8 / bf16 nominal ratio)" if fp8 else "bf16_tflops") + \
+            " (burst: the kernel is timed alone)"
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = profiled_traffic(dom, cfg.name)
     roof["kernel"] = dom

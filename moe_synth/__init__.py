@@ -15,6 +15,8 @@ for the W4A16 format):
   qwen3_prefill  T=8192, H=2048, I=768,  E=128, k=8   bf16, logits + N(0,0.5) per-expert bias
   skewed         T=4096, H=4096, I=1536, E=64,  k=6   bf16, logits + 3 ln Zipf(1.2)
   w4a16_decode   T=256,  H=7168, I=2048, E=256, k=8   int4 weights, 1 bf16 scale / 128 K
+  mxfp8_decode   T=64,   H=2048, I=768,  E=128, k=8   MXFP8 weights (E4M3, 1 E8M0 scale / 32 K)
+  shared_decode  T=64,   H=2048, I=768,  E=64,  k=6   bf16, plus 2 shared experts
 
 Draw recipe. Every tensor has its own torch CPU generator, seeded from
 (seed, stream id), so a single expert's weights can be regenerated alone:
@@ -87,6 +89,10 @@ CONFIGS: Dict[str, MoeConfig] = {
         MoeConfig("qwen3_prefill", 8192, 2048, 768, 128, 8, logit_extra="bias0.5"),
         MoeConfig("skewed", 4096, 4096, 1536, 64, 6, logit_extra="zipf1.2"),
         MoeConfig("w4a16_decode", 256, 7168, 2048, 256, 8, fmt="int4_g128"),
+        # beyond the five workloads above: the Qwen3 decode shape with MXFP8
+        # weights, and a decode layer with two shared experts
+        MoeConfig("mxfp8_decode", 64, 2048, 768, 128, 8, fmt="mxfp8"),
+        MoeConfig("shared_decode", 64, 2048, 768, 64, 6, n_shared=2),
     ]
 }
 
