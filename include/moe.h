@@ -204,6 +204,23 @@ MOE_API moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits,
                          const moe_shape_t *shape, moe_bf16_t *out,
                          void *ws, size_t ws_bytes, moe_stream_t stream);
 
+/* The whole layer for a decode batch in ONE persistent kernel: routing,
+ * bucketing, gate/up + SwiGLU, down and finalize, with no kernel boundary
+ * between them (the GC-MoE abstract fuses the layer's steps into one graph;
+ * the steps and their arithmetic are those of moe_forward, which it equals
+ * bit for bit on these shapes). Every CTA routes and buckets the batch in
+ * shared memory; a down tile starts once its expert's gate/up tiles have
+ * finished (counters in the workspace, bounded waits) and finalize once
+ * every down tile has. The launch is cooperative (one CTA per SM, all
+ * resident).
+ *   bf16 weights, 1 <= T <= 64, top_k + n_shared <= 16, E + n_shared <= 256;
+ *   other shapes return MOE_ERR_UNSUPPORTED before anything is enqueued.
+ *   ws: at least moe_workspace_size(shape) bytes, 256-byte aligned; it also
+ *   holds the routing and the permutation of the call (as moe_forward's). */
+MOE_API moe_status_t moe_forward_fused(const moe_bf16_t *hidden, const float *logits, const void *w_gu,
+                                       const void *w_d, const moe_shape_t *shape, moe_bf16_t *out, void *ws,
+                                       size_t ws_bytes, moe_stream_t stream);
+
 /* moe_forward with hidden, logits and out in HOST memory (page-locked memory
  * gives asynchronous copies). Copies the inputs into the workspace, runs the
  * layer and copies out back, all on `stream`, then waits for the stream:

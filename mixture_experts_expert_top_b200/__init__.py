@@ -27,6 +27,7 @@ __all__ = [
     "moe_get_device_error", "moe_status_string", "moe_permute_noalloc", "moe_selftest_bounded_wait",
     "moe_forward_kernel_count", "moe_forward_gathers_in_gemm", "forward", "debug_bounds_library",
     "moe_mx_quantize", "moe_grouped_gemm_swiglu_mx", "moe_grouped_gemm_down_mx", "FMT_MXFP8",
+    "moe_forward_fused",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -130,6 +131,7 @@ def _load(debug_bounds: bool) -> ctypes.CDLL:
         "moe_forward_host": ([vp, vp, vp, vp, vp, vp, sp, vp, vp, sz, vp], ctypes.c_int),
         "moe_dequant_int4": ([vp, vp, i32, i32, vp, vp], ctypes.c_int),
         "moe_mx_quantize": ([vp, i32, i32, vp, vp, vp], ctypes.c_int),
+        "moe_forward_fused": ([vp, vp, vp, vp, sp, vp, vp, sz, vp], ctypes.c_int),
         "moe_grouped_gemm_swiglu_mx": ([vp, vp, vp, vp, vp, vp, sp, vp, vp, vp], ctypes.c_int),
         "moe_grouped_gemm_down_mx": ([vp, vp, vp, vp, vp, sp, vp, vp], ctypes.c_int),
         "moe_permute_noalloc": ([vp, sp, vp, vp, vp, vp, vp, vp, vp], ctypes.c_int),
@@ -257,6 +259,13 @@ def moe_forward_host(hidden_host, logits_host, w_gu, w_gu_scales, w_d, w_d_scale
                                   _p(w_gu_scales, BF16, U8), _p(w_d, BF16, U8), _p(w_d_scales, BF16, U8),
                                   ctypes.byref(_shape(shape)), _p(out_host, BF16), _p(ws), nbytes, _s(stream)),
            "moe_forward_host")
+
+
+def moe_forward_fused(hidden, logits, w_gu, w_d, shape, out, ws, stream=None) -> None:
+    nbytes = ws.numel() * ws.element_size()
+    _check(lib().moe_forward_fused(_p(hidden, BF16), _p(logits, F32), _p(w_gu, BF16), _p(w_d, BF16),
+                                   ctypes.byref(_shape(shape)), _p(out, BF16), _p(ws), nbytes, _s(stream)),
+           "moe_forward_fused")
 
 
 def moe_mx_quantize(x, rows: int, K: int, q, scales, stream=None) -> None:

@@ -65,6 +65,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Layout {
     size_t ids, w, counts, offsets, perm, inv, scratch, hperm, act, y;
     size_t hq, hs, aq, as;                 // MXFP8: hidden and act, E4M3 codes and E8M0 scales
+    size_t done;                           // moe_forward_fused: per-expert and finish counters
     size_t hidden_in, logits_in, out_st;   // staging for moe_forward_host
     size_t total;
 };
@@ -97,6 +98,7 @@ Layout layout(const moe_shape_t *s, bool host) {
         L.aq = take(P * s->I);
         L.as = take(P * s->I / 32);
     }
+    L.done = take(static_cast<size_t>(E + 1) * 4);
     L.hidden_in = L.logits_in = L.out_st = 0;
     if (host) {
         L.hidden_in = take(static_cast<size_t>(s->T) * s->H * 2);
@@ -362,6 +364,33 @@ moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits, const vo
     if (!aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
     return forward_device(hidden, logits, w_gu, w_gu_scales, w_d, w_d_scales, shape, out,
                           static_cast<uint8_t *>(ws), L, static_cast<cudaStream_t>(stream));
+}
+
+moe_status_t moe_forward_fused(const moe_bf16_t *hidden, const float *logits, const void *w_gu, const void *w_d,
+                               const moe_shape_t *shape, moe_bf16_t *out, void *ws, size_t ws_bytes,
+                               moe_stream_t stream) {
+    const moe::NvtxRange nvtx("moe_forward_fused");
+    moe_status_t st = check_shape(shape);
+    if (st != MOE_OK) return st;
+    if (shape->T == 0) return MOE_OK;
+    if (!moe::fused_decode_supported(shape->T, shape->H, shape->I, shape->E, shape->top_k, shape->n_shared,
+                                     shape->fmt))
+        return MOE_ERR_UNSUPPORTED;
+    if (!hidden || !logits || !out || !aligned(hidden, 16) || !aligned(out, 16) || !aligned(logits, 4))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_weights(shape, w_gu, nullptr)) != MOE_OK) return st;
+    if ((st = check_weights(shape, w_d, nullptr)) != MOE_OK) return st;
+    const Layout L = layout(shape, false);
+    if (!ws || ws_bytes < L.total) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    if (!aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
+    auto *b = static_cast<uint8_t *>(ws);
+    return cuda_status(moe::launch_fused_decode(
+        logits, hidden, w_gu, w_d, shape->T, shape->H, shape->I, shape->E, shape->top_k, shape->n_shared,
+        reinterpret_cast<int32_t *>(b + L.ids), reinterpret_cast<float *>(b + L.w),
+        reinterpret_cast<int32_t *>(b + L.counts), reinterpret_cast<int32_t *>(b + L.offsets),
+        reinterpret_cast<int32_t *>(b + L.perm), reinterpret_cast<int32_t *>(b + L.inv),
+        reinterpret_cast<uint16_t *>(b + L.act), reinterpret_cast<uint16_t *>(b + L.y), out,
+        reinterpret_cast<unsigned int *>(b + L.done), error_flag_ptr(), static_cast<cudaStream_t>(stream)));
 }
 
 moe_status_t moe_forward_host(const moe_bf16_t *hidden_host, const float *logits_host, const void *w_gu,

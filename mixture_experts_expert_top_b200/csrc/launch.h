@@ -117,6 +117,14 @@ struct MxGemmArgs {
     uint8_t *out_sf;            // gate/up: act E8M0 [P, I/32]
 };
 cudaError_t launch_grouped_gemm_mxfp8(const MxGemmArgs &g, cudaStream_t s);
+// ---- fused_decode_sm100.cu: the whole bf16 layer for a decode batch in one
+// persistent cooperative kernel (T <= 64, k + S <= 16, E + S <= 256). done:
+// E + S + 1 counters of the workspace, zeroed by the launcher.
+bool fused_decode_supported(int T, int H, int I, int E, int k, int S, int fmt);
+cudaError_t launch_fused_decode(const float *logits, const uint16_t *hidden, const void *w_gu, const void *w_d,
+                                int T, int H, int I, int E, int k, int S, int32_t *ids, float *w, int32_t *counts,
+                                int32_t *offsets, int32_t *perm, int32_t *inv_perm, uint16_t *act, uint16_t *y,
+                                uint16_t *out, unsigned int *done, int *err, cudaStream_t s);
 // bf16 rows [rows, K] -> E4M3 [rows, K] and E8M0 [rows, K/32] (K % 32 == 0).
 cudaError_t launch_mx_quantize(const uint16_t *x, int rows, int K, uint8_t *q, uint8_t *scales, cudaStream_t s);
 
