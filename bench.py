@@ -57,8 +57,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NORTH_STAR_HBM_GBS = 8000.0       # the roofline literals the layer's target is stated against
 NORTH_STAR_BF16_TFLOPS = 2250.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
-# the grouped-GEMM kernels' sources: a change to any of them invalidates stored counters
+# the GEMM kernels' sources: a change to any of them invalidates stored counters
 KERNEL_SOURCES = ["mixture_experts_expert_top_b200/csrc/gemm_sm100.cu",
+                  "mixture_experts_expert_top_b200/csrc/fused_decode_sm100.cu",
+                  "mixture_experts_expert_top_b200/csrc/route_dev.cuh",
                   "mixture_experts_expert_top_b200/csrc/gemm_prefill_sm100.cu",
                   "mixture_experts_expert_top_b200/csrc/gemm_wm_pair_sm100.cu",
                   "mixture_experts_expert_top_b200/csrc/gemm_mxfp8_sm100.cu",
@@ -322,6 +324,9 @@ def work_per_step(cfg, counts):
         "permute": {"bytes": P * 4 * 3 + (2 * E + 1) * 4 + T * H * 2 + P * H * 2, "flops": 0},
         "quantize": {"bytes": T * H * 2 + T * xb(H), "flops": 0},
         "finalize": {"bytes": P * H * 2 + T * H * 2 + P * 8, "flops": 0},
+        # the persistent decode kernel: the bytes the layer must move (weights,
+        # hidden, logits, out); act and y stay on chip or in L2
+        "fused": {"bytes": w_gu + w_d + T * H * 2 + T * cfg.E * 4 + T * H * 2, "flops": 2 * P * 3 * H * I},
         "layer_flops": 2 * P * 3 * H * I,
     }
 
@@ -503,6 +508,12 @@ def measure(cfg, args, dev, world, rank, sampler, headline):
             lambda: moe.moe_grouped_gemm_down(act, offsets, d["w_d"], scales[1], shape, y, stream),
             lambda: moe.moe_finalize(y, wts, inv, shape, out, stream),
         ]
+    fused = moe.moe_forward_is_fused(shape)
+    if fused:
+        # moe_forward runs the layer as one persistent kernel: time it too
+        stages.append("fused")
+        calls.append(lambda: moe.moe_forward_fused(d["hidden"], d["logits"], d["w_gu"], d["w_d"], shape, out, ws,
+                                                   stream))
     for _ in range(W):
         for c in calls:
             c()
@@ -552,7 +563,7 @@ def measure(cfg, args, dev, world, rank, sampler, headline):
     # each stage is timed on its own (a sub-millisecond launch between events),
     # so a tensor-bound kernel is held against the burst bf16 peak
     peaks, peak_src = read_peaks()
-    dom = max(("gemm_swiglu", "gemm_down"), key=lambda s: stage_ms[s])
+    dom = "fused" if fused else max(("gemm_swiglu", "gemm_down"), key=lambda s: stage_ms[s])
     wk = work[dom]
     # an MXFP8 contraction's peak: the measured bf16 peak times the nominal
     # fp8 / bf16 ratio of 2 (4.5 / 2.25 PFLOP/s dense)

@@ -180,6 +180,11 @@ MOE_API moe_status_t moe_finalize(const moe_bf16_t *y, const float *topk_w, cons
  * when the shape is invalid). Host-side only; launches nothing. */
 MOE_API int32_t moe_forward_kernel_count(const moe_shape_t *shape);
 
+/* 1 when moe_forward runs this shape as moe_forward_fused (one persistent
+ * kernel after a counter reset), 0 when it runs the step kernels, -1 for an
+ * invalid shape. Host-side only. */
+MOE_API int32_t moe_forward_is_fused(const moe_shape_t *shape);
+
 /* 1 when moe_forward's gate/up GEMM reads the token rows through perm itself
  * (no gathered copy is written), 0 when it gathers first, -1 for an invalid
  * shape. The same choice for moe_grouped_gemm_swiglu with a non-NULL perm
@@ -193,7 +198,10 @@ MOE_API int32_t moe_forward_gathers_in_gemm(const moe_shape_t *shape);
  * route, permute (with the gather when many tokens share each expert;
  * otherwise the gate/up GEMM gathers through perm itself), gate/up + SwiGLU,
  * down, finalize, enqueued on one stream with no host synchronisation. The
- * result equals the step entry points called in that order.
+ * result equals the step entry points called in that order. A decode batch
+ * with bf16 weights (the shapes moe_forward_fused takes, moe_forward_is_fused
+ * says which) runs as moe_forward_fused: the same result in one persistent
+ * kernel.
  *   hidden [T,H] bf16, logits [T,E] fp32, weights as above, out [T,H] bf16.
  *   ws: at least moe_workspace_size(shape) bytes, 256-byte aligned; the
  *   call overwrites it, so calls that overlap on the GPU need distinct
@@ -209,10 +217,11 @@ MOE_API moe_status_t moe_forward(const moe_bf16_t *hidden, const float *logits,
  * between them (the GC-MoE abstract fuses the layer's steps into one graph;
  * the steps and their arithmetic are those of moe_forward, which it equals
  * bit for bit on these shapes). Every CTA routes and buckets the batch in
- * shared memory; a down tile starts once its expert's gate/up tiles have
- * finished (counters in the workspace, bounded waits) and finalize once
- * every down tile has. The launch is cooperative (one CTA per SM, all
- * resident).
+ * shared memory and takes tiles from a counter in the workspace; a down
+ * tile loads act once its expert's gate/up tiles have finished and finalize
+ * starts once every down tile has (counters in the workspace, bounded
+ * waits). A one-warp kernel zeroes the counters first: two kernels in all,
+ * both with programmatic dependent launch.
  *   bf16 weights, 1 <= T <= 64, top_k + n_shared <= 16, E + n_shared <= 256;
  *   other shapes return MOE_ERR_UNSUPPORTED before anything is enqueued.
  *   ws: at least moe_workspace_size(shape) bytes, 256-byte aligned; it also

@@ -27,7 +27,7 @@ __all__ = [
     "moe_get_device_error", "moe_status_string", "moe_permute_noalloc", "moe_selftest_bounded_wait",
     "moe_forward_kernel_count", "moe_forward_gathers_in_gemm", "forward", "debug_bounds_library",
     "moe_mx_quantize", "moe_grouped_gemm_swiglu_mx", "moe_grouped_gemm_down_mx", "FMT_MXFP8",
-    "moe_forward_fused",
+    "moe_forward_fused", "moe_forward_is_fused",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -139,6 +139,7 @@ def _load(debug_bounds: bool) -> ctypes.CDLL:
         "moe_selftest_bounded_wait": ([ctypes.c_int64, vp], ctypes.c_int),
         "moe_forward_kernel_count": ([sp], ctypes.c_int32),
         "moe_forward_gathers_in_gemm": ([sp], ctypes.c_int32),
+        "moe_forward_is_fused": ([sp], ctypes.c_int32),
         "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
     }
     for name, (args, res) in sigs.items():
@@ -294,6 +295,13 @@ def moe_dequant_int4(q, scales, rows: int, K: int, out, stream=None) -> None:
 
 def moe_forward_kernel_count(shape) -> int:
     return int(lib().moe_forward_kernel_count(ctypes.byref(_shape(shape))))
+
+
+def moe_forward_is_fused(shape) -> bool:
+    v = int(lib().moe_forward_is_fused(ctypes.byref(_shape(shape))))
+    if v < 0:
+        raise MoeError(1, "moe_forward_is_fused: invalid shape")
+    return v == 1
 
 
 def moe_forward_gathers_in_gemm(shape) -> bool:

@@ -98,7 +98,7 @@ Layout layout(const moe_shape_t *s, bool host) {
         L.aq = take(P * s->I);
         L.as = take(P * s->I / 32);
     }
-    L.done = take(static_cast<size_t>(E + 1) * 4);
+    L.done = take(moe::fused_counter_words(s->E, s->n_shared) * 4);
     L.hidden_in = L.logits_in = L.out_st = 0;
     if (host) {
         L.hidden_in = take(static_cast<size_t>(s->T) * s->H * 2);
@@ -172,6 +172,12 @@ moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const
     auto *inv = reinterpret_cast<int32_t *>(ws + L.inv);
     auto *act = reinterpret_cast<uint16_t *>(ws + L.act);
     auto *y = reinterpret_cast<uint16_t *>(ws + L.y);
+    // a decode batch with bf16 weights: the whole layer in one persistent kernel
+    if (moe::fused_decode_supported(T, H, s->I, Er, kr, S, s->fmt))
+        return cuda_status(moe::launch_fused_decode(logits, hidden, w_gu, w_d, T, H, s->I, Er, kr, S, ids, w, counts,
+                                                    offsets, perm, inv, act, y, out,
+                                                    reinterpret_cast<unsigned int *>(ws + L.done), error_flag_ptr(),
+                                                    st));
     cudaError_t e;
     if (moe::route_permute_fusable(T, E, k)) {
         e = moe::launch_route_permute(logits, T, Er, kr, S, ids, w, counts, offsets, perm, inv, error_flag_ptr(), st);
@@ -332,6 +338,7 @@ int32_t moe_forward_kernel_count(const moe_shape_t *shape) {
     if (shape->T == 0) return 0;
     const int T = shape->T, k = slots(shape), E = experts(shape);
     const long long P = static_cast<long long>(T) * k;
+    if (moe_forward_is_fused(shape) == 1) return 2;                  // counter reset, the persistent kernel
     int32_t n = 0;
     if (moe::route_permute_fusable(T, E, k))
         n += 1;                                                       // route + permute in one CTA
@@ -340,6 +347,14 @@ int32_t moe_forward_kernel_count(const moe_shape_t *shape) {
     if (!moe::gemm_gathers_in_kernel(static_cast<int>(P), E, shape->fmt)) n += 1;   // gather
     if (shape->fmt == MOE_W_MXFP8) n += 1;                            // MX quantisation of hidden
     return n + 3;                                                     // gate/up, down, finalize
+}
+
+int32_t moe_forward_is_fused(const moe_shape_t *shape) {
+    if (check_shape(shape) != MOE_OK) return -1;
+    return moe::fused_decode_supported(shape->T, shape->H, shape->I, shape->E, shape->top_k, shape->n_shared,
+                                       shape->fmt)
+               ? 1
+               : 0;
 }
 
 int32_t moe_forward_gathers_in_gemm(const moe_shape_t *shape) {

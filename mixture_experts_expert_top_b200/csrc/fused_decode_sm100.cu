@@ -6,25 +6,38 @@
 // FlashInfer PR #7196 analysis §1 for finalize, §2 for the runtime-N tiles;
 // the GC-MoE abstract fuses the layer's steps into one graph). One launch, no
 // host synchronisation and no kernel boundary between the steps:
-//  - Every CTA routes and buckets the whole batch itself, in shared memory
-//    (a decode batch is at most 64 tokens: the logits are 32 KB from L2), so
-//    no CTA waits for another to learn the tile list. CTA 0 also writes the
-//    routing and permutation to the workspace.
-//  - Tiles: the gate/up tiles of every expert, then the down tiles, walked
-//    blockIdx.x + i * gridDim.x by the same warp-specialised pipeline as the
-//    weights-on-M kernel (warp 0 TMA, warp 1 MMA, warps 2-5 epilogue): gate/up
-//    reads the token rows through perm (gather4), down reads act rows.
+//  - Before it waits for the previous kernel, every CTA prefetches into L2 the
+//    first K-blocks of the gate/up weights of the CTA-th tile, so HBM streams
+//    weights while the batch is routed (weights are constant inputs).
+//  - CTA t < T routes token t (route_token, one warp) into the workspace and
+//    counts it (release); every CTA waits for the T tokens (acquire, bounded)
+//    and buckets the whole batch in shared memory from per-expert token
+//    masks (bit t of mask[e]: token t has a slot routed to e). A token has at
+//    most one slot per expert, so the rank of slot (t, j) inside expert e is
+//    the number of lower tokens in mask[e]: the stable order by slot id that
+//    the permute kernels produce, with no histogram passes.
+//  - Tiles: 256 weight rows (two M = 128 halves sharing the token operand) x
+//    all tokens of one expert (N = align16(count) <= 64). Gate/up tile of
+//    expert e and 128-feature block mb: half 0 = gate rows, half 1 = up rows;
+//    down tile: halves = output rows mb*256 .. +127 and +128 .. +255. Both
+//    kinds have the same shared-memory stage (32 KB of weights + 8 KB of
+//    token rows, K = 64) and the same TMEM accumulators.
+//  - The tile list (gate/up tiles of the non-empty experts, then their down
+//    tiles) is handed out dynamically: the producer warp takes the next tile
+//    number from a counter in global memory and passes it to the MMA and
+//    epilogue warps through a queue in shared memory. A CTA holds no tile it
+//    has not started, so no CTA waits on a CTA that is not running, and the
+//    CTAs finish together whatever the tiles' sizes.
 //  - A down tile of expert e reads act rows written by the gate/up tiles of
 //    e, which may run on other CTAs: their epilogues count finished tiles per
-//    expert in global memory (release), and the producer waits for the count
-//    (acquire, bounded) before it loads act. Finalize waits likewise for the
-//    count of finished down tiles, then every CTA combines a share of the
-//    tokens in the finalize kernel's order of operations.
-//  - The launch is cooperative, so every CTA is resident at once: a CTA
-//    waits only for tiles that CTAs already running will finish, and every
-//    CTA finishes its gate/up tiles before its down tiles. Every wait is
-//    bounded (a timeout raises the device flag and the CTA unwinds).
-#include "bucket_dev.cuh"
+//    expert in global memory (release). The producer loads the down tile's
+//    first weight stages, then waits for the count (acquire, bounded), then
+//    loads act. Finalize waits likewise for the count of finished down
+//    tiles; then every CTA combines a share of the tokens in the finalize
+//    kernel's order of operations.
+//  - A one-warp reset kernel zeroes the counters before each call; both are
+//    launched with programmatic dependent launch, so the reset and this
+//    kernel's set-up and prefetch overlap the previous kernel's tail.
 #include "gemm_common.cuh"
 #include "launch_util.cuh"
 #include "route_dev.cuh"
@@ -35,17 +48,19 @@ namespace {
 using namespace gemm;
 
 constexpr int kFThreads = 256;          // 0 TMA, 1 MMA, 2-5 epilogue; all 8 warps route, bucket and finalize
-constexpr int kFBN = 32;                // token rows per tile
+constexpr int kFWarps = kFThreads / 32;
+constexpr int kFBN = 64;                // token rows per tile: every token of one expert (T <= 64)
 constexpr int kFMaxT = 64;
 constexpr int kFMaxSlots = 16;
 constexpr int kFMaxP = kFMaxT * kFMaxSlots;
 constexpr int kFMaxE = 256;
 constexpr int kFStages = 5;
-constexpr int kFGuStage = 2 * kTileBytesA + kFBN * kBK * 2;        // 36 KB: gate, up, token rows (K = 64)
-constexpr int kFDnStage = 2 * (kTileBytesA + kFBN * kBK * 2);      // 40 KB: two K = 64 blocks of W_d and act
-constexpr int kFSlot = kFDnStage;
-constexpr int kFAccCols = 2 * kFBN;     // per buffer: g and u (down uses the first kFBN columns)
-constexpr int kFTmemCols = 128;
+constexpr int kFBBytes = kFBN * kBK * 2;                    // 8 KB of token rows per stage
+constexpr int kFSlot = 2 * kTileBytesA + kFBBytes;          // 40 KB: two weight halves + token rows (K = 64)
+constexpr int kFAccCols = 2 * kFBN;                         // per TMEM buffer: half 0, half 1
+constexpr int kFTmemCols = 2 * kFAccCols;
+constexpr int kFQueue = 8;                                  // tile numbers in flight between the roles
+constexpr int kFPrefetchKB = 6;                             // K-blocks prefetched to L2 before routing
 constexpr unsigned long long kFDepLimitNs = 2000000000ull;
 
 struct FusedArgs {
@@ -58,31 +73,24 @@ struct FusedArgs {
     uint16_t *out;                      // [T, H]
     unsigned int *gu_done;              // [E + S] finished gate/up tiles x 4 epilogue warps, per expert
     unsigned int *dn_done;              // [1] finished down tiles x 4 epilogue warps
+    unsigned int *next_tile;            // [1] tiles handed out
+    unsigned int *routed;               // [1] tokens routed
     int *err;
 };
 
 struct FusedSmem {
+    unsigned long long mask[kFMaxE];    // bit t: token t has a slot routed to expert e
+    int32_t ids[kFMaxP];
     int32_t perm[kFMaxP];
     int32_t inv[kFMaxP];
     float w[kFMaxP];
     int off[kFMaxE + 1];
-    int pre_gu[kFMaxE + 1];
-    int pre_dn[kFMaxE + 1];
+    int ne[kFMaxE];                     // non-empty experts, ascending
+    int n_ne;
+    int first_tile;
+    int warp_sums[kFWarps];
+    int tile_q[kFQueue];
 };
-
-// Tile prefix over experts from offsets already in shared memory (every
-// thread of the CTA calls it).
-__device__ void tile_prefix_smem(const int *off, int E, int MB, int *pre) {
-    if (threadIdx.x == 0) {
-        int run = 0;
-        pre[0] = 0;
-        for (int e = 0; e < E; ++e) {
-            run += ((off[e + 1] - off[e] + kFBN - 1) / kFBN) * MB;
-            pre[e + 1] = run;
-        }
-    }
-    __syncthreads();
-}
 
 __device__ __forceinline__ unsigned int ld_acquire_u32(const unsigned int *p) {
     unsigned int v;
@@ -114,22 +122,71 @@ __device__ bool wait_count(const unsigned int *p, unsigned int target, volatile 
             return false;
         }
         __nanosleep(sleep_ns);
-        if (sleep_ns < 1024) sleep_ns <<= 1;
+        if (sleep_ns < 512) sleep_ns <<= 1;
     }
     return true;
 }
 
 struct FTile {
     bool gu;        // gate/up tile (else down)
-    TileInfo t;
+    bool two;       // a second 128-row half (always for gate/up)
+    int h0;         // down: first 128-row half of the 256-row block (1 for the upper half of a split tile)
+    int e, mb, row0, valid, n_mma;
 };
 
-__device__ __forceinline__ FTile fused_tile(int tile, int n_gu, const FusedSmem &fs, int E, int MB_gu, int MB_dn) {
+// Tile numbers: [0, n_gu) gate/up tiles, expert-major; then the down tiles,
+// expert-major, of which the last n_split (one per CTA) are split into their
+// two 128-row halves, so that the tiles handed out last are the shortest.
+struct TileCounts {
+    int n_gu, n_dn, n_split;
+    __device__ __forceinline__ int total() const { return n_gu + n_dn + n_split; }
+};
+
+__device__ __forceinline__ TileCounts tile_counts(const FusedSmem &fs, int MB_gu, int MB_dn) {
+    TileCounts c;
+    c.n_gu = fs.n_ne * MB_gu;
+    c.n_dn = fs.n_ne * MB_dn;
+    c.n_split = min(c.n_dn, static_cast<int>(gridDim.x));
+    return c;
+}
+
+__device__ __forceinline__ FTile fused_tile(int tile, const TileCounts &c, const FusedSmem &fs, int MB_gu,
+                                            int MB_dn, int H) {
     FTile f;
-    f.gu = tile < n_gu;
-    f.t = f.gu ? decode_tile(tile, fs.pre_gu, fs.off, E, MB_gu, kFBN)
-               : decode_tile(tile - n_gu, fs.pre_dn, fs.off, E, MB_dn, kFBN);
+    f.gu = tile < c.n_gu;
+    int local = f.gu ? tile : tile - c.n_gu;
+    f.h0 = 0;
+    bool split = false;
+    if (!f.gu && local >= c.n_dn - c.n_split) {
+        const int h = local - (c.n_dn - c.n_split);
+        local = c.n_dn - c.n_split + h / 2;
+        f.h0 = h & 1;
+        split = true;
+    }
+    const int MB = f.gu ? MB_gu : MB_dn;
+    f.e = fs.ne[local / MB];
+    f.mb = local % MB;
+    f.row0 = fs.off[f.e];
+    f.valid = fs.off[f.e + 1] - f.row0;
+    f.n_mma = (f.valid + 15) & ~15;
+    f.two = f.gu || (!split && f.mb * 2 * kBM + kBM < H);
     return f;
+}
+
+// Queue entry qs: waits until it is filled, reads the tile number and frees
+// the entry (one thread per consuming warp).
+__device__ __forceinline__ bool pop_tile(const FusedSmem &fs, uint64_t *q_full, uint64_t *q_empty, int qs,
+                                         uint32_t qph, volatile int *abort, int *err, int &tile) {
+    if (!mbar_wait(&q_full[qs], qph, abort, err, 256)) return false;
+    tile = reinterpret_cast<const volatile int *>(fs.tile_q)[qs];
+    mbar_arrive(&q_empty[qs]);
+    return true;
+}
+
+__global__ void __launch_bounds__(32) fused_reset_kernel(unsigned int *counters, int n) {
+    griddep_launch_dependents();
+    griddep_wait();                     // the previous call may still read its counters
+    for (int i = threadIdx.x; i < n; i += 32) counters[i] = 0u;
 }
 
 template <int PER_LANE>
@@ -145,7 +202,9 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap tmWgu, const __grid_cons
     uint64_t *empty_bar = full_bar + kFStages;
     uint64_t *tfull_bar = empty_bar + kFStages;
     uint64_t *tempty_bar = tfull_bar + 2;
-    uint64_t *drain_bar = tempty_bar + 2;
+    uint64_t *q_full = tempty_bar + 2;
+    uint64_t *q_empty = q_full + kFQueue;
+    uint64_t *drain_bar = q_empty + kFQueue;
     uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(drain_bar + 1);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
     FusedSmem &fs = *reinterpret_cast<FusedSmem *>(tmem_holder + 16);
@@ -153,8 +212,10 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap tmWgu, const __grid_cons
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int K = a.k + a.S, Et = a.E + a.S, P = a.T * K;
-    const int MB_gu = (a.I + kBM - 1) / kBM, MB_dn = (a.H + kBM - 1) / kBM;
+    const int MB_gu = (a.I + kBM - 1) / kBM, MB_dn = (a.H + 2 * kBM - 1) / (2 * kBM);
+    const int KB_gu = (a.H + kBK - 1) / kBK, KB_dn = (a.I + kBK - 1) / kBK;
 
+    // ---- set-up and L2 prefetch (reads nothing written by earlier kernels) ----
     if (threadIdx.x == 0) {
         for (int s = 0; s < kFStages; ++s) {
             mbar_init(&full_bar[s], 1);
@@ -163,6 +224,10 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap tmWgu, const __grid_cons
         for (int b = 0; b < 2; ++b) {
             mbar_init(&tfull_bar[b], 1);
             mbar_init(&tempty_bar[b], kEpiThreads);
+        }
+        for (int q = 0; q < kFQueue; ++q) {
+            mbar_init(&q_full[q], 1);
+            mbar_init(&q_empty[q], 1 + kEpiThreads / 32);      // the MMA thread and one lane per epilogue warp
         }
         mbar_init(drain_bar, 1);
         *abort_flag = 0;
@@ -173,51 +238,105 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap tmWgu, const __grid_cons
         prefetch_tmap(&tmWd);
         prefetch_tmap(&tmX);
         prefetch_tmap(&tmAct);
+        // the gate/up tile that this CTA's number names when no expert is
+        // empty: the first tiles handed out are these, in some order
+        const int e = blockIdx.x / MB_gu, mb = blockIdx.x % MB_gu;
+        if (e < Et) {
+            const int row = e * 2 * a.I + mb * kBM;
+            for (int kb = 0; kb < kFPrefetchKB && kb < KB_gu; ++kb) {
+                tma_prefetch_l2_2d(&tmWgu, kb * kBK, row);
+                tma_prefetch_l2_2d(&tmWgu, kb * kBK, row + a.I);
+            }
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_holder, kFTmemCols);
         tmem_relinquish();
     }
+    for (int e = threadIdx.x; e < kFMaxE; e += kFThreads) fs.mask[e] = 0ull;
+    griddep_wait();
+    // the first tile number: its round trip overlaps the routing
+    unsigned int first_tile = 0;
+    if (threadIdx.x == 0) first_tile = atomicAdd(a.next_tile, 1u);
+    __syncthreads();
 
-    // ---- routing and bucketing of the whole batch, in shared memory ----------
-    // (the ring is free until the tiles start: ids and the bucketing scratch live there)
-    int32_t *ids_s = reinterpret_cast<int32_t *>(ring);                   // [P]
-    int32_t *counts_s = ids_s + kFMaxP;                                   // [Et]
-    int *bucket_scratch = counts_s + kFMaxE;                              // [(8 + 2) * Et]
-    for (int t = warp; t < a.T; t += kFThreads / 32) {
+    // ---- routing: CTA t routes token t; every CTA reads the T tokens' slots ----
+    if (warp == 0 && static_cast<int>(blockIdx.x) < a.T) {
+        const int t = blockIdx.x;
         int id;
         float wt;
         route_token<PER_LANE>(a.logits + static_cast<size_t>(t) * a.E, a.E, a.k, id, wt);
         shared_slot(lane, a.k, a.E, id, wt);
         if (lane < K) {
-            ids_s[t * K + lane] = id;
-            fs.w[t * K + lane] = wt;
+            a.ids[t * K + lane] = id;
+            a.w[t * K + lane] = wt;
+        }
+        __syncwarp();
+        if (lane == 0) red_release_add_u32(a.routed, 1u);
+    }
+    if (threadIdx.x == 0) {
+        fs.first_tile = static_cast<int>(first_tile);
+        wait_count(a.routed, static_cast<unsigned int>(a.T), abort_flag, a.err);
+    }
+    __syncthreads();
+    for (int s = threadIdx.x; s < P; s += kFThreads) {
+        const int id = __ldcg(a.ids + s);
+        const int t = s / K;
+        fs.ids[s] = id;
+        fs.w[s] = __ldcg(a.w + s);
+        if (id >= 0 && id < Et) atomicOr(reinterpret_cast<unsigned int *>(&fs.mask[id]) + (t >> 5), 1u << (t & 31));
+        else raise_error(a.err, kErrBadExpertId);
+    }
+    __syncthreads();
+    // ---- bucketing: counts, offsets and the non-empty experts in one scan ------
+    {
+        const int e = threadIdx.x;                          // Et <= kFThreads
+        const int c = e < Et ? __popcll(fs.mask[e]) : 0;
+        const int packed = c | ((c > 0 ? 1 : 0) << 16);     // count (<= 1024) | non-empty flag
+        int x = packed;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) fs.warp_sums[warp] = x;
+        __syncthreads();
+        int before = 0;
+        for (int w = 0; w < warp; ++w) before += fs.warp_sums[w];
+        const int excl = before + x - packed;
+        if (e < Et) {
+            fs.off[e] = excl & 0xFFFF;
+            if (c > 0) fs.ne[excl >> 16] = e;
+        }
+        if (e == Et - 1) {
+            fs.off[Et] = (excl + packed) & 0xFFFF;
+            fs.n_ne = (excl + packed) >> 16;
         }
     }
     __syncthreads();
-    bucket_single_cta<kFThreads>(ids_s, P, Et, counts_s, fs.off, fs.perm, fs.inv, bucket_scratch, a.err);
+    for (int s = threadIdx.x; s < P; s += kFThreads) {
+        const int t = s / K, e = min(max(fs.ids[s], 0), Et - 1);
+        const int r = fs.off[e] + __popcll(fs.mask[e] & ((1ull << t) - 1ull));
+        fs.perm[r] = s;
+        fs.inv[s] = r;
+    }
     __syncthreads();
     if (blockIdx.x == 0) {
         for (int i = threadIdx.x; i < P; i += kFThreads) {
-            a.ids[i] = ids_s[i];
-            a.w[i] = fs.w[i];
             a.perm[i] = fs.perm[i];
             a.inv_perm[i] = fs.inv[i];
         }
         for (int e = threadIdx.x; e <= Et; e += kFThreads) {
             a.offsets[e] = fs.off[e];
-            if (e < Et) a.counts[e] = counts_s[e];
+            if (e < Et) a.counts[e] = fs.off[e + 1] - fs.off[e];
         }
     }
-    tile_prefix_smem(fs.off, Et, MB_gu, fs.pre_gu);
-    tile_prefix_smem(fs.off, Et, MB_dn, fs.pre_dn);
-    fence_proxy_async_smem();            // the ring's routing scratch is overwritten by TMA next
     tc_fence_before_sync();
     __syncthreads();
     tc_fence_after_sync();
     const uint32_t tmem_base = *tmem_holder;
-    const int n_gu = fs.pre_gu[Et], n_dn = fs.pre_dn[Et];
-    const int total_tiles = n_gu + n_dn;
+    const TileCounts tc = tile_counts(fs, MB_gu, MB_dn);
+    const int total_tiles = tc.total();
     // token row of permuted row r (rows past P read row 0; they are never stored)
     auto token_of = [&](int r) { return r < P ? fs.perm[r] / K : 0; };
 
@@ -225,110 +344,134 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap tmWgu, const __grid_cons
         // ================================ TMA producer ==========================
         const uint64_t pol_w = l2_policy_evict_first();
         const uint64_t pol_x = l2_policy_evict_last();
-        int stage = 0;
-        uint32_t phase = 0;
+        int stage = 0, qs = 0;
+        uint32_t phase = 0, qph = 0;
         bool ok = true;
-        for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-            const FTile ft = fused_tile(tile, n_gu, fs, Et, MB_gu, MB_dn);
-            const TileInfo &ti = ft.t;
-            const int nbox = ti.n_mma / kBoxN;
+        int tile = fs.first_tile;
+        while (ok) {
+            const bool last = tile >= total_tiles;
+            if (lane == 0) ok = mbar_wait(&q_empty[qs], qph ^ 1, abort_flag, a.err, 256);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            if (lane == 0) {
+                reinterpret_cast<volatile int *>(fs.tile_q)[qs] = last ? -1 : tile;
+                mbar_arrive(&q_full[qs]);
+            }
+            if (++qs == kFQueue) { qs = 0; qph ^= 1; }
+            if (last) break;
+            unsigned int next = 0;
+            if (lane == 0) next = atomicAdd(a.next_tile, 1u);
+            const FTile ft = fused_tile(tile, tc, fs, MB_gu, MB_dn, a.H);
+            const int nbox = ft.n_mma / kBoxN;
             if (ft.gu) {
-                const int a_row = ti.e * 2 * a.I + ti.mb * kBM;
+                const int row = ft.e * 2 * a.I + ft.mb * kBM;
                 const uint32_t tx = 2 * kTileBytesA + nbox * kBoxBytesB;
-                const bool gather_lane = 4 * lane < ti.n_mma;
+                const bool gather_lane = 4 * lane < ft.n_mma;
                 int tr[4] = {0, 0, 0, 0};
                 if (gather_lane) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) tr[j] = token_of(ti.row0 + 4 * lane + j);
+                    for (int j = 0; j < 4; ++j) tr[j] = token_of(ft.row0 + 4 * lane + j);
                 }
-                const int KB = (a.H + kBK - 1) / kBK;
-                for (int kb = 0; kb < KB; ++kb) {
+                for (int kb = 0; kb < KB_gu; ++kb) {
                     if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, a.err, 0);
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
                     uint8_t *st = ring + stage * kFSlot;
                     if (lane == 0) {
                         mbar_arrive_expect_tx(&full_bar[stage], tx);
-                        tma_load_2d(st, &tmWgu, &full_bar[stage], kb * kBK, a_row, pol_w);
-                        tma_load_2d(st + kTileBytesA, &tmWgu, &full_bar[stage], kb * kBK, a_row + a.I, pol_w);
+                        tma_load_2d(st, &tmWgu, &full_bar[stage], kb * kBK, row, pol_w);
+                        tma_load_2d(st + kTileBytesA, &tmWgu, &full_bar[stage], kb * kBK, row + a.I, pol_w);
                     }
                     __syncwarp();
                     if (gather_lane)
-                        tma_gather4(st + 2 * kTileBytesA + lane * 4 * kBK * 2, &tmX, &full_bar[stage], kb * kBK, tr[0],
-                                    tr[1], tr[2], tr[3], pol_x);
+                        tma_gather4(st + 2 * kTileBytesA + lane * 4 * kBK * 2, &tmX, &full_bar[stage], kb * kBK,
+                                    tr[0], tr[1], tr[2], tr[3], pol_x);
                     if (++stage == kFStages) { stage = 0; phase ^= 1; }
                 }
             } else {
-                // act rows of expert e: every gate/up tile of e has finished (4 epilogue warps each)
-                const int cnt = fs.off[ti.e + 1] - fs.off[ti.e];
-                const unsigned int need = 4u * MB_gu * ((cnt + kFBN - 1) / kFBN);
-                if (lane == 0) ok = wait_count(a.gu_done + ti.e, need, abort_flag, a.err);
-                ok = __shfl_sync(0xffffffffu, ok, 0);
-                if (!ok) break;
-                fence_proxy_async_global();              // act was written by other threads' generic stores
-                const int a_row = ti.e * a.H + ti.mb * kBM;
-                const uint32_t tx = 2 * (kTileBytesA + nbox * kBoxBytesB);
-                const int KB = (a.I + 2 * kBK - 1) / (2 * kBK);
-                for (int kb = 0; kb < KB; ++kb) {
-                    if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, a.err, 0);
-                    ok = __shfl_sync(0xffffffffu, ok, 0);
-                    if (!ok) break;
-                    uint8_t *st = ring + stage * kFSlot;
+                const int row = ft.e * a.H + ft.mb * 2 * kBM + ft.h0 * kBM;
+                const uint32_t tx = (ft.two ? 2 : 1) * kTileBytesA + nbox * kBoxBytesB;
+                // the weights of the first stages go out before the wait for act
+                const int pre = KB_dn < kFStages ? KB_dn : kFStages;
+                const int stage0 = stage;
+                for (int kb = 0; kb < pre && ok; ++kb) {
                     if (lane == 0) {
-                        mbar_arrive_expect_tx(&full_bar[stage], tx);
-                        for (int u = 0; u < 2; ++u) {
-                            uint8_t *su = st + u * (kTileBytesA + kFBN * kBK * 2);
-                            const int x = (2 * kb + u) * kBK;
-                            tma_load_2d(su, &tmWd, &full_bar[stage], x, a_row, pol_w);
-                            for (int b = 0; b < nbox; ++b)
-                                tma_load_2d(su + kTileBytesA + b * kBoxBytesB, &tmAct, &full_bar[stage], x,
-                                            ti.row0 + b * kBoxN, pol_x);
+                        ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, a.err, 0);
+                        if (ok) {
+                            uint8_t *st = ring + stage * kFSlot;
+                            mbar_arrive_expect_tx(&full_bar[stage], tx);
+                            tma_load_2d(st, &tmWd, &full_bar[stage], kb * kBK, row, pol_w);
+                            if (ft.two)
+                                tma_load_2d(st + kTileBytesA, &tmWd, &full_bar[stage], kb * kBK, row + kBM, pol_w);
                         }
                     }
-                    __syncwarp();
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
+                    if (++stage == kFStages) { stage = 0; phase ^= 1; }
+                }
+                // act rows of expert e: every gate/up tile of e has finished (4 epilogue warps each)
+                if (ok && lane == 0) ok = wait_count(a.gu_done + ft.e, 4u * MB_gu, abort_flag, a.err);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                if (lane == 0) {
+                    fence_proxy_async_global();          // act was written by other threads' generic stores
+                    for (int kb = 0; kb < pre; ++kb) {
+                        const int s = (stage0 + kb) % kFStages;
+                        uint8_t *sb = ring + s * kFSlot + 2 * kTileBytesA;
+                        for (int b = 0; b < nbox; ++b)
+                            tma_load_2d(sb + b * kBoxBytesB, &tmAct, &full_bar[s], kb * kBK, ft.row0 + b * kBoxN,
+                                        pol_x);
+                    }
+                }
+                for (int kb = pre; kb < KB_dn && ok; ++kb) {
+                    if (lane == 0) {
+                        ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, a.err, 0);
+                        if (ok) {
+                            uint8_t *st = ring + stage * kFSlot;
+                            mbar_arrive_expect_tx(&full_bar[stage], tx);
+                            tma_load_2d(st, &tmWd, &full_bar[stage], kb * kBK, row, pol_w);
+                            if (ft.two)
+                                tma_load_2d(st + kTileBytesA, &tmWd, &full_bar[stage], kb * kBK, row + kBM, pol_w);
+                            for (int b = 0; b < nbox; ++b)
+                                tma_load_2d(st + 2 * kTileBytesA + b * kBoxBytesB, &tmAct, &full_bar[stage],
+                                            kb * kBK, ft.row0 + b * kBoxN, pol_x);
+                        }
+                    }
+                    ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (++stage == kFStages) { stage = 0; phase ^= 1; }
                 }
             }
+            tile = static_cast<int>(__shfl_sync(0xffffffffu, next, 0));
         }
     } else if (warp == 1) {
         // ================================ MMA issuer ============================
         if (lane == 0) {
-            int stage = 0;
-            uint32_t phase = 0;
-            int buf = 0;
-            uint32_t bphase = 0;
+            int stage = 0, qs = 0, buf = 0;
+            uint32_t phase = 0, qph = 0, bphase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
-                const FTile ft = fused_tile(tile, n_gu, fs, Et, MB_gu, MB_dn);
-                const uint32_t idesc = idesc_bf16_f32(kBM, ft.t.n_mma);
+            while (ok) {
+                int tile = -1;
+                ok = pop_tile(fs, q_full, q_empty, qs, qph, abort_flag, a.err, tile);
+                if (++qs == kFQueue) { qs = 0; qph ^= 1; }
+                if (!ok || tile < 0) break;
+                const FTile ft = fused_tile(tile, tc, fs, MB_gu, MB_dn, a.H);
+                const uint32_t idesc = idesc_bf16_f32(kBM, ft.n_mma);
                 ok = mbar_wait(&tempty_bar[buf], bphase ^ 1, abort_flag, a.err);
                 if (!ok) break;
                 tc_fence_after_sync();
                 const uint32_t d0 = tmem_base + buf * kFAccCols;
-                const int KB = ft.gu ? (a.H + kBK - 1) / kBK : (a.I + 2 * kBK - 1) / (2 * kBK);
+                const int KB = ft.gu ? KB_gu : KB_dn;
                 for (int kb = 0; kb < KB; ++kb) {
                     ok = mbar_wait(&full_bar[stage], phase, abort_flag, a.err, 0);
                     if (!ok) break;
                     tc_fence_after_sync();
                     const uint32_t st = smem_u32(ring + stage * kFSlot);
-                    if (ft.gu) {
-                        const uint64_t dg = sw128_kmajor_desc(st), du = sw128_kmajor_desc(st + kTileBytesA);
-                        const uint64_t db = sw128_kmajor_desc(st + 2 * kTileBytesA);
+                    const uint64_t da0 = sw128_kmajor_desc(st), da1 = sw128_kmajor_desc(st + kTileBytesA);
+                    const uint64_t db = sw128_kmajor_desc(st + 2 * kTileBytesA);
 #pragma unroll
-                        for (int k = 0; k < kBK / 16; ++k) {
-                            const uint32_t acc = (kb | k) != 0;
-                            umma_bf16_ss(d0, dg + 2 * k, db + 2 * k, idesc, acc);
-                            umma_bf16_ss(d0 + kFBN, du + 2 * k, db + 2 * k, idesc, acc);
-                        }
-                    } else {
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            const uint32_t su = st + u * (kTileBytesA + kFBN * kBK * 2);
-                            const uint64_t da = sw128_kmajor_desc(su), db = sw128_kmajor_desc(su + kTileBytesA);
-#pragma unroll
-                            for (int k = 0; k < kBK / 16; ++k)
-                                umma_bf16_ss(d0, da + 2 * k, db + 2 * k, idesc, (kb | u | k) != 0);
-                        }
+                    for (int k = 0; k < kBK / 16; ++k) {
+                        const uint32_t acc = (kb | k) != 0;
+                        umma_bf16_ss(d0, da0 + 2 * k, db + 2 * k, idesc, acc);
+                        if (ft.two) umma_bf16_ss(d0 + kFBN, da1 + 2 * k, db + 2 * k, idesc, acc);
                     }
                     umma_commit(&empty_bar[stage]);
                     if (++stage == kFStages) { stage = 0; phase ^= 1; }
@@ -344,30 +487,55 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap tmWgu, const __grid_cons
     } else if (warp < 6) {
         // ============================ warps 2-5: epilogue ========================
         const int q = warp & 3;
-        int buf = 0;
-        uint32_t bphase = 0;
-        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x) {
-            const FTile ft = fused_tile(tile, n_gu, fs, Et, MB_gu, MB_dn);
-            const TileInfo &ti = ft.t;
+        int buf = 0, qs = 0;
+        uint32_t bphase = 0, qph = 0;
+        for (;;) {
+            int tile = -1;
+            bool ok = true;
+            if (lane == 0) ok = pop_tile(fs, q_full, q_empty, qs, qph, abort_flag, a.err, tile);
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            tile = __shfl_sync(0xffffffffu, tile, 0);
+            if (++qs == kFQueue) { qs = 0; qph ^= 1; }
+            if (!ok || tile < 0) break;
+            const FTile ft = fused_tile(tile, tc, fs, MB_gu, MB_dn, a.H);
             if (!__shfl_sync(0xffffffffu, mbar_wait(&tfull_bar[buf], bphase, abort_flag, a.err, 128), 0)) break;
             tc_fence_after_sync();
-            const int m_out = ft.gu ? a.I : a.H;
-            const int f = ti.mb * kBM + q * 32 + lane;
-            const bool f_ok = f < m_out;
-            uint16_t *dst = (ft.gu ? a.act : a.y) + static_cast<size_t>(ti.row0) * m_out + f;
             const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + buf * kFAccCols;
-            for (int c0 = 0; c0 < ti.n_mma; c0 += 16) {
-                uint32_t g[16], u[16];
-                tmem_ld_32x32b_x16(tb + c0, g);
-                if (ft.gu) tmem_ld_32x32b_x16(tb + kFBN + c0, u);
-                tmem_wait_ld();
+            if (ft.gu) {
+                const int f = ft.mb * kBM + q * 32 + lane;
+                const bool f_ok = f < a.I;
+                uint16_t *dst = a.act + static_cast<size_t>(ft.row0) * a.I + f;
+                for (int c0 = 0; c0 < ft.n_mma; c0 += 16) {
+                    uint32_t g[16], u[16];
+                    tmem_ld_32x32b_x16(tb + c0, g);
+                    tmem_ld_32x32b_x16(tb + kFBN + c0, u);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const int n = c0 + j;
-                    if (f_ok && n < ti.valid) {
-                        float v = __uint_as_float(g[j]);
-                        if (ft.gu) v = v / (1.0f + expf(-v)) * __uint_as_float(u[j]);
-                        dst[static_cast<size_t>(n) * m_out] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+                    for (int j = 0; j < 16; ++j) {
+                        const int n = c0 + j;
+                        if (f_ok && n < ft.valid) {
+                            float v = __uint_as_float(g[j]);
+                            v = v / (1.0f + expf(-v)) * __uint_as_float(u[j]);
+                            dst[static_cast<size_t>(n) * a.I] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+                        }
+                    }
+                }
+            } else {
+                for (int h = 0; h < (ft.two ? 2 : 1); ++h) {
+                    const int f = ft.mb * 2 * kBM + (ft.h0 + h) * kBM + q * 32 + lane;
+                    const bool f_ok = f < a.H;
+                    uint16_t *dst = a.y + static_cast<size_t>(ft.row0) * a.H + f;
+                    for (int c0 = 0; c0 < ft.n_mma; c0 += 16) {
+                        uint32_t v[16];
+                        tmem_ld_32x32b_x16(tb + h * kFBN + c0, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int j = 0; j < 16; ++j) {
+                            const int n = c0 + j;
+                            if (f_ok && n < ft.valid)
+                                dst[static_cast<size_t>(n) * a.H] =
+                                    __bfloat16_as_ushort(__float2bfloat16_rn(__uint_as_float(v[j])));
+                        }
                     }
                 }
             }
@@ -377,14 +545,16 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap tmWgu, const __grid_cons
             // of this expert (TMA reads of act) or for finalize
             if (ft.gu) fence_proxy_async_global();
             __syncwarp();
-            if (lane == 0) red_release_add_u32(ft.gu ? a.gu_done + ti.e : a.dn_done, 1u);
+            if (lane == 0) red_release_add_u32(ft.gu ? a.gu_done + ft.e : a.dn_done, 1u);
             if (++buf == 2) { buf = 0; bphase ^= 1; }
         }
     }
 
     // ---- finalize: once every down tile has finished, on every CTA ---------------
     __syncthreads();
-    if (threadIdx.x == 0) wait_count(a.dn_done, 4u * static_cast<unsigned int>(n_dn), abort_flag, a.err);
+    griddep_launch_dependents();
+    if (threadIdx.x == 0)
+        wait_count(a.dn_done, 4u * static_cast<unsigned int>(tc.n_dn + tc.n_split), abort_flag, a.err);
     __syncthreads();
     if (!*abort_flag) {
         ld_acquire_u32(a.dn_done);
@@ -396,18 +566,30 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap tmWgu, const __grid_cons
              i += static_cast<long long>(gridDim.x) * kFThreads) {
             const int t = static_cast<int>(i / vpr);
             const int v = static_cast<int>(i - static_cast<long long>(t) * vpr);
-            float acc[8];
-            for (int j = 0; j < K; ++j) {
-                const int r = fs.inv[t * K + j];
-                const float wj = fs.w[t * K + j];
-                uint4 qv = make_uint4(0u, 0u, 0u, 0u);
-                if (r >= 0 && r < P) qv = __ldcg(y4 + static_cast<size_t>(r) * vpr + v);
-                else if (v == 0) raise_error(a.err, kErrBadRow);
-                const uint32_t qs[4] = {qv.x, qv.y, qv.z, qv.w};
+            // every slot's y row first (one L2 latency), then the sum in slot order
+            uint4 yv[kFMaxSlots];
+            float wv[kFMaxSlots];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float x = bf16_bits_to_float((qs[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu);
-                    acc[e] = (j == 0) ? __fmul_rn(x, wj) : __fmaf_rn(x, wj, acc[e]);
+            for (int j = 0; j < kFMaxSlots; ++j) {
+                yv[j] = make_uint4(0u, 0u, 0u, 0u);
+                wv[j] = 0.f;
+                if (j < K) {
+                    const int r = fs.inv[t * K + j];
+                    wv[j] = fs.w[t * K + j];
+                    if (r >= 0 && r < P) yv[j] = __ldcg(y4 + static_cast<size_t>(r) * vpr + v);
+                    else if (v == 0) raise_error(a.err, kErrBadRow);
+                }
+            }
+            float acc[8];
+#pragma unroll
+            for (int j = 0; j < kFMaxSlots; ++j) {
+                if (j < K) {
+                    const uint32_t qs[4] = {yv[j].x, yv[j].y, yv[j].z, yv[j].w};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const float x = bf16_bits_to_float((qs[e >> 1] >> ((e & 1) * 16)) & 0xFFFFu);
+                        acc[e] = (j == 0) ? __fmul_rn(x, wv[j]) : __fmaf_rn(x, wv[j], acc[e]);
+                    }
                 }
             }
             uint4 o;
@@ -431,35 +613,21 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap tmWgu, const __grid_cons
     }
 }
 
-constexpr size_t kFSmemBytes = 1024 + static_cast<size_t>(kFStages) * kFSlot + 8 * (2 * kFStages + 5) + 64 +
-                               sizeof(FusedSmem);
+constexpr size_t kFBarBytes = 8 * (2 * kFStages + 4 + 2 * kFQueue + 1);
+constexpr size_t kFSmemBytes = 1024 + static_cast<size_t>(kFStages) * kFSlot + kFBarBytes + 64 + sizeof(FusedSmem);
 static_assert(kFSmemBytes + 64 <= kSmemLimit, "shared memory");
-static_assert(kFGuStage <= kFSlot, "a gate/up stage fits a ring slot");
-// routing scratch in the ring: ids, counts, and the bucketing's (8 + 2) x E histograms
-static_assert((kFMaxP + kFMaxE + 10 * kFMaxE) * 4 <= kFStages * kFSlot, "routing scratch fits the ring");
+static_assert(kFMaxE <= kFThreads, "one scan thread per expert");
+static_assert(kFMaxT <= 64, "token masks are 64 bits");
+static_assert(kFTmemCols <= 512, "TMEM");
 
 template <int PER_LANE>
 cudaError_t launch_fused_t(const FusedArgs &a, const CUtensorMap (&m)[4], cudaStream_t s) {
     auto kern = fused_decode_kernel<PER_LANE>;
     cudaError_t st = ensure_dynamic_smem(kern, kFSmemBytes);
     if (st != cudaSuccess) return st;
-    int dev = 0, blocks_per_sm = 0;
-    if ((st = cudaGetDevice(&dev)) != cudaSuccess) return st;
-    if ((st = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks_per_sm, kern, kFThreads, kFSmemBytes)) !=
-        cudaSuccess)
-        return st;
-    if (blocks_per_sm < 1) return cudaErrorInvalidConfiguration;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(num_sms());           // one CTA per SM, all resident (cooperative launch)
-    cfg.blockDim = dim3(kFThreads);
-    cfg.dynamicSmemBytes = kFSmemBytes;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], a);
+    // one CTA per SM (the shared memory admits no second); tiles are handed
+    // out dynamically, so no CTA needs another to be resident at the same time
+    return launch_pdl(kern, dim3(num_sms()), dim3(kFThreads), kFSmemBytes, s, m[0], m[1], m[2], m[3], a);
 }
 
 }  // namespace
@@ -468,6 +636,8 @@ bool fused_decode_supported(int T, int H, int I, int E, int k, int S, int fmt) {
     return fmt == 0 && T >= 1 && T <= kFMaxT && k + S <= kFMaxSlots && E + S <= kFMaxE && E <= kFMaxE &&
            H % 8 == 0 && I % 8 == 0;
 }
+
+size_t fused_counter_words(int E, int S) { return static_cast<size_t>(E + S) + 3; }
 
 cudaError_t launch_fused_decode(const float *logits, const uint16_t *hidden, const void *w_gu, const void *w_d,
                                 int T, int H, int I, int E, int k, int S, int32_t *ids, float *w, int32_t *counts,
@@ -483,8 +653,9 @@ cudaError_t launch_fused_decode(const float *logits, const uint16_t *hidden, con
               make_map(&m[2], hidden, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, H, T, kBK, 1, CU_TENSOR_MAP_SWIZZLE_128B) &&
               make_map(&m[3], act, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, I, P, kBK, kBoxN, CU_TENSOR_MAP_SWIZZLE_128B);
     if (!ok) return cudaErrorInvalidValue;
-    // the completion counters start at zero on every call
-    cudaError_t st = cudaMemsetAsync(done, 0, sizeof(unsigned int) * (Et + 1), s);
+    // the counters start at zero on every call
+    cudaError_t st = launch_pdl(fused_reset_kernel, dim3(1), dim3(32), 0, s, done,
+                                static_cast<int>(fused_counter_words(E, S)));
     if (st != cudaSuccess) return st;
     FusedArgs a;
     a.logits = logits;
@@ -505,6 +676,8 @@ cudaError_t launch_fused_decode(const float *logits, const uint16_t *hidden, con
     a.out = out;
     a.gu_done = done;
     a.dn_done = done + Et;
+    a.next_tile = done + Et + 1;
+    a.routed = done + Et + 2;
     a.err = err;
     const int per_lane = (E + 31) / 32;
     if (per_lane <= 1) return launch_fused_t<1>(a, m, s);

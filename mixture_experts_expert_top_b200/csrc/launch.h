@@ -118,8 +118,10 @@ struct MxGemmArgs {
 };
 cudaError_t launch_grouped_gemm_mxfp8(const MxGemmArgs &g, cudaStream_t s);
 // ---- fused_decode_sm100.cu: the whole bf16 layer for a decode batch in one
-// persistent cooperative kernel (T <= 64, k + S <= 16, E + S <= 256). done:
-// E + S + 1 counters of the workspace, zeroed by the launcher.
+// persistent kernel (T <= 64, k + S <= 16, E + S <= 256). done:
+// fused_counter_words(E, S) counters of the workspace, zeroed on the stream
+// by the launcher before the kernel.
+size_t fused_counter_words(int E, int S);
 bool fused_decode_supported(int T, int H, int I, int E, int k, int S, int fmt);
 cudaError_t launch_fused_decode(const float *logits, const uint16_t *hidden, const void *w_gu, const void *w_d,
                                 int T, int H, int I, int E, int k, int S, int32_t *ids, float *w, int32_t *counts,

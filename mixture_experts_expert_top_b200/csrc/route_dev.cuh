@@ -55,10 +55,12 @@ __device__ __forceinline__ void route_token(const float *row, int E, int k, int 
         for (int i = PER_LANE - 1; i >= 0; --i)
             if (key[i] == best) cand = static_cast<uint32_t>(lane + 32 * i);
         const int bid = static_cast<int>(__reduce_min_sync(0xffffffffu, cand));
-        if ((bid & 31) == lane) {
+        const bool mine = (bid & 31) == lane;
+        if constexpr (PER_LANE <= 8) {
 #pragma unroll
-            for (int i = 0; i < PER_LANE; ++i)
-                if (i == (bid >> 5)) key[i] = 0u;
+            for (int i = 0; i < PER_LANE; ++i) key[i] = (mine && i == (bid >> 5)) ? 0u : key[i];   // in registers
+        } else if (mine) {
+            key[bid >> 5] = 0u;
         }
         if (lane == j) {
             my_id = bid;

@@ -136,14 +136,23 @@ def test_empty_batch_is_a_no_op():
 
 
 def test_forward_kernel_count():
+    # bf16 decode batches: the counter reset and the persistent kernel; else
     # one-CTA route+permute for T <= 64; the decode-shaped gate/up reads its
     # token rows through perm; prefill shapes add two bucketing kernels (three
     # past 64 chunks of 2048 pairs or 512 experts) and the gather
-    sh = lambda c: moe.Shape.of(c.T, c.H, c.I, c.E, c.k, c.fmt)
+    sh = lambda c: moe.Shape.of(c.T, c.H, c.I, c.E, c.k, c.fmt, n_shared=c.n_shared)
     count = lambda c: moe.moe_forward_kernel_count(sh(c))
-    assert count(moe_synth.get_config("qwen3_decode")) == 4
-    assert count(moe_synth.get_config("tiny")) == 4
+    assert count(moe_synth.get_config("qwen3_decode")) == 2
+    assert count(moe_synth.get_config("tiny")) == 2
+    assert count(moe_synth.get_config("shared_decode")) == 2
+    assert count(moe_synth.get_config("mxfp8_decode")) == 5
+    assert count(moe_synth.get_config("qwen3_decode", T=65)) == 5            # past the persistent kernel's batch
     assert count(moe_synth.get_config("w4a16_decode")) == 5
+    fused = lambda c: moe.moe_forward_is_fused(sh(c))
+    assert fused(moe_synth.get_config("qwen3_decode")) and fused(moe_synth.get_config("shared_decode"))
+    assert not fused(moe_synth.get_config("w4a16_decode")) and not fused(moe_synth.get_config("mxfp8_decode"))
+    assert not fused(moe_synth.get_config("qwen3_prefill"))
+    assert not fused(moe_synth.get_config("qwen3_decode", E=300))                # more experts than it takes
     assert count(moe_synth.get_config("qwen3_prefill")) == 7
     assert count(moe_synth.get_config("skewed")) == 7
     assert count(moe_synth.get_config("qwen3_prefill", T=20000)) == 8           # 79 chunks: separate scan
@@ -180,7 +189,7 @@ int main(void) {
     int rc = 0;
     if (ws == 0) rc = 1;
     if (moe_workspace_size(&bad) != 0) rc = 2;
-    if (moe_forward_kernel_count(&s) != 4) rc = 3;
+    if (moe_forward_kernel_count(&s) != 2 || moe_forward_is_fused(&s) != 1) rc = 3;
     if (strcmp(moe_status_string(MOE_OK), "ok") != 0) rc = 4;
     /* T = 0 enqueues nothing and succeeds without a GPU */
     s.T = 0;

@@ -109,7 +109,9 @@ def test_bench_work_accounting():
     assert w["active_experts"] == 120
     assert w["weight_bytes"] == 120 * 3 * 2048 * 768 * 2
     assert w["layer_flops"] == 2 * 64 * 8 * 3 * 2048 * 768
-    assert bench.launches_per_step(cfg) == 4          # route+permute, gate/up (own gather), down, finalize
+    assert bench.launches_per_step(cfg) == 2          # counter reset, the persistent decode kernel
+    assert w["fused"]["bytes"] == w["weight_bytes"] + 64 * 2048 * 2 * 2 + 64 * 128 * 4
+    assert bench.launches_per_step(moe_synth.get_config("qwen3_decode", T=65)) == 5   # route, permute, 2 GEMMs, finalize
     assert bench.launches_per_step(moe_synth.get_config("qwen3_prefill")) == 7
     q = moe_synth.get_config("w4a16_decode")
     wq = bench.work_per_step(q, [8] * 256)
