@@ -16,6 +16,7 @@ for the W4A16 format):
   skewed         T=4096, H=4096, I=1536, E=64,  k=6   bf16, logits + 3 ln Zipf(1.2)
   w4a16_decode   T=256,  H=7168, I=2048, E=256, k=8   int4 weights, 1 bf16 scale / 128 K
   mxfp8_decode   T=64,   H=2048, I=768,  E=128, k=8   MXFP8 weights (E4M3, 1 E8M0 scale / 32 K)
+  mxfp4_decode   T=64,   H=2048, I=768,  E=128, k=8   MXFP4 weights (E2M1, 1 E8M0 scale / 32 K)
   shared_decode  T=64,   H=2048, I=768,  E=64,  k=6   bf16, plus 2 shared experts
 
 Draw recipe. Every tensor has its own torch CPU generator, seeded from
@@ -32,6 +33,9 @@ generator, by scales U(0.002,0.02) fp32 rounded to bf16, one per 128
 consecutive K elements of a row. MXFP8 weights are E4M3 codes with a uniform
 sign, an exponent field uniform on 4..7 and a uniform mantissa, followed by
 E8M0 scale codes uniform on 120..122, one per 32 consecutive K elements.
+MXFP4 weights are E2M1 codes with a uniform sign and a magnitude code
+uniform on 1..7, two per byte (the even K index in the low nibble), followed
+by E8M0 scale codes uniform on 119..121, one per 32 consecutive K elements.
 """
 
 from __future__ import annotations
@@ -62,7 +66,7 @@ class MoeConfig:
     I: int
     E: int
     k: int
-    fmt: str = "bf16"          # "bf16", "int4_g128" or "mxfp8"
+    fmt: str = "bf16"          # "bf16", "int4_g128", "mxfp8" or "mxfp4"
     logit_extra: str = "none"  # "none", "bias0.5" or "zipf1.2"
     weight_std: float = 0.02
     n_shared: int = 0          # shared experts: weight arrays hold E + n_shared experts
@@ -92,6 +96,7 @@ CONFIGS: Dict[str, MoeConfig] = {
         # beyond the five workloads above: the Qwen3 decode shape with MXFP8
         # weights, and a decode layer with two shared experts
         MoeConfig("mxfp8_decode", 64, 2048, 768, 128, 8, fmt="mxfp8"),
+        MoeConfig("mxfp4_decode", 64, 2048, 768, 128, 8, fmt="mxfp4"),
         MoeConfig("shared_decode", 64, 2048, 768, 64, 6, n_shared=2),
     ]
 }
@@ -171,6 +176,20 @@ def gen_expert_weights(cfg: MoeConfig, e: int, seed: int = 0) -> Dict[str, torch
             out[name] = (sign | expo | mant).to(torch.uint8)
             out[name + "_scales"] = torch.randint(120, 123, (rows, K // 32), generator=g, dtype=torch.int32).to(torch.uint8)
         return out
+    if cfg.fmt == "mxfp4":
+        if H % 32 or I % 32:
+            raise ValueError("mxfp4 needs H and I multiples of 32")
+        out = {}
+        for name, g, rows, K in (("w_gu", g_gu, 2 * I, H), ("w_d", g_d, H, I)):
+            # E2M1 codes: sign uniform, magnitude code uniform on 1..7 (0.5 .. 6),
+            # two per byte with the even K index in the low nibble; E8M0 scale
+            # codes uniform on 119..121 (2^-8 .. 2^-6)
+            sign = torch.randint(0, 2, (rows, K), generator=g, dtype=torch.int32) << 3
+            mag = torch.randint(1, 8, (rows, K), generator=g, dtype=torch.int32)
+            nib = sign | mag
+            out[name] = (nib[:, 0::2] | (nib[:, 1::2] << 4)).to(torch.uint8)
+            out[name + "_scales"] = torch.randint(119, 122, (rows, K // 32), generator=g, dtype=torch.int32).to(torch.uint8)
+        return out
     raise ValueError(f"unknown weight format {cfg.fmt!r}")
 
 
@@ -190,6 +209,13 @@ def gen_inputs(cfg: MoeConfig, seed: int = 0, experts: Optional[Iterable[int]] =
     E, H, I = cfg.E + cfg.n_shared, cfg.H, cfg.I       # routed experts, then the shared ones
     if cfg.fmt == "bf16":
         shapes = {"w_gu": ((E, 2 * I, H), torch.bfloat16), "w_d": ((E, H, I), torch.bfloat16)}
+    elif cfg.fmt == "mxfp4":
+        shapes = {
+            "w_gu": ((E, 2 * I, H // 2), torch.uint8),
+            "w_gu_scales": ((E, 2 * I, H // 32), torch.uint8),
+            "w_d": ((E, H, I // 2), torch.uint8),
+            "w_d_scales": ((E, H, I // 32), torch.uint8),
+        }
     elif cfg.fmt == "mxfp8":
         shapes = {
             "w_gu": ((E, 2 * I, H), torch.uint8),

@@ -49,6 +49,7 @@ def lib() -> ctypes.CDLL:
         L.oracle_set_num_threads.argtypes = [i32]
         L.oracle_mx_quantize.argtypes = [vp, i32, i32, vp, vp]
         L.oracle_mx_dequantize.argtypes = [vp, vp, i32, i32, vp]
+        L.oracle_mx4_dequantize.argtypes = [vp, vp, i32, i32, vp]
         for f in ("oracle_route", "oracle_permute", "oracle_forward", "oracle_forward_shared",
                   "oracle_forward_tokens", "oracle_num_threads"):
             getattr(L, f).restype = ctypes.c_int
@@ -99,6 +100,8 @@ def _fmt_code(fmt: str) -> int:
         return 1
     if fmt == "mxfp8":
         return 2
+    if fmt == "mxfp4":
+        return 3
     raise ValueError(fmt)
 
 
@@ -120,6 +123,18 @@ def mx_dequantize(q, scales) -> np.ndarray:
     rows, K = qa.shape
     out = np.zeros((rows, K), np.float64)
     lib().oracle_mx_dequantize(_p(qa), _p(sa), rows, K, _p(out))
+    return out
+
+
+def mx4_dequantize(q, scales) -> np.ndarray:
+    """Decoded values (float64 [rows, K]) of MXFP4 weights: E2M1 codes packed
+    two per byte [rows, K/2] (even K index in the low nibble) and E8M0 scale
+    codes [rows, K/32]."""
+    qa = _np(q, np.uint8)
+    sa = _np(scales, np.uint8)
+    rows, K = qa.shape[0], qa.shape[1] * 2
+    out = np.zeros((rows, K), np.float64)
+    lib().oracle_mx4_dequantize(_p(qa), _p(sa), rows, K, _p(out))
     return out
 
 
@@ -217,8 +232,8 @@ def _weights(inputs: Dict[str, torch.Tensor], fmt: str):
 
 
 def _inner(d: np.ndarray, f: int) -> int:
-    """I from the down weights [E, H, I] (int4: packed, I/2 bytes per row)."""
-    return d.shape[2] * 2 if f == 1 else d.shape[2]
+    """I from the down weights [E, H, I] (int4 and MXFP4: packed, I/2 bytes per row)."""
+    return d.shape[2] * 2 if f in (1, 3) else d.shape[2]
 
 
 def forward(inputs: Dict[str, torch.Tensor], k: int, fmt: str = "bf16", n_shared: int = 0) -> Dict[str, np.ndarray]:

@@ -177,6 +177,28 @@ void oracle_mx_quantize(const uint16_t *x, int rows, int K, uint8_t *q, uint8_t 
     }
 }
 
+/* ---- MXFP4 weights (OCP MX v1.0: E2M1 elements, one E8M0 scale per 32) ------
+ * E2M1: sign bit 3, 2-bit exponent field (bits 2-1, bias 1), 1-bit mantissa
+ * (bit 0); field 0 is subnormal (m * 2^-1), otherwise (1 + m/2) * 2^(field-1);
+ * no infinities or NaN. Two elements per byte, the even K index in the low
+ * nibble (the int4 layout's packing). */
+static double e2m1_value(unsigned code) {
+    int sign = (code >> 3) & 1, ex = (code >> 1) & 3, m = code & 1;
+    double v = ex == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, ex - 1);
+    return sign ? -v : v;
+}
+
+static double mx4_value(const uint8_t *row_q, const uint8_t *row_s, int k) {
+    uint8_t b = row_q[k / 2];
+    return e2m1_value((k & 1) ? (b >> 4) : (b & 15)) * e8m0_value(row_s[k / 32]);
+}
+
+void oracle_mx4_dequantize(const uint8_t *q, const uint8_t *scales, int rows, int K, double *out) {
+    for (int r = 0; r < rows; ++r)
+        for (int k = 0; k < K; ++k)
+            out[(size_t)r * K + k] = mx4_value(q + (size_t)r * (K / 2), scales + (size_t)r * (K / 32), k);
+}
+
 /* Decoded value of element k of an MX row: E4M3 element times its block's E8M0 scale. */
 static double mx_value(const uint8_t *row_q, const uint8_t *row_s, int k) {
     return e4m3_value(row_q[k]) * e8m0_value(row_s[k / 32]);
@@ -317,22 +339,26 @@ void oracle_dequant_int4(const uint8_t *q, const uint16_t *scales, int rows, int
  * #500 §2.2 (gate/up grouped GEMM, then SwiGLU);
  * y[h] = bf16(sum_i act[i] * W_d[h][i]) (R6), the down grouped GEMM.
  * Weights are bf16 (fmt 0), int4 + bf16 scales (fmt 1, decoded per element)
- * or MXFP8 (fmt 2: E4M3 + one E8M0 scale per 32 K, decoded per element; the
+ * MXFP8 (fmt 2: E4M3 + one E8M0 scale per 32 K, decoded per element; the
  * activation row x, and act before the down projection, are MX-quantised
- * first, since the block-scaled MMA takes both operands in MXFP8).
+ * first, since the block-scaled MMA takes both operands in MX form) or MXFP4
+ * (fmt 3: E2M1 + one E8M0 scale per 32 K, with activations MX-quantised to
+ * E4M3 as for fmt 2: FP4 weights times FP8 activations).
  */
 static double weight_at(int fmt, const void *w, const void *s, int K, int row, int col) {
     if (fmt == 0) return (double)bf16_to_f32(((const uint16_t *)w)[(size_t)row * K + col]);
     if (fmt == 1)
         return (double)bf16_to_f32(dequant_one((const uint8_t *)w + (size_t)row * (K / 2),
                                                (const uint16_t *)s + (size_t)row * (K / 128), col));
+    if (fmt == 3)
+        return mx4_value((const uint8_t *)w + (size_t)row * (K / 2), (const uint8_t *)s + (size_t)row * (K / 32), col);
     return mx_value((const uint8_t *)w + (size_t)row * K, (const uint8_t *)s + (size_t)row * (K / 32), col);
 }
 
-/* The activation row as the MMA sees it: bf16 values, or for fmt 2 the
- * decoded MX quantisation of the row. xv has K entries. */
+/* The activation row as the MMA sees it: bf16 values, or for fmt 2 and 3 the
+ * decoded MXFP8 quantisation of the row. xv has K entries. */
 static void activation_values(int fmt, const uint16_t *x, int K, double *xv) {
-    if (fmt != 2) {
+    if (fmt < 2) {
         for (int k = 0; k < K; ++k) xv[k] = (double)bf16_to_f32(x[k]);
         return;
     }
@@ -425,10 +451,10 @@ void oracle_finalize(const uint16_t *y, const float *w, const int32_t *inv_perm,
  * independent. */
 /* Bytes of one expert's weight matrix [rows, K] and of its scales in format fmt. */
 static size_t weight_bytes(int fmt, int rows, int K) {
-    return fmt == 0 ? (size_t)rows * K * 2 : fmt == 1 ? (size_t)rows * (K / 2) : (size_t)rows * K;
+    return fmt == 0 ? (size_t)rows * K * 2 : fmt == 2 ? (size_t)rows * K : (size_t)rows * (K / 2);
 }
 static size_t scale_bytes(int fmt, int rows, int K) {
-    return fmt == 1 ? (size_t)rows * (K / 128) * 2 : fmt == 2 ? (size_t)rows * (K / 32) : 0;
+    return fmt == 1 ? (size_t)rows * (K / 128) * 2 : fmt >= 2 ? (size_t)rows * (K / 32) : 0;
 }
 
 static void ffn_rows(int fmt, const uint16_t *hidden, const void *w_gu, const void *w_gu_s, const void *w_d,
@@ -452,7 +478,7 @@ int oracle_forward(int fmt, const uint16_t *hidden, const float *logits,
                    int32_t *ids, float *w, int32_t *counts, int32_t *offsets,
                    int32_t *perm, int32_t *inv_perm, uint16_t *act, uint16_t *y, uint16_t *out) {
     if (T < 0 || H < 1 || I < 1 || k < 1 || k > E) return -1;
-    if ((fmt == 1 && (H % 128 || I % 128)) || (fmt == 2 && (H % 32 || I % 32)) || fmt < 0 || fmt > 2) return -1;
+    if ((fmt == 1 && (H % 128 || I % 128)) || (fmt >= 2 && (H % 32 || I % 32)) || fmt < 0 || fmt > 3) return -1;
     int P = T * k;
     if (oracle_route(logits, T, E, k, ids, w)) return -1;
     if (oracle_permute(ids, P, E, counts, offsets, perm, inv_perm)) return -1;
@@ -479,7 +505,7 @@ int oracle_forward_shared(int fmt, const uint16_t *hidden, const float *logits,
     if (S == 0) return oracle_forward(fmt, hidden, logits, w_gu, w_gu_s, w_d, w_d_s, T, H, I, E, k,
                                       ids, w, counts, offsets, perm, inv_perm, act, y, out);
     if (T < 0 || H < 1 || I < 1 || k < 1 || k > E) return -1;
-    if ((fmt == 1 && (H % 128 || I % 128)) || (fmt == 2 && (H % 32 || I % 32)) || fmt < 0 || fmt > 2) return -1;
+    if ((fmt == 1 && (H % 128 || I % 128)) || (fmt >= 2 && (H % 32 || I % 32)) || fmt < 0 || fmt > 3) return -1;
     int K = k + S, P = T * K;
     int32_t *ids_k = (int32_t *)malloc(sizeof(int32_t) * (size_t)(T > 0 ? T : 1) * k);
     float *w_k = (float *)malloc(sizeof(float) * (size_t)(T > 0 ? T : 1) * k);
@@ -515,7 +541,7 @@ int oracle_forward_tokens(int fmt, const uint16_t *hidden, const float *logits,
                           int T, int H, int I, int E, int k, const int32_t *tokens, int n_tokens,
                           int32_t *ids_out, float *w_out, uint16_t *out_rows) {
     if (T < 0 || H < 1 || I < 1 || k < 1 || k > E || n_tokens < 0) return -1;
-    if ((fmt == 1 && (H % 128 || I % 128)) || (fmt == 2 && (H % 32 || I % 32)) || fmt < 0 || fmt > 2) return -1;
+    if ((fmt == 1 && (H % 128 || I % 128)) || (fmt >= 2 && (H % 32 || I % 32)) || fmt < 0 || fmt > 3) return -1;
     for (int n = 0; n < n_tokens; ++n) {
         if (tokens[n] < 0 || tokens[n] >= T) return -1;
         if (oracle_route(logits + (size_t)tokens[n] * E, 1, E, k, ids_out + (size_t)n * k, w_out + (size_t)n * k))

@@ -533,3 +533,87 @@ def test_mxfp8_ffn_matches_dense_double_of_the_decoded_operands():
             aq = oracle.mx_dequantize(*oracle.mx_quantize(a_ref[None]))[0]
             y_ref = torch.from_numpy(np.float32(wd @ aq)).to(torch.bfloat16)
             assert np.array_equal(y, bf16_bits(y_ref))
+
+
+# ------------------------------------------------- MXFP4 weights (fmt 3) --
+
+# The E2M1 element values of the OCP Microscaling Formats (MX) v1.0 spec
+# (FP4 E2M1: bias 1, 1 mantissa bit, no infinities or NaN), by code 0..7;
+# codes 8..15 are the same magnitudes negated.
+E2M1_TABLE = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+def _unpack_e2m1(q: np.ndarray) -> np.ndarray:
+    """Codes [rows, K] from packed bytes [rows, K/2], even K in the low nibble."""
+    lo, hi = q & 15, q >> 4
+    return np.stack([lo, hi], axis=-1).reshape(q.shape[0], -1)
+
+
+def _e2m1_table_values(codes: np.ndarray) -> np.ndarray:
+    mag = np.array(E2M1_TABLE)[codes & 7]
+    return np.where(codes & 8, -mag, mag)
+
+
+def test_e2m1_codes_decode_as_the_mx_table_with_their_block_scale():
+    codes = np.arange(16, dtype=np.uint8)
+    q = np.zeros((16, 16), np.uint8)
+    q[:, 0] = codes                         # element 0 (low nibble) = code, element 1 = 0
+    q[:, 1] = codes << 4                    # element 3 (high nibble of byte 1) = code
+    sc = np.full((16, 1), 127 + 3, np.uint8)   # scale 2^3
+    dec = oracle.mx4_dequantize(q, sc)
+    ref = _e2m1_table_values(codes.astype(np.int64)) * 8.0
+    assert np.array_equal(dec[:, 0], ref)
+    assert np.array_equal(dec[:, 3], ref)
+    assert not dec[:, [1, 2]].any() and not dec[:, 4:].any()
+    # code 8 is -0.0 (sign bit only)
+    assert math.copysign(1.0, dec[8, 0]) == -1.0 and dec[8, 0] == 0.0
+    # the scale applies per 32 elements: two blocks of one row with scales 2^-1 and 2^2
+    q = np.full((1, 32), 0x22, np.uint8)                  # every element code 2 (1.0)
+    dec = oracle.mx4_dequantize(q, np.array([[126, 129]], np.uint8))
+    assert np.array_equal(dec[0], np.r_[np.full(32, 0.5), np.full(32, 4.0)])
+
+
+def test_mxfp4_weight_ffn_matches_dense_double_of_the_table_decoded_operands():
+    # FP4 weights (decoded here from the MX table, not by the oracle), FP8
+    # activations (the oracle's MX quantisation, pinned above), double sums
+    cfg = moe_synth.MoeConfig("mx4_small", T=5, H=128, I=64, E=3, k=2, fmt="mxfp4")
+    inp = moe_synth.gen_inputs(cfg, seed=33)
+
+    def table_decode(q, s):
+        codes = _unpack_e2m1(q.numpy())
+        return _e2m1_table_values(codes.astype(np.int64)) * np.repeat(
+            2.0 ** (s.numpy().astype(np.int64) - 127), 32, axis=1)
+
+    for e in range(cfg.E):
+        wgu = table_decode(inp["w_gu"][e], inp["w_gu_scales"][e])
+        wd = table_decode(inp["w_d"][e], inp["w_d_scales"][e])
+        assert np.array_equal(wgu, oracle.mx4_dequantize(inp["w_gu"][e], inp["w_gu_scales"][e]))
+        for t in range(cfg.T):
+            act, y = oracle.expert_ffn(inp["hidden"][t], inp["w_gu"][e], inp["w_d"][e], cfg.H, cfg.I, fmt="mxfp4",
+                                       w_gu_scales=inp["w_gu_scales"][e], w_d_scales=inp["w_d_scales"][e])
+            xq = oracle.mx_dequantize(*oracle.mx_quantize(inp["hidden"][t:t + 1]))[0]
+            g = np.float32(wgu[:cfg.I] @ xq).astype(np.float64)
+            u = np.float32(wgu[cfg.I:] @ xq).astype(np.float64)
+            a_ref = torch.from_numpy((g / (1 + np.exp(-g)) * u).astype(np.float32)).to(torch.bfloat16)
+            assert np.array_equal(act, bf16_bits(a_ref))
+            aq = oracle.mx_dequantize(*oracle.mx_quantize(a_ref[None]))[0]
+            y_ref = torch.from_numpy(np.float32(wd @ aq)).to(torch.bfloat16)
+            assert np.array_equal(y, bf16_bits(y_ref))
+
+
+def test_mxfp4_layer_equals_its_steps_and_zero_down_weights_give_zero():
+    cfg = moe_synth.MoeConfig("mx4_layer", T=8, H=128, I=64, E=4, k=2, fmt="mxfp4")
+    inp = moe_synth.gen_inputs(cfg, seed=34)
+    r = oracle.forward(inp, cfg.k, fmt="mxfp4")
+    # every permuted row's act/y equals the single-expert evaluation
+    ids = r["ids"].reshape(-1)
+    for row in range(cfg.P):
+        pair = int(r["perm"][row])
+        t, e = pair // cfg.k, int(ids[pair])
+        act, y = oracle.expert_ffn(inp["hidden"][t], inp["w_gu"][e], inp["w_d"][e], cfg.H, cfg.I, fmt="mxfp4",
+                                   w_gu_scales=inp["w_gu_scales"][e], w_d_scales=inp["w_d_scales"][e])
+        assert np.array_equal(r["act"][row], act) and np.array_equal(r["y"][row], y)
+    z = dict(inp)
+    z["w_d"] = torch.zeros_like(inp["w_d"])        # code 0 = +0.0 for every weight
+    rz = oracle.forward(z, cfg.k, fmt="mxfp4")
+    assert not (rz["out"] & 0x7FFF).any()
