@@ -52,7 +52,7 @@ TARGETS = {"qwen3_decode": ("hbm", 0.70), "w4a16_decode": ("hbm", 0.70),
            "qwen3_prefill": ("tensor", 0.60), "skewed": ("tensor", 0.60), "tiny": (None, None)}
 # measured beside the graded workloads (no target of their own): MXFP8
 # weights on the block-scaled MMA, and shared experts
-UNGRADED = ["mxfp8_decode", "shared_decode"]
+UNGRADED = ["mxfp8_decode", "mxfp4_decode", "shared_decode"]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 NORTH_STAR_HBM_GBS = 8000.0       # the roofline literals the layer's target is stated against
 NORTH_STAR_BF16_TFLOPS = 2250.0
@@ -299,6 +299,8 @@ def weight_row_bytes(fmt, K):
         return 2 * K
     if fmt == "int4_g128":
         return K // 2 + (K // 128) * 2
+    if fmt == "mxfp4":
+        return K // 2 + K // 32                 # E2M1 codes (two per byte) + E8M0 scales
     return K + K // 32                          # mxfp8: E4M3 codes + E8M0 scales
 
 
@@ -314,7 +316,7 @@ def work_per_step(cfg, counts):
     w_gu = active * 2 * I * weight_row_bytes(cfg.fmt, H)
     w_d = active * H * weight_row_bytes(cfg.fmt, I)
     # token operand bytes per element: bf16, or MX codes + scales
-    xb = (lambda K: K + K // 32) if cfg.fmt == "mxfp8" else (lambda K: 2 * K)
+    xb = (lambda K: K + K // 32) if cfg.fmt in ("mxfp8", "mxfp4") else (lambda K: 2 * K)
     return {
         "active_experts": active,
         "weight_bytes": w_gu + w_d,
@@ -362,10 +364,8 @@ def config_of(cfg, world):
 
 
 def expert_weight_bytes(cfg):
-    """Bytes of all E experts' weights (and int4 scales) of a workload."""
-    if cfg.fmt == "bf16":
-        return cfg.E * 3 * cfg.H * cfg.I * 2
-    return cfg.E * (2 * cfg.I * (cfg.H // 2 + cfg.H // 64) + cfg.H * (cfg.I // 2 + cfg.I // 64))
+    """Bytes of all E experts' weights (and scales) of a workload."""
+    return cfg.E * (2 * cfg.I * weight_row_bytes(cfg.fmt, cfg.H) + cfg.H * weight_row_bytes(cfg.fmt, cfg.I))
 
 
 def layer_fractions(cfg, work, layer_s, peaks):
@@ -479,7 +479,7 @@ def measure(cfg, args, dev, world, rank, sampler, headline):
     act = torch.empty(P, cfg.I, dtype=torch.bfloat16, device=dev)
     y = torch.empty(P, cfg.H, dtype=torch.bfloat16, device=dev)
     pws = torch.empty(max(1, moe.moe_permute_workspace_size(shape)), dtype=torch.uint8, device=dev)
-    if cfg.fmt == "mxfp8":
+    if cfg.fmt in ("mxfp8", "mxfp4"):
         # the MXFP8 layer: hidden quantised once per token, gate/up reads its
         # rows through perm and writes act quantised, down reads act's codes
         u8 = dict(dtype=torch.uint8, device=dev)
@@ -567,7 +567,7 @@ def measure(cfg, args, dev, world, rank, sampler, headline):
     wk = work[dom]
     # an MXFP8 contraction's peak: the measured bf16 peak times the nominal
     # fp8 / bf16 ratio of 2 (4.5 / 2.25 PFLOP/s dense)
-    fp8 = cfg.fmt == "mxfp8"
+    fp8 = cfg.fmt in ("mxfp8", "mxfp4")     # FP8 (or FP4 x FP8) operands on the block-scaled MMA
     tensor_peak = peaks["bf16_tflops"] * (2.0 if fp8 else 1.0)
     ridge = tensor_peak * 1e12 / (peaks["hbm_gbs"] * 1e9)
     launch_ms = stage_ms[dom]

@@ -23,12 +23,13 @@
  *  - Arguments are validated before anything is enqueued; a non-OK status
  *    means nothing was launched. T = 0 is valid and enqueues nothing.
  *  - Shape limits: 1 <= E <= 1024, 1 <= top_k <= min(E, 32), T*top_k < 2^31;
- *    H and I multiples of 8 (multiples of 128 for MOE_W_INT4_G128 and
- *    MOE_W_MXFP8).
+ *    H and I multiples of 8 (multiples of 128 for MOE_W_INT4_G128,
+ *    MOE_W_MXFP8 and MOE_W_MXFP4).
  *  - Weight scales are passed as untyped pointers: bf16 [rows, K/128] for
- *    MOE_W_INT4_G128, E8M0 bytes [rows, K/32] for MOE_W_MXFP8, NULL for bf16.
- *    Device pointers must be 16-byte aligned (4-byte for logits/topk_w and
- *    the int32 arrays).
+ *    MOE_W_INT4_G128, E8M0 bytes [rows, K/32] for MOE_W_MXFP8 and
+ *    MOE_W_MXFP4, NULL for bf16. Device pointers must be 16-byte aligned
+ *    (32-byte for MOE_W_MXFP4 weights; 4-byte for logits/topk_w and the
+ *    int32 arrays).
  *  - Pair ids: p = t*K + j for token t and slot j, with K = top_k +
  *    n_shared slots per token. Routed slot order is descending logit; equal
  *    logits go to the lower expert id; shared slots follow.
@@ -70,8 +71,10 @@ typedef enum {
 typedef enum {
     MOE_W_BF16 = 0,        /* bf16 weights */
     MOE_W_INT4_G128 = 1,   /* W4A16: int4 weights, one bf16 scale per 128 K */
-    MOE_W_MXFP8 = 2        /* MXFP8 (OCP MX v1.0): E4M3 weights, one E8M0 scale per 32 K;
+    MOE_W_MXFP8 = 2,       /* MXFP8 (OCP MX v1.0): E4M3 weights, one E8M0 scale per 32 K;
                               the activations are MX-quantised by the layer */
+    MOE_W_MXFP4 = 3        /* MXFP4 weights (OCP MX v1.0 E2M1, two per byte, even K in the
+                              low nibble, one E8M0 scale per 32 K) with MXFP8 activations */
 } moe_weight_fmt_t;
 
 /* Layer shape. T tokens, hidden size H, expert intermediate size I, E routed
@@ -257,11 +260,13 @@ MOE_API moe_status_t moe_forward_host(const moe_bf16_t *hidden_host, const float
 MOE_API moe_status_t moe_mx_quantize(const moe_bf16_t *x, int32_t rows, int32_t K, uint8_t *q, uint8_t *scales,
                                      moe_stream_t stream);
 
-/* Gate/up + SwiGLU with MXFP8 weights (shape->fmt = MOE_W_MXFP8):
+/* Gate/up + SwiGLU with MXFP8 or MXFP4 weights (shape->fmt = MOE_W_MXFP8
+ * or MOE_W_MXFP4; the token operand is MXFP8 either way):
  *   a_q, a_scales  perm == NULL: permuted rows [T*top_k, H] / [T*top_k, H/32];
  *                  perm != NULL: hidden's quantisation [T, H] / [T, H/32], rows
  *                  read through perm (TMA gather4)
- *   w_gu [E,2I,H] E4M3, w_gu_scales [E,2I,H/32] E8M0
+ *   w_gu MOE_W_MXFP8: [E,2I,H] E4M3; MOE_W_MXFP4: [E,2I,H/2] packed E2M1;
+ *        w_gu_scales [E,2I,H/32] E8M0
  *   act_q [T*top_k, I] E4M3 and act_scales [T*top_k, I/32] out: the MX
  *   quantisation of act = bf16(silu(g) * u), fp32 accumulation. */
 MOE_API moe_status_t moe_grouped_gemm_swiglu_mx(const uint8_t *a_q, const uint8_t *a_scales, const int32_t *perm,
@@ -269,8 +274,9 @@ MOE_API moe_status_t moe_grouped_gemm_swiglu_mx(const uint8_t *a_q, const uint8_
                                                 const moe_shape_t *shape, uint8_t *act_q, uint8_t *act_scales,
                                                 moe_stream_t stream);
 
-/* Down with MXFP8 weights: act_q [T*top_k, I] E4M3 + act_scales [T*top_k,
- * I/32], w_d [E,H,I] E4M3 + w_d_scales [E,H,I/32] -> y [T*top_k, H] bf16. */
+/* Down with MXFP8 or MXFP4 weights: act_q [T*top_k, I] E4M3 + act_scales
+ * [T*top_k, I/32], w_d [E,H,I] E4M3 (MXFP4: [E,H,I/2] packed E2M1) +
+ * w_d_scales [E,H,I/32] -> y [T*top_k, H] bf16. */
 MOE_API moe_status_t moe_grouped_gemm_down_mx(const uint8_t *act_q, const uint8_t *act_scales,
                                               const int32_t *offsets, const void *w_d, const void *w_d_scales,
                                               const moe_shape_t *shape, moe_bf16_t *y, moe_stream_t stream);

@@ -26,7 +26,7 @@ __all__ = [
     "moe_finalize", "moe_forward", "moe_forward_host", "moe_dequant_int4",
     "moe_get_device_error", "moe_status_string", "moe_permute_noalloc", "moe_selftest_bounded_wait",
     "moe_forward_kernel_count", "moe_forward_gathers_in_gemm", "forward", "debug_bounds_library",
-    "moe_mx_quantize", "moe_grouped_gemm_swiglu_mx", "moe_grouped_gemm_down_mx", "FMT_MXFP8",
+    "moe_mx_quantize", "moe_grouped_gemm_swiglu_mx", "moe_grouped_gemm_down_mx", "FMT_MXFP8", "FMT_MXFP4",
     "moe_forward_fused", "moe_forward_is_fused",
 ]
 
@@ -36,6 +36,7 @@ library_path = os.path.join(HERE, "libmoe_b200.so")
 FMT_BF16 = 0
 FMT_INT4_G128 = 1
 FMT_MXFP8 = 2
+FMT_MXFP4 = 3
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
           3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_FLAG"}
@@ -58,7 +59,7 @@ class Shape(ctypes.Structure):
     @classmethod
     def of(cls, T, H, I, E, top_k, fmt=FMT_BF16, n_shared=0) -> "Shape":
         if isinstance(fmt, str):
-            fmt = {"bf16": FMT_BF16, "int4_g128": FMT_INT4_G128, "mxfp8": FMT_MXFP8}[fmt]
+            fmt = {"bf16": FMT_BF16, "int4_g128": FMT_INT4_G128, "mxfp8": FMT_MXFP8, "mxfp4": FMT_MXFP4}[fmt]
         return cls(int(T), int(H), int(I), int(E), int(top_k), int(fmt), int(n_shared))
 
     @property
@@ -332,16 +333,19 @@ def forward(hidden: torch.Tensor, logits: torch.Tensor, w_gu: torch.Tensor, w_d:
             out: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """moe_forward on device tensors; allocates out and the workspace with
     torch when they are not given. hidden [T,H] bf16, logits [T,E] fp32,
-    w_gu [E+S,2I,H] bf16 (or uint8 [E+S,2I,H/2] + scales), w_d [E+S,H,I] (or
-    uint8): weight arrays with more experts than logits columns hold S shared
-    experts after the E routed ones."""
+    w_gu [E+S,2I,H] bf16 (or uint8: int4 [E+S,2I,H/2] with bf16 scales, MXFP8
+    [E+S,2I,H] or MXFP4 [E+S,2I,H/2] with uint8 scales), w_d likewise:
+    weight arrays with more experts than logits columns hold S shared experts
+    after the E routed ones."""
     T, H = hidden.shape
     E = logits.shape[1]
     if w_gu.dtype != torch.uint8:
         fmt = FMT_BF16
+    elif w_gu_scales is None or w_gu_scales.dtype != torch.uint8:
+        fmt = FMT_INT4_G128
     else:
-        fmt = FMT_MXFP8 if (w_gu_scales is not None and w_gu_scales.dtype == torch.uint8) else FMT_INT4_G128
-    I = w_d.shape[2] * (2 if fmt == FMT_INT4_G128 else 1)
+        fmt = FMT_MXFP4 if w_gu.shape[2] * 2 == H else FMT_MXFP8
+    I = w_d.shape[2] * (2 if fmt in (FMT_INT4_G128, FMT_MXFP4) else 1)
     shape = Shape.of(T, H, I, E, top_k, fmt, n_shared=w_gu.shape[0] - E)
     if out is None:
         out = torch.empty(T, H, dtype=torch.bfloat16, device=hidden.device)

@@ -40,12 +40,15 @@ inline bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintp
 // Slots per token (routed, then shared) and experts in the weight arrays.
 inline int slots(const moe_shape_t *s) { return s->top_k + s->n_shared; }
 inline int experts(const moe_shape_t *s) { return s->E + s->n_shared; }
+// Block-scaled formats: MX weights, MXFP8 activations.
+inline bool is_mx(int fmt) { return fmt == MOE_W_MXFP8 || fmt == MOE_W_MXFP4; }
 
 moe_status_t check_shape(const moe_shape_t *s) {
     if (!s) return MOE_ERR_INVALID_ARG;
     if (s->T < 0 || s->H <= 0 || s->I <= 0 || s->E < 1 || s->top_k < 1 || s->top_k > s->E || s->n_shared < 0)
         return MOE_ERR_INVALID_ARG;
-    if (s->fmt != MOE_W_BF16 && s->fmt != MOE_W_INT4_G128 && s->fmt != MOE_W_MXFP8) return MOE_ERR_INVALID_ARG;
+    if (s->fmt != MOE_W_BF16 && s->fmt != MOE_W_INT4_G128 && s->fmt != MOE_W_MXFP8 && s->fmt != MOE_W_MXFP4)
+        return MOE_ERR_INVALID_ARG;
     if (static_cast<long long>(s->E) + s->n_shared > 1024 || static_cast<long long>(s->top_k) + s->n_shared > 32)
         return MOE_ERR_UNSUPPORTED;
     if (s->H % 8 || s->I % 8) return MOE_ERR_UNSUPPORTED;
@@ -64,7 +67,7 @@ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // Byte offsets of moe_forward's intermediates inside the workspace.
 struct Layout {
     size_t ids, w, counts, offsets, perm, inv, scratch, hperm, act, y;
-    size_t hq, hs, aq, as;                 // MXFP8: hidden and act, E4M3 codes and E8M0 scales
+    size_t hq, hs, aq, as;                 // MX formats: hidden and act, E4M3 codes and E8M0 scales
     size_t done;                           // moe_forward_fused: per-expert and finish counters
     size_t hidden_in, logits_in, out_st;   // staging for moe_forward_host
     size_t total;
@@ -88,7 +91,7 @@ Layout layout(const moe_shape_t *s, bool host) {
     L.inv = take(P * 4);
     L.scratch = take(moe::permute_scratch_bytes(static_cast<long long>(P), E));
     L.hperm = moe::gemm_gathers_in_kernel(static_cast<int>(P), E, s->fmt) ? o : take(P * s->H * 2);
-    const bool mx = s->fmt == MOE_W_MXFP8;
+    const bool mx = is_mx(s->fmt);
     L.act = mx ? o : take(P * s->I * 2);
     L.y = take(P * s->H * 2);
     L.hq = L.hs = L.aq = L.as = o;
@@ -132,7 +135,8 @@ moe::GemmArgs gemm_args(const moe_shape_t *s, const void *a, const int32_t *perm
 }
 
 moe_status_t check_weights(const moe_shape_t *s, const void *w, const void *scales) {
-    if (!w || !aligned(w, 16)) return MOE_ERR_INVALID_ARG;
+    // MXFP4 weights are read by TMA as packed 4-bit elements: 32-byte aligned
+    if (!w || !aligned(w, s->fmt == MOE_W_MXFP4 ? 32 : 16)) return MOE_ERR_INVALID_ARG;
     if (s->fmt != MOE_W_BF16) {
         if (!scales || !aligned(scales, 4)) return MOE_ERR_INVALID_ARG;
     } else if (scales) {
@@ -188,8 +192,8 @@ moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const
             cudaSuccess)
             return cuda_status(e);
     }
-    if (s->fmt == MOE_W_MXFP8) {
-        // MXFP8: hidden quantised once per token; gate/up gathers its rows through
+    if (is_mx(s->fmt)) {
+        // MX weights: hidden quantised once per token; gate/up gathers its rows through
         // perm and writes act quantised; down reads act's codes and scales
         auto *hq = ws + L.hq, *hs = ws + L.hs, *aq = ws + L.aq, *as = ws + L.as;
         if ((e = moe::launch_mx_quantize(hidden, T, H, hq, hs, st)) != cudaSuccess) return cuda_status(e);
@@ -295,7 +299,7 @@ moe_status_t moe_grouped_gemm_swiglu(const moe_bf16_t *a, const int32_t *perm, c
     const moe::NvtxRange nvtx("moe_grouped_gemm_swiglu");
     moe_status_t st = check_shape(shape);
     if (st != MOE_OK) return st;
-    if (shape->fmt == MOE_W_MXFP8) return MOE_ERR_UNSUPPORTED;     // moe_grouped_gemm_swiglu_mx
+    if (is_mx(shape->fmt)) return MOE_ERR_UNSUPPORTED;             // moe_grouped_gemm_swiglu_mx
     if (shape->T == 0) return MOE_OK;
     if (!a || !offsets || !act || !aligned(a, 16) || !aligned(act, 16) || !aligned(offsets, 4))
         return MOE_ERR_INVALID_ARG;
@@ -311,7 +315,7 @@ moe_status_t moe_grouped_gemm_down(const moe_bf16_t *act, const int32_t *offsets
     const moe::NvtxRange nvtx("moe_grouped_gemm_down");
     moe_status_t st = check_shape(shape);
     if (st != MOE_OK) return st;
-    if (shape->fmt == MOE_W_MXFP8) return MOE_ERR_UNSUPPORTED;     // moe_grouped_gemm_down_mx
+    if (is_mx(shape->fmt)) return MOE_ERR_UNSUPPORTED;             // moe_grouped_gemm_down_mx
     if (shape->T == 0) return MOE_OK;
     if (!act || !offsets || !y || !aligned(act, 16) || !aligned(y, 16) || !aligned(offsets, 4))
         return MOE_ERR_INVALID_ARG;
@@ -345,7 +349,7 @@ int32_t moe_forward_kernel_count(const moe_shape_t *shape) {
     else
         n += 1 + moe::permute_kernel_count(P, E);                     // route; permute in 1, 2 or 3 kernels
     if (!moe::gemm_gathers_in_kernel(static_cast<int>(P), E, shape->fmt)) n += 1;   // gather
-    if (shape->fmt == MOE_W_MXFP8) n += 1;                            // MX quantisation of hidden
+    if (is_mx(shape->fmt)) n += 1;                                    // MX quantisation of hidden
     return n + 3;                                                     // gate/up, down, finalize
 }
 
@@ -456,7 +460,7 @@ moe_status_t moe_grouped_gemm_swiglu_mx(const uint8_t *a_q, const uint8_t *a_sca
     const moe::NvtxRange nvtx("moe_grouped_gemm_swiglu_mx");
     moe_status_t st = check_shape(shape);
     if (st != MOE_OK) return st;
-    if (shape->fmt != MOE_W_MXFP8) return MOE_ERR_INVALID_ARG;
+    if (!is_mx(shape->fmt)) return MOE_ERR_INVALID_ARG;
     if (shape->T == 0) return MOE_OK;
     if (!a_q || !a_scales || !offsets || !act_q || !act_scales || !aligned(a_q, 16) || !aligned(a_scales, 4) ||
         !aligned(act_q, 16) || !aligned(offsets, 4))
@@ -474,7 +478,7 @@ moe_status_t moe_grouped_gemm_down_mx(const uint8_t *act_q, const uint8_t *act_s
     const moe::NvtxRange nvtx("moe_grouped_gemm_down_mx");
     moe_status_t st = check_shape(shape);
     if (st != MOE_OK) return st;
-    if (shape->fmt != MOE_W_MXFP8) return MOE_ERR_INVALID_ARG;
+    if (!is_mx(shape->fmt)) return MOE_ERR_INVALID_ARG;
     if (shape->T == 0) return MOE_OK;
     if (!act_q || !act_scales || !offsets || !y || !aligned(act_q, 16) || !aligned(act_scales, 4) ||
         !aligned(y, 16) || !aligned(offsets, 4))

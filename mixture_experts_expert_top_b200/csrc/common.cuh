@@ -409,12 +409,17 @@ __device__ __forceinline__ uint64_t sf_smem_desc(uint32_t smem_addr) {
     return d;
 }
 
-// Instruction descriptor of kind::mxf8f6f4 with block scaling: E4M3 A and B
-// (K-major), E8M0 scale factors, fp32 D, shape M x N; sf ids select the byte
-// of each 32-bit TMEM scale-factor word (the K block of 32 within 128).
-__host__ __device__ __forceinline__ uint32_t idesc_mxf8_e4m3(int M, int N, uint32_t a_sf_id, uint32_t b_sf_id) {
+// Operand formats of kind::mxf8f6f4 (instruction descriptor codes).
+constexpr uint32_t kMxE4M3 = 0, kMxE2M1 = 5;
+
+// Instruction descriptor of kind::mxf8f6f4 with block scaling: A of format
+// a_fmt (E4M3, or E2M1 for MXFP4 weights) and E4M3 B, both K-major, E8M0
+// scale factors, fp32 D, shape M x N; sf ids select the byte of each 32-bit
+// TMEM scale-factor word (the K block of 32 within 128).
+__host__ __device__ __forceinline__ uint32_t idesc_mxf8f6f4(int M, int N, uint32_t a_fmt, uint32_t a_sf_id,
+                                                            uint32_t b_sf_id) {
     return (b_sf_id << 4)                                   // B scale factor id
-           | (0u << 7) | (0u << 10)                         // A, B format: E4M3
+           | (a_fmt << 7) | (kMxE4M3 << 10)                 // A, B format
            | (static_cast<uint32_t>(N >> 3) << 17)          // N >> 3
            | (1u << 23)                                     // scale format: E8M0
            | (static_cast<uint32_t>(M >> 4) << 24)          // M >> 4

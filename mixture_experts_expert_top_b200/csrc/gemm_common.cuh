@@ -204,6 +204,20 @@ inline bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, i
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The same with an explicit row pitch in bytes (for packed 4-bit elements,
+// whose rows are cols / 2 bytes).
+inline bool make_map_pitched(CUtensorMap *m, const void *base, CUtensorMapDataType dt, uint64_t cols, uint64_t rows,
+                             uint64_t row_bytes, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {row_bytes};
+    cuuint32_t box[2] = {box_cols, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // Tensor map of the token operand: a [rows, K] bf16 with the 128-byte
 // swizzle; a box of box_rows rows, or of one row for gather4 loads.
 inline bool make_token_map(CUtensorMap *m, const GemmArgs &g, uint32_t box_rows) {

@@ -693,7 +693,7 @@ bool gemm_gathers_in_kernel(int P, int E, int fmt) { return !uses_prefill_kernel
 
 cudaError_t launch_grouped_gemm(const GemmArgs &g, cudaStream_t s) {
     if (g.P == 0) return cudaSuccess;
-    if (g.fmt == 2) return cudaErrorInvalidValue;      // MXFP8: launch_grouped_gemm_mxfp8
+    if (g.fmt >= 2) return cudaErrorInvalidValue;      // MX formats: launch_grouped_gemm_mxfp8
     if (g.fmt == 0) {
         // many tokens per expert: weights on M across CTA pairs (gemm_wm_pair_sm100.cu)
         if (uses_prefill_kernel(g.P, g.E, g.fmt)) return launch_grouped_gemm_prefill(g, s);

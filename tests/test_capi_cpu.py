@@ -146,11 +146,13 @@ def test_forward_kernel_count():
     assert count(moe_synth.get_config("tiny")) == 2
     assert count(moe_synth.get_config("shared_decode")) == 2
     assert count(moe_synth.get_config("mxfp8_decode")) == 5
+    assert count(moe_synth.get_config("mxfp4_decode")) == 5
     assert count(moe_synth.get_config("qwen3_decode", T=65)) == 5            # past the persistent kernel's batch
     assert count(moe_synth.get_config("w4a16_decode")) == 5
     fused = lambda c: moe.moe_forward_is_fused(sh(c))
     assert fused(moe_synth.get_config("qwen3_decode")) and fused(moe_synth.get_config("shared_decode"))
     assert not fused(moe_synth.get_config("w4a16_decode")) and not fused(moe_synth.get_config("mxfp8_decode"))
+    assert not fused(moe_synth.get_config("mxfp4_decode"))
     assert not fused(moe_synth.get_config("qwen3_prefill"))
     assert not fused(moe_synth.get_config("qwen3_decode", E=300))                # more experts than it takes
     assert count(moe_synth.get_config("qwen3_prefill")) == 7

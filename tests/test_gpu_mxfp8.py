@@ -1,4 +1,5 @@
-"""MXFP8 weights (OCP MX v1.0: E4M3 + one E8M0 scale per 32 K) on the
+"""MXFP8 weights (OCP MX v1.0: E4M3 + one E8M0 scale per 32 K) and MXFP4
+weights (E2M1 + one E8M0 scale per 32 K, with MXFP8 activations) on the
 block-scaled tensor-core MMA, against the CPU oracle through the C ABI.
 
 Bit-exact: the MX quantisation of the activations. Within tolerance: the
@@ -58,11 +59,11 @@ def test_mx_quantize_is_bit_exact(rows, K):
     assert np.array_equal(gq, oq)
 
 
-MX_GEMM = [
-    moe_synth.MoeConfig("mx_bn32", T=48, H=1024, I=384, E=12, k=4, fmt="mxfp8"),      # 16 rows per expert
-    moe_synth.MoeConfig("mx_bn64", T=96, H=1024, I=384, E=24, k=8, fmt="mxfp8"),      # 32 rows per expert
-    moe_synth.MoeConfig("mx_bn128", T=256, H=512, I=256, E=16, k=4, fmt="mxfp8"),     # 64 rows per expert
-]
+MX_GEMM = [moe_synth.MoeConfig(f"{name}_{fmt}", T=T, H=H, I=I, E=E, k=k, fmt=fmt)
+           for fmt in ("mxfp8", "mxfp4")
+           for name, T, H, I, E, k in (("mx_bn32", 48, 1024, 384, 12, 4),     # 16 rows per expert
+                                       ("mx_bn64", 96, 1024, 384, 24, 8),     # 32 rows per expert
+                                       ("mx_bn128", 256, 512, 256, 16, 4))]   # 64 rows per expert
 
 
 def _e4m3_step(v):
@@ -75,9 +76,9 @@ def _e4m3_step(v):
 @pytest.mark.parametrize("gather", [False, True], ids=["rows", "perm"])
 def test_mx_grouped_gemms_match_oracle(cfg, gather):
     inp = moe_synth.gen_inputs(cfg, seed=41)
-    r = oracle.forward(inp, cfg.k, fmt="mxfp8")
+    r = oracle.forward(inp, cfg.k, fmt=cfg.fmt)
     P = cfg.P
-    sh = moe.Shape.of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, "mxfp8")
+    sh = moe.Shape.of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.fmt)
     offsets = dev(r["offsets"])
     if gather:      # hidden quantised once per token, rows read through perm
         xq, xs = oracle.mx_quantize(inp["hidden"])
@@ -108,16 +109,16 @@ def test_mx_grouped_gemms_match_oracle(cfg, gather):
                   + 1e-30), float(diff.max())
 
 
-MX_LAYERS = [moe_synth.MoeConfig("mxfp8_decode", T=64, H=2048, I=768, E=128, k=8, fmt="mxfp8"),
-             moe_synth.MoeConfig("mxfp8_prefill", T=1024, H=2048, I=768, E=128, k=8, fmt="mxfp8",
-                                 logit_extra="bias0.5")]
+MX_LAYERS = [moe_synth.MoeConfig(f"{fmt}_{kind}", T=T, H=2048, I=768, E=128, k=8, fmt=fmt, logit_extra=extra)
+             for fmt in ("mxfp8", "mxfp4")
+             for kind, T, extra in (("decode", 64, "none"), ("prefill", 1024, "bias0.5"))]
 
 
 @pytest.mark.parametrize("cfg", MX_LAYERS, ids=lambda c: c.name)
 def test_mx_layer_matches_oracle(cfg):
     inp = moe_synth.gen_inputs(cfg, seed=0)
     d = {n: t.to(DEV) for n, t in inp.items()}
-    sh = moe.Shape.of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, "mxfp8")
+    sh = moe.Shape.of(cfg.T, cfg.H, cfg.I, cfg.E, cfg.k, cfg.fmt)
     ws = torch.empty(moe.moe_workspace_size(sh), dtype=torch.uint8, device=DEV)
     out = torch.empty(cfg.T, cfg.H, dtype=torch.bfloat16, device=DEV)
     moe.moe_forward(d["hidden"], d["logits"], d["w_gu"], d["w_gu_scales"], d["w_d"], d["w_d_scales"], sh, out, ws)
@@ -125,7 +126,7 @@ def test_mx_layer_matches_oracle(cfg):
     moe.moe_forward(d["hidden"], d["logits"], d["w_gu"], d["w_gu_scales"], d["w_d"], d["w_d_scales"], sh, out2, ws)
     torch.cuda.synchronize()
     assert torch.equal(out.view(torch.int16), out2.view(torch.int16))        # deterministic
-    r = oracle.forward(inp, cfg.k, fmt="mxfp8")
+    r = oracle.forward(inp, cfg.k, fmt=cfg.fmt)
     y_abs = weighted_abs_y(r["y"], r["w"], r["inv_perm"], cfg.T, cfg.H, cfg.k)
     layer_output_close(bf16_bits(out), r["out"], cfg.name, y_abs=y_abs)
     assert moe.moe_forward_kernel_count(sh) == (5 if cfg.T <= 64 else 6)
