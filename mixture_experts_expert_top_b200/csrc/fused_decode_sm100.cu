@@ -61,7 +61,6 @@ constexpr int kFAccCols = 2 * kFBN;                         // per TMEM buffer: 
 constexpr int kFTmemCols = 2 * kFAccCols;
 constexpr int kFQueue = 8;                                  // tile numbers in flight between the roles
 constexpr int kFPrefetchKB = 6;                             // K-blocks prefetched to L2 before routing
-constexpr int kFL2Ahead = 8;                                // weight stages prefetched to L2 ahead of the ring
 constexpr unsigned long long kFDepLimitNs = 2000000000ull;
 
 struct FusedArgs {
@@ -364,36 +363,6 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap tmWgu, const __grid_cons
             if (lane == 0) next = atomicAdd(a.next_tile, 1u);
             const FTile ft = fused_tile(tile, tc, fs, MB_gu, MB_dn, a.H);
             const int nbox = ft.n_mma / kBoxN;
-            // L2 prefetch of the weights kFL2Ahead stages ahead of the ring (this
-            // tile's later stages, then the next tile's first ones): the ring
-            // alone keeps too few bytes in flight for HBM's latency under load
-            bool next_known = false, next_valid = false;
-            FTile nft = ft;
-            auto prefetch_stage = [&](const FTile &f, int j) {
-                if (f.gu) {
-                    const int r = f.e * 2 * a.I + f.mb * kBM;
-                    tma_prefetch_l2_2d(&tmWgu, j * kBK, r);
-                    tma_prefetch_l2_2d(&tmWgu, j * kBK, r + a.I);
-                } else {
-                    const int r = f.e * a.H + f.mb * 2 * kBM + f.h0 * kBM;
-                    tma_prefetch_l2_2d(&tmWd, j * kBK, r);
-                    if (f.two) tma_prefetch_l2_2d(&tmWd, j * kBK, r + kBM);
-                }
-            };
-            auto lookahead = [&](int kb) {          // lane 0, at stage kb of this tile
-                const int kbc = ft.gu ? KB_gu : KB_dn;
-                const int t = kb + kFL2Ahead;
-                if (t < kbc) {
-                    prefetch_stage(ft, t);
-                    return;
-                }
-                if (!next_known) {
-                    next_known = true;
-                    next_valid = static_cast<int>(next) < total_tiles;
-                    if (next_valid) nft = fused_tile(static_cast<int>(next), tc, fs, MB_gu, MB_dn, a.H);
-                }
-                if (next_valid && t - kbc < (nft.gu ? KB_gu : KB_dn)) prefetch_stage(nft, t - kbc);
-            };
             if (ft.gu) {
                 const int row = ft.e * 2 * a.I + ft.mb * kBM;
                 const uint32_t tx = 2 * kTileBytesA + nbox * kBoxBytesB;
@@ -404,7 +373,6 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap tmWgu, const __grid_cons
                     for (int j = 0; j < 4; ++j) tr[j] = token_of(ft.row0 + 4 * lane + j);
                 }
                 for (int kb = 0; kb < KB_gu; ++kb) {
-                    if (lane == 0) lookahead(kb);
                     if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, a.err, 0);
                     ok = __shfl_sync(0xffffffffu, ok, 0);
                     if (!ok) break;
@@ -428,7 +396,6 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap tmWgu, const __grid_cons
                 const int stage0 = stage;
                 for (int kb = 0; kb < pre && ok; ++kb) {
                     if (lane == 0) {
-                        lookahead(kb);
                         ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, a.err, 0);
                         if (ok) {
                             uint8_t *st = ring + stage * kFSlot;
@@ -457,7 +424,6 @@ fused_decode_kernel(const __grid_constant__ CUtensorMap tmWgu, const __grid_cons
                 }
                 for (int kb = pre; kb < KB_dn && ok; ++kb) {
                     if (lane == 0) {
-                        lookahead(kb);
                         ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, a.err, 0);
                         if (ok) {
                             uint8_t *st = ring + stage * kFSlot;

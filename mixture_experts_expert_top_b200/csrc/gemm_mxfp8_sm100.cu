@@ -45,7 +45,6 @@ using namespace gemm;
 constexpr int kMxBK = 128;                      // K elements (bytes) per stage and operand row
 constexpr int kMxTileA = kBM * kMxBK;           // 16 KB
 constexpr int kSfBlock = 512;                   // scale factors of 128 rows x 4 K blocks
-constexpr int kMxL2Ahead = 8;                   // weight stages prefetched into L2 ahead of the ring
 
 // E4M3 code of x (round to nearest even, saturate to +-448).
 __device__ __forceinline__ uint8_t e4m3_rn_sat(float x) {
@@ -196,143 +195,79 @@ grouped_gemm_mxfp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_
         // Lane 0 runs the ring and the TMA loads (with perm, lanes i < N/4 issue
         // the token rows as gather4 loads); every lane writes the scale factors
         // of 4 weight rows (and 4 token rows) into the stage's 512-byte blocks.
-        // The scale factors of the next stage are loaded from global memory
-        // while this stage is filled, so that their round trip overlaps the
-        // wait for a free ring slot instead of adding to every stage.
         const uint64_t pol_w = p.evict_first_weights ? l2_policy_evict_first() : l2_policy_evict_last();
         const uint64_t pol_x = l2_policy_evict_last();
-        struct TileSf {
-            TileInfo ti;
-            int a_row;
-            int sf_tok[4];      // token rows of this lane's scale factors: n = lane + 32 i (-1: none)
-        };
-        auto setup = [&](int tile, TileSf &t) {
-            t.ti = decode_tile(tile, pre_s, off_s, E, MB, BN);
-            t.a_row = t.ti.e * p.w_rows + t.ti.mb * kBM;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int n = lane + 32 * i;
-                t.sf_tok[i] = (n < BN && n < t.ti.n_mma) ? token_row(p, t.ti.row0 + n) : -1;
-                if (t.sf_tok[i] >= mp.x_rows) t.sf_tok[i] = -1;
-            }
-        };
-        // scale factors of K block kb: weight rows m = lane + 32 i (gate, then up), then token rows
-        auto load_sf = [&](const TileSf &t, int kb, uint32_t (&wa)[2][4], uint32_t (&wb)[4]) {
-#pragma unroll
-            for (int a = 0; a < C::kNumA; ++a) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int row = t.a_row + (a ? p.m_out : 0) + lane + 32 * i;
-                    wa[a][i] = row < mp.w_total_rows
-                                   ? __ldg(reinterpret_cast<const uint32_t *>(mp.w_sf + static_cast<size_t>(row) *
-                                                                                         sf_row_bytes) + kb)
-                                   : 0u;
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                wb[i] = t.sf_tok[i] >= 0
-                            ? __ldg(reinterpret_cast<const uint32_t *>(mp.x_sf + static_cast<size_t>(t.sf_tok[i]) *
-                                                                      sf_row_bytes) + kb)
-                            : 0u;
-        };
         int stage = 0;
         uint32_t phase = 0;
         bool ok = true;
-        // the position after the current one (tile, K block) and its scale factors
-        int n_tile = blockIdx.x, n_kb = 0;
-        TileSf nt;
-        uint32_t n_wa[2][4] = {}, n_wb[4] = {};
-        if (n_tile < total_tiles) {
-            setup(n_tile, nt);
-            load_sf(nt, 0, n_wa, n_wb);
-        }
-        // L2 prefetch of the weight tiles kMxL2Ahead stages ahead: the ring
-        // holds only a few stages, and at decode every stage's load waits
-        // several microseconds for HBM under load, so the ring alone keeps
-        // too few bytes in flight; the prefetches keep HBM busy and the ring's
-        // loads then find their tiles in L2.
-        int p_tile = blockIdx.x, p_kb = 0, p_row = 0;
-        if (p_tile < total_tiles) {
-            const TileInfo pt = decode_tile(p_tile, pre_s, off_s, E, MB, BN);
-            p_row = pt.e * p.w_rows + pt.mb * kBM;
-        }
-        auto prefetch_next = [&]() {
-            if (p_tile >= total_tiles) return;
-            if (lane == 0) {
-                tma_prefetch_l2_2d(&tmA, p_kb * kMxBK, p_row);
-                if (SWIGLU) tma_prefetch_l2_2d(&tmA, p_kb * kMxBK, p_row + p.m_out);
-            }
-            if (++p_kb == KB) {
-                p_kb = 0;
-                p_tile += gridDim.x;
-                if (p_tile < total_tiles) {
-                    const TileInfo pt = decode_tile(p_tile, pre_s, off_s, E, MB, BN);
-                    p_row = pt.e * p.w_rows + pt.mb * kBM;
-                }
-            }
-        };
-        for (int d = 0; d < kMxL2Ahead; ++d) prefetch_next();
-        TileSf ct;
-        int tr[4] = {0, 0, 0, 0};
-        bool gather_lane = false;
-        while (n_tile < total_tiles && ok) {
-            prefetch_next();
-            // this position
-            const int kb = n_kb;
-            if (kb == 0) {
-                ct = nt;
-                gather_lane = p.perm && 4 * lane < ct.ti.n_mma;
-                if (gather_lane) {
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) tr[j] = token_row(p, ct.ti.row0 + 4 * lane + j);
-                }
-            }
-            uint32_t wa[2][4], wb[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                wa[0][i] = n_wa[0][i];
-                wa[1][i] = n_wa[1][i];
-                wb[i] = n_wb[i];
-            }
-            // the next position: its scale factors are in flight while this stage fills
-            if (++n_kb == KB) {
-                n_kb = 0;
-                n_tile += gridDim.x;
-                if (n_tile < total_tiles) setup(n_tile, nt);
-            }
-            if (n_tile < total_tiles) load_sf(nt, n_kb, n_wa, n_wb);
-            const int nbox = ct.ti.n_mma / kBoxN;
+        for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+            const TileInfo ti = decode_tile(tile, pre_s, off_s, E, MB, BN);
+            const int nbox = ti.n_mma / kBoxN;
+            const int a_row = ti.e * p.w_rows + ti.mb * kBM;
             // a 4-bit weight tile moves (and counts) 8 bytes per 16 elements
             const uint32_t tx = (W4 ? C::kABytes / 2 : C::kABytes) + nbox * kBoxN * kMxBK;
-            if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.err, 0);
-            ok = __shfl_sync(0xffffffffu, ok, 0);
-            if (!ok) break;
-            uint8_t *st = ring + stage * C::kStageBytes;
-            uint8_t *sb = st + C::kABytes;
-            uint8_t *sf = sb + C::kBBytes;
+            const bool gather_lane = p.perm && 4 * lane < ti.n_mma;
+            int tr[4] = {0, 0, 0, 0};
+            if (gather_lane) {
 #pragma unroll
-            for (int a = 0; a < C::kNumA; ++a)
-                *reinterpret_cast<uint4 *>(sf + a * kSfBlock + lane * 16) =
-                    make_uint4(wa[a][0], wa[a][1], wa[a][2], wa[a][3]);
-            *reinterpret_cast<uint4 *>(sf + C::kNumA * kSfBlock + lane * 16) = make_uint4(wb[0], wb[1], wb[2], wb[3]);
-            fence_proxy_async_smem();            // the tcgen05.cp of these bytes is an async-proxy read
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive_expect_tx(&full_bar[stage], tx);
-                tma_load_2d(st, &tmA, &full_bar[stage], kb * kMxBK, ct.a_row, pol_w);
-                if (SWIGLU)
-                    tma_load_2d(st + kMxTileA, &tmA, &full_bar[stage], kb * kMxBK, ct.a_row + p.m_out, pol_w);
-                if (!p.perm)
-                    for (int b = 0; b < nbox; ++b)
-                        tma_load_2d(sb + b * kBoxN * kMxBK, &tmB, &full_bar[stage], kb * kMxBK,
-                                    ct.ti.row0 + b * kBoxN, pol_x);
+                for (int j = 0; j < 4; ++j) tr[j] = token_row(p, ti.row0 + 4 * lane + j);
             }
-            __syncwarp();
-            if (gather_lane)
-                tma_gather4(sb + lane * 4 * kMxBK, &tmB, &full_bar[stage], kb * kMxBK, tr[0], tr[1], tr[2], tr[3],
-                            pol_x);
-            if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            // token rows of this lane's scale factors: n = lane + 32 i
+            int sf_tok[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int n = lane + 32 * i;
+                sf_tok[i] = (n < BN && n < ti.n_mma) ? token_row(p, ti.row0 + n) : -1;
+                if (sf_tok[i] >= mp.x_rows) sf_tok[i] = -1;
+            }
+            for (int kb = 0; kb < KB; ++kb) {
+                if (lane == 0) ok = mbar_wait(&empty_bar[stage], phase ^ 1, abort_flag, p.err, 0);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                uint8_t *st = ring + stage * C::kStageBytes;
+                uint8_t *sb = st + C::kABytes;
+                uint8_t *sf = sb + C::kBBytes;
+                // scale factors: weight rows m = lane + 32 i (gate, then up), then token rows
+                for (int a = 0; a < C::kNumA; ++a) {
+                    uint32_t v[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int row = a_row + (a ? p.m_out : 0) + lane + 32 * i;
+                        v[i] = row < mp.w_total_rows
+                                   ? __ldg(reinterpret_cast<const uint32_t *>(mp.w_sf + static_cast<size_t>(row) *
+                                                                                         sf_row_bytes) + kb)
+                                   : 0u;
+                    }
+                    *reinterpret_cast<uint4 *>(sf + a * kSfBlock + lane * 16) = make_uint4(v[0], v[1], v[2], v[3]);
+                }
+                {
+                    uint32_t v[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        v[i] = sf_tok[i] >= 0
+                                   ? __ldg(reinterpret_cast<const uint32_t *>(mp.x_sf + static_cast<size_t>(sf_tok[i]) *
+                                                                                         sf_row_bytes) + kb)
+                                   : 0u;
+                    *reinterpret_cast<uint4 *>(sf + C::kNumA * kSfBlock + lane * 16) =
+                        make_uint4(v[0], v[1], v[2], v[3]);
+                }
+                fence_proxy_async_smem();            // the tcgen05.cp of these bytes is an async-proxy read
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&full_bar[stage], tx);
+                    tma_load_2d(st, &tmA, &full_bar[stage], kb * kMxBK, a_row, pol_w);
+                    if (SWIGLU) tma_load_2d(st + kMxTileA, &tmA, &full_bar[stage], kb * kMxBK, a_row + p.m_out, pol_w);
+                    if (!p.perm)
+                        for (int b = 0; b < nbox; ++b)
+                            tma_load_2d(sb + b * kBoxN * kMxBK, &tmB, &full_bar[stage], kb * kMxBK,
+                                        ti.row0 + b * kBoxN, pol_x);
+                }
+                __syncwarp();
+                if (gather_lane)
+                    tma_gather4(sb + lane * 4 * kMxBK, &tmB, &full_bar[stage], kb * kMxBK, tr[0], tr[1], tr[2], tr[3],
+                                pol_x);
+                if (++stage == STAGES) { stage = 0; phase ^= 1; }
+            }
         }
     } else if (warp == 1) {
         // ================================ MMA issuer ============================
