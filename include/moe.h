@@ -333,6 +333,64 @@ MOE_API moe_status_t moe_permute_noalloc(const int32_t *topk_ids, const moe_shap
                                          const moe_bf16_t *hidden, moe_bf16_t *hidden_perm,
                                          moe_stream_t stream);
 
+/* ---- Expert parallelism ------------------------------------------------------
+ * The experts split over `world` ranks (rank d owns experts d*E/world ..
+ * (d+1)*E/world - 1, and their weights), each rank holding its own tokens
+ * (GC-MoE abstract: experts partitioned over GPUs, tokens dispatched to their
+ * experts' GPU and the outputs combined back). The steps write straight into
+ * other ranks' buffers through the pointers of moe_ep_peers_t: buffers of the
+ * same GPU, or of peer GPUs with peer access enabled (the stores then cross
+ * NVLink). No kernel waits for another rank; between the phases the caller
+ * puts a barrier over all ranks (marked | below). On each rank r, with
+ * shape = {T_r tokens, H, I, E all routed experts, top_k, fmt, n_shared 0}:
+ *   moe_route, moe_permute (counts, offsets, perm, inv_perm over all E)
+ *   moe_ep_count                          |
+ *   moe_ep_dispatch                       |
+ *   moe_ep_local_offsets, then moe_grouped_gemm_swiglu and _down on
+ *     recv_rows[r] (perm NULL, the local offsets, the E/world local experts'
+ *     weights, a shape with E = E/world and T*top_k >= the rows received)
+ *   moe_ep_combine                        |
+ *   moe_finalize(y_ret[r], topk_w, identity inv_perm) -> out.
+ * Every pair's arithmetic is moe_forward's on rank r's own tokens; the
+ * result equals it bit for bit.
+ * Receive buffer of rank d: rows grouped by d's local expert, then by source
+ * rank, then in the source's permutation order; recv_src holds each row's
+ * origin as (source rank << 24) | pair id. */
+#define MOE_EP_MAX_RANKS 8
+typedef struct {
+    int32_t world;                                /* ranks, 1 .. MOE_EP_MAX_RANKS */
+    int32_t rank;                                 /* this rank */
+    int32_t capacity;                             /* rows of every receive buffer */
+    int32_t *counts[MOE_EP_MAX_RANKS];            /* rank d: [world, E/world] int32: row s = pairs of
+                                                     source s per local expert */
+    moe_bf16_t *recv_rows[MOE_EP_MAX_RANKS];      /* rank d: [capacity, H] bf16, 16-byte aligned */
+    int32_t *recv_src[MOE_EP_MAX_RANKS];          /* rank d: [capacity] origins */
+    moe_bf16_t *y_ret[MOE_EP_MAX_RANKS];          /* rank r: [T_r*top_k, H] bf16: the down output of
+                                                     each of r's pairs, at its pair id */
+    int32_t pairs[MOE_EP_MAX_RANKS];              /* rank r: T_r*top_k, the rows of y_ret[r] */
+} moe_ep_peers_t;
+
+/* This rank's pairs per expert (from its offsets [E+1]) into row `rank` of
+ * every owner's counts. */
+MOE_API moe_status_t moe_ep_count(const int32_t *offsets, const moe_shape_t *shape, const moe_ep_peers_t *peers,
+                                  moe_stream_t stream);
+/* After every rank's count: this rank's permuted rows (hidden [T,H] through
+ * perm [T*top_k], offsets [E+1]) into their owners' receive buffers. A row
+ * past `capacity` is not written and raises device error 4. */
+MOE_API moe_status_t moe_ep_dispatch(const moe_bf16_t *hidden, const int32_t *perm, const int32_t *offsets,
+                                     const moe_shape_t *shape, const moe_ep_peers_t *peers, moe_stream_t stream);
+/* After every rank's dispatch: offsets_local [E/world + 1] of this rank's
+ * receive buffer over its local experts (offsets_local[E/world] = rows
+ * received). */
+MOE_API moe_status_t moe_ep_local_offsets(const moe_shape_t *shape, const moe_ep_peers_t *peers,
+                                          int32_t *offsets_local, moe_stream_t stream);
+/* After the local GEMMs: y_local [capacity, H] (the down output of this
+ * rank's received rows) back to each row's source, into y_ret[source] at the
+ * row's pair id (a pair id at or past pairs[source] raises device error 4 and
+ * is skipped). */
+MOE_API moe_status_t moe_ep_combine(const moe_bf16_t *y_local, const int32_t *offsets_local,
+                                    const moe_shape_t *shape, const moe_ep_peers_t *peers, moe_stream_t stream);
+
 /* Static description of a status code. */
 MOE_API const char *moe_status_string(moe_status_t status);
 

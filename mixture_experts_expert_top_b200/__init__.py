@@ -28,6 +28,8 @@ __all__ = [
     "moe_forward_kernel_count", "moe_forward_gathers_in_gemm", "forward", "debug_bounds_library",
     "moe_mx_quantize", "moe_grouped_gemm_swiglu_mx", "moe_grouped_gemm_down_mx", "FMT_MXFP8", "FMT_MXFP4",
     "moe_forward_fused", "moe_forward_is_fused",
+    "EP_MAX_RANKS", "EpPeers", "moe_ep_count", "moe_ep_dispatch", "moe_ep_local_offsets", "moe_ep_combine",
+    "ep_forward",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -40,6 +42,17 @@ FMT_MXFP4 = 3
 
 STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED",
           3: "MOE_ERR_WORKSPACE_TOO_SMALL", 4: "MOE_ERR_CUDA", 5: "MOE_ERR_DEVICE_FLAG"}
+
+
+EP_MAX_RANKS = 8
+
+
+class EpPeers(ctypes.Structure):
+    """moe_ep_peers_t: every rank's expert-parallel buffers (device addresses)."""
+    _fields_ = [("world", ctypes.c_int32), ("rank", ctypes.c_int32), ("capacity", ctypes.c_int32),
+                ("counts", ctypes.c_void_p * EP_MAX_RANKS), ("recv_rows", ctypes.c_void_p * EP_MAX_RANKS),
+                ("recv_src", ctypes.c_void_p * EP_MAX_RANKS), ("y_ret", ctypes.c_void_p * EP_MAX_RANKS),
+                ("pairs", ctypes.c_int32 * EP_MAX_RANKS)]
 
 
 class MoeError(RuntimeError):
@@ -141,6 +154,10 @@ def _load(debug_bounds: bool) -> ctypes.CDLL:
         "moe_forward_kernel_count": ([sp], ctypes.c_int32),
         "moe_forward_gathers_in_gemm": ([sp], ctypes.c_int32),
         "moe_forward_is_fused": ([sp], ctypes.c_int32),
+        "moe_ep_count": ([vp, sp, ctypes.POINTER(EpPeers), vp], ctypes.c_int),
+        "moe_ep_dispatch": ([vp, vp, vp, sp, ctypes.POINTER(EpPeers), vp], ctypes.c_int),
+        "moe_ep_local_offsets": ([sp, ctypes.POINTER(EpPeers), vp, vp], ctypes.c_int),
+        "moe_ep_combine": ([vp, vp, sp, ctypes.POINTER(EpPeers), vp], ctypes.c_int),
         "moe_status_string": ([ctypes.c_int], ctypes.c_char_p),
     }
     for name, (args, res) in sigs.items():
@@ -353,3 +370,118 @@ def forward(hidden: torch.Tensor, logits: torch.Tensor, w_gu: torch.Tensor, w_d:
         ws = torch.empty(max(moe_workspace_size(shape), 1), dtype=torch.uint8, device=hidden.device)
     moe_forward(hidden, logits, w_gu, w_gu_scales, w_d, w_d_scales, shape, out, ws, stream)
     return out
+
+
+# ---- expert parallelism -----------------------------------------------------
+
+def moe_ep_count(offsets, shape, peers: EpPeers, stream=None) -> None:
+    _check(lib().moe_ep_count(_p(offsets, I32), ctypes.byref(_shape(shape)), ctypes.byref(peers), _s(stream)),
+           "moe_ep_count")
+
+
+def moe_ep_dispatch(hidden, perm, offsets, shape, peers: EpPeers, stream=None) -> None:
+    _check(lib().moe_ep_dispatch(_p(hidden, BF16), _p(perm, I32), _p(offsets, I32), ctypes.byref(_shape(shape)),
+                                 ctypes.byref(peers), _s(stream)), "moe_ep_dispatch")
+
+
+def moe_ep_local_offsets(shape, peers: EpPeers, offsets_local, stream=None) -> None:
+    _check(lib().moe_ep_local_offsets(ctypes.byref(_shape(shape)), ctypes.byref(peers), _p(offsets_local, I32),
+                                      _s(stream)), "moe_ep_local_offsets")
+
+
+def moe_ep_combine(y_local, offsets_local, shape, peers: EpPeers, stream=None) -> None:
+    _check(lib().moe_ep_combine(_p(y_local, BF16), _p(offsets_local, I32), ctypes.byref(_shape(shape)),
+                                ctypes.byref(peers), _s(stream)), "moe_ep_combine")
+
+
+def ep_forward(ranks, w_gu_shards, w_d_shards, top_k: int, devices=None):
+    """The layer with its experts split over len(ranks) ranks driven from one
+    process: rank r holds tokens ranks[r] = (hidden [T_r,H] bf16, logits
+    [T_r,E] fp32) and the weights of experts r*E/R .. (r+1)*E/R - 1
+    (w_gu_shards[r] [E/R,2I,H], w_d_shards[r] [E/R,H,I], bf16), all on device
+    devices[r] (default: the current device for every rank, i.e. R ranks
+    emulated on one GPU; ranks on different GPUs need peer access between
+    them). The phases (route and permute, count, dispatch, local GEMMs,
+    combine, finalize) are separated by a synchronisation of every rank's
+    device, the barrier moe_ep_peers_t's steps ask for. Returns each rank's
+    out [T_r,H] bf16."""
+    R = len(ranks)
+    if not 1 <= R <= EP_MAX_RANKS:
+        raise ValueError(f"1 <= ranks <= {EP_MAX_RANKS}")
+    devs = [torch.device(d) for d in (devices or [torch.cuda.current_device()] * R)]
+    H = ranks[0][0].shape[1]
+    E = ranks[0][1].shape[1]
+    E_loc, I = w_d_shards[0].shape[0], w_d_shards[0].shape[2]
+    if E_loc * R != E:
+        raise ValueError("the weight shards must split the E experts evenly")
+    k = int(top_k)
+    Ts = [int(h.shape[0]) for h, _ in ranks]
+    capacity = ((sum(Ts) * k + k - 1) // k) * k          # every pair of every rank at one owner
+    i32 = torch.int32
+    st = []
+    for r, (h, lg) in enumerate(ranks):
+        d = devs[r]
+        P = Ts[r] * k
+        st.append({
+            "shape": Shape.of(Ts[r], H, I, E, k),
+            "ids": torch.empty(Ts[r], k, dtype=i32, device=d), "w": torch.empty(Ts[r], k, device=d),
+            "counts_g": torch.empty(E, dtype=i32, device=d), "offsets": torch.empty(E + 1, dtype=i32, device=d),
+            "perm": torch.empty(P, dtype=i32, device=d), "inv": torch.empty(P, dtype=i32, device=d),
+            "counts": torch.zeros(R, E_loc, dtype=i32, device=d),
+            "recv_rows": torch.empty(capacity, H, dtype=torch.bfloat16, device=d),
+            "recv_src": torch.empty(capacity, dtype=i32, device=d),
+            "y_ret": torch.empty(max(P, 1), H, dtype=torch.bfloat16, device=d),
+            "off_loc": torch.empty(E_loc + 1, dtype=i32, device=d),
+            "act": torch.empty(capacity, I, dtype=torch.bfloat16, device=d),
+            "y_loc": torch.empty(capacity, H, dtype=torch.bfloat16, device=d),
+            "out": torch.empty(Ts[r], H, dtype=torch.bfloat16, device=d),
+            "pws": torch.empty(max(1, moe_permute_workspace_size(Shape.of(Ts[r], H, I, E, k))), dtype=torch.uint8,
+                               device=d),
+        })
+    shape_loc = Shape.of(capacity // k, H, I, E_loc, k)
+
+    def peers(r):
+        pe = EpPeers()
+        pe.world, pe.rank, pe.capacity = R, r, capacity
+        for q in range(R):
+            pe.counts[q] = st[q]["counts"].data_ptr()
+            pe.recv_rows[q] = st[q]["recv_rows"].data_ptr()
+            pe.recv_src[q] = st[q]["recv_src"].data_ptr()
+            pe.y_ret[q] = st[q]["y_ret"].data_ptr()
+            pe.pairs[q] = Ts[q] * k
+        return pe
+
+    def barrier():
+        for d in set(devs):
+            torch.cuda.synchronize(d)
+
+    def each(fn):
+        for r in range(R):
+            with torch.cuda.device(devs[r]):
+                fn(r)
+        barrier()
+
+    def route_permute(r):
+        h, lg = ranks[r]
+        s = st[r]
+        moe_route(lg, s["shape"], s["ids"], s["w"])
+        moe_permute(s["ids"], s["shape"], s["counts_g"], s["offsets"], s["perm"], s["inv"], None, None, s["pws"])
+
+    def local_gemms(r):
+        s = st[r]
+        moe_ep_local_offsets(s["shape"], peers(r), s["off_loc"])
+        moe_grouped_gemm_swiglu(s["recv_rows"], None, s["off_loc"], w_gu_shards[r], None, shape_loc, s["act"])
+        moe_grouped_gemm_down(s["act"], s["off_loc"], w_d_shards[r], None, shape_loc, s["y_loc"])
+
+    def finalize(r):
+        s = st[r]
+        ident = torch.arange(Ts[r] * k, dtype=i32, device=devs[r])
+        moe_finalize(s["y_ret"], s["w"], ident, s["shape"], s["out"])
+
+    each(route_permute)
+    each(lambda r: moe_ep_count(st[r]["offsets"], st[r]["shape"], peers(r)))
+    each(lambda r: moe_ep_dispatch(ranks[r][0], st[r]["perm"], st[r]["offsets"], st[r]["shape"], peers(r)))
+    each(local_gemms)
+    each(lambda r: moe_ep_combine(st[r]["y_loc"], st[r]["off_loc"], st[r]["shape"], peers(r)))
+    each(finalize)
+    return [s["out"] for s in st]

@@ -178,6 +178,7 @@ def test_binding_refuses_tensors_of_the_wrong_dtype():
 
 
 C_CLIENT = r"""
+#include <stddef.h>
 #include <stdio.h>
 #include <string.h>
 #include "moe.h"
@@ -196,7 +197,7 @@ int main(void) {
     /* T = 0 enqueues nothing and succeeds without a GPU */
     s.T = 0;
     if (moe_forward(NULL, NULL, NULL, NULL, NULL, NULL, &s, NULL, NULL, 0, NULL) != MOE_OK) rc = 5;
-    printf("%zu %d\n", ws, rc);
+    printf("%zu %d %zu %zu\n", ws, rc, sizeof(moe_ep_peers_t), offsetof(moe_ep_peers_t, pairs));
     return rc;
 }
 """
@@ -221,7 +222,36 @@ def test_the_header_compiles_as_c99_and_a_c_program_links_and_runs(tmp_path):
     assert r.returncode == 0, r.stderr
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0, (r.stdout, r.stderr)
-    assert int(r.stdout.split()[0]) > 0
+    out = r.stdout.split()
+    assert int(out[0]) > 0
+    # the binding's moe_ep_peers_t has the C layout
+    assert int(out[2]) == ctypes.sizeof(moe.EpPeers) and int(out[3]) == moe.EpPeers.pairs.offset
+
+
+def test_ep_entry_points_validate_on_the_host():
+    # refused before anything is enqueued: no GPU needed (addresses are never used)
+    sh = moe.Shape.of(16, 128, 64, 8, 2)
+    pe = moe.EpPeers()
+    pe.world, pe.rank, pe.capacity = 3, 0, 32            # 8 experts do not split over 3 ranks
+    for q in range(3):
+        pe.counts[q] = pe.recv_rows[q] = pe.recv_src[q] = pe.y_ret[q] = 1 << 20
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_ep_count(1 << 20, sh, pe, stream=0)
+    assert ei.value.status == 2
+    pe.world, pe.rank = 2, 2                             # rank outside the world
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_ep_count(1 << 20, sh, pe, stream=0)
+    assert ei.value.status == 1
+    pe.rank = 1
+    pe.recv_rows[1] = (1 << 20) + 8                      # receive rows not 16-byte aligned
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_ep_dispatch(1 << 20, 1 << 20, 1 << 20, sh, pe, stream=0)
+    assert ei.value.status == 1
+    shs = moe.Shape.of(16, 128, 64, 8, 2, n_shared=1)    # shared experts are not dispatched
+    pe.recv_rows[1] = 1 << 20
+    with pytest.raises(moe.MoeError) as ei:
+        moe.moe_ep_local_offsets(shs, pe, 1 << 20, stream=0)
+    assert ei.value.status == 2
 
 
 @pytest.mark.parametrize("shape,status", [
