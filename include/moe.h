@@ -235,8 +235,14 @@ MOE_API moe_status_t moe_forward_fused(const moe_bf16_t *hidden, const float *lo
 
 /* moe_forward with hidden, logits and out in HOST memory (page-locked memory
  * gives asynchronous copies). Copies the inputs into the workspace, runs the
- * layer and copies out back, all on `stream`, then waits for the stream:
- * when it returns OK, out_host holds the result. Weights stay device-resident.
+ * layer and copies out back, then waits: when it returns OK, out_host holds
+ * the result. Weights stay device-resident. Up to 2047 tokens everything runs
+ * on `stream`. Larger batches are cut into 2 to 4 chunks of at least 1024
+ * tokens. The inputs of one chunk are copied in, and the output of the one
+ * before is copied out, on two streams the library creates once per device,
+ * while `stream` computes the current chunk. Each token's result depends only
+ * on its own row, so the output is the same bits. Calls on one device take
+ * turns on those streams, and a cudaDeviceReset invalidates them.
  *   ws: at least moe_forward_host_workspace_size(shape) bytes. */
 MOE_API size_t moe_forward_host_workspace_size(const moe_shape_t *shape);
 MOE_API moe_status_t moe_forward_host(const moe_bf16_t *hidden_host, const float *logits_host,

@@ -6,6 +6,9 @@
 
 #include <algorithm>
 #include <atomic>
+#include <map>
+#include <memory>
+#include <mutex>
 
 #include "launch.h"
 #include "moe.h"
@@ -227,6 +230,93 @@ moe_status_t forward_device(const moe_bf16_t *hidden, const float *logits, const
     return cuda_status(moe::launch_finalize(y, w, inv, T, H, k, out, error_flag_ptr(), st));
 }
 
+// ---- moe_forward_host for large batches: chunks in a copy/compute pipeline ----
+// Each token's output depends only on its own row, so the batch can be cut
+// into chunks of tokens without changing a bit. Chunk c's inputs are copied
+// in on one library stream while chunk c-1 computes on the caller's stream,
+// and chunk c-1's output is copied out on another while chunk c computes.
+constexpr int kHostChunkTokens = 1024;   // smallest chunk
+constexpr int kHostMaxChunks = 4;
+
+int host_chunks(const moe_shape_t *s) {
+    const int c = s->T / kHostChunkTokens;
+    return c < 2 ? 1 : (c < kHostMaxChunks ? c : kHostMaxChunks);
+}
+
+// The two copy streams and the events of one device, created on first use
+// and kept for the process; a call holds `m` from its first copy to its end.
+struct HostPipe {
+    std::mutex m;
+    cudaStream_t in = nullptr, out = nullptr;
+    cudaEvent_t start = nullptr, in_done[kHostMaxChunks] = {}, comp_done[kHostMaxChunks] = {};
+    bool ready = false;
+};
+
+HostPipe *host_pipe(int dev) {
+    static std::mutex mu;
+    static std::map<int, std::unique_ptr<HostPipe>> pipes;
+    std::lock_guard<std::mutex> lock(mu);
+    auto &p = pipes[dev];
+    if (!p) p.reset(new HostPipe());
+    return p.get();
+}
+
+moe_status_t forward_host_chunked(const moe_bf16_t *hidden_host, const float *logits_host, const void *w_gu,
+                                  const void *w_gu_scales, const void *w_d, const void *w_d_scales,
+                                  const moe_shape_t *shape, moe_bf16_t *out_host, uint8_t *base, const Layout &L,
+                                  cudaStream_t s) {
+    const int C = host_chunks(shape);
+    const int Tc = (shape->T + C - 1) / C;
+    moe_shape_t cs = *shape;
+    cs.T = Tc;
+    const Layout Lc = layout(&cs, false);            // a chunk's intermediates, inside the full layout's
+    if (Lc.total > L.hidden_in) return MOE_ERR_WORKSPACE_TOO_SMALL;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+    HostPipe *hp = host_pipe(dev);
+    std::lock_guard<std::mutex> lock(hp->m);
+    if (!hp->ready) {
+        bool ok = cudaStreamCreateWithFlags(&hp->in, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaStreamCreateWithFlags(&hp->out, cudaStreamNonBlocking) == cudaSuccess &&
+                  cudaEventCreateWithFlags(&hp->start, cudaEventDisableTiming) == cudaSuccess;
+        for (int c = 0; ok && c < kHostMaxChunks; ++c)
+            ok = cudaEventCreateWithFlags(&hp->in_done[c], cudaEventDisableTiming) == cudaSuccess &&
+                 cudaEventCreateWithFlags(&hp->comp_done[c], cudaEventDisableTiming) == cudaSuccess;
+        if (!ok) return MOE_ERR_CUDA;
+        hp->ready = true;
+    }
+    const size_t H = shape->H, E = shape->E;
+    // the copies start after the work already on the caller's stream
+    if (cudaEventRecord(hp->start, s) != cudaSuccess || cudaStreamWaitEvent(hp->in, hp->start, 0) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    for (int c = 0; c < C; ++c) {
+        const size_t t0 = static_cast<size_t>(c) * Tc;
+        const int tc = static_cast<int>(std::min<size_t>(Tc, shape->T - t0));
+        if (cudaMemcpyAsync(base + L.hidden_in + t0 * H * 2, hidden_host + t0 * H, tc * H * 2,
+                            cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+            cudaMemcpyAsync(base + L.logits_in + t0 * E * 4, logits_host + t0 * E, tc * E * 4,
+                            cudaMemcpyHostToDevice, hp->in) != cudaSuccess ||
+            cudaEventRecord(hp->in_done[c], hp->in) != cudaSuccess || cudaStreamWaitEvent(s, hp->in_done[c], 0) != cudaSuccess)
+            return MOE_ERR_CUDA;
+        cs.T = tc;
+        const moe_status_t st = forward_device(
+            reinterpret_cast<const moe_bf16_t *>(base + L.hidden_in) + t0 * H,
+            reinterpret_cast<const float *>(base + L.logits_in) + t0 * E, w_gu, w_gu_scales, w_d, w_d_scales, &cs,
+            reinterpret_cast<moe_bf16_t *>(base + L.out_st) + t0 * H, base, layout(&cs, false), s);
+        if (st != MOE_OK) return st;
+        if (cudaEventRecord(hp->comp_done[c], s) != cudaSuccess ||
+            cudaStreamWaitEvent(hp->out, hp->comp_done[c], 0) != cudaSuccess ||
+            cudaMemcpyAsync(out_host + t0 * H, base + L.out_st + t0 * H * 2, tc * H * 2, cudaMemcpyDeviceToHost,
+                            hp->out) != cudaSuccess)
+            return MOE_ERR_CUDA;
+    }
+    // the caller's stream continues after the last copy out; the call returns
+    // when everything is done
+    if (cudaEventRecord(hp->start, hp->out) != cudaSuccess || cudaStreamWaitEvent(s, hp->start, 0) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    return cuda_status(cudaStreamSynchronize(s));
+}
+
 }  // namespace
 
 namespace moe {
@@ -428,6 +518,9 @@ moe_status_t moe_forward_host(const moe_bf16_t *hidden_host, const float *logits
     if (!aligned(ws, 256)) return MOE_ERR_INVALID_ARG;
     auto *base = static_cast<uint8_t *>(ws);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (host_chunks(shape) > 1)
+        return forward_host_chunked(hidden_host, logits_host, w_gu, w_gu_scales, w_d, w_d_scales, shape, out_host,
+                                    base, L, s);
     const size_t hb = static_cast<size_t>(shape->T) * shape->H * 2;
     const size_t lb = static_cast<size_t>(shape->T) * shape->E * 4;
     if (cudaMemcpyAsync(base + L.hidden_in, hidden_host, hb, cudaMemcpyHostToDevice, s) != cudaSuccess)

@@ -199,8 +199,11 @@ def test_captured_forward_has_the_advertised_number_of_kernels():
     assert kernels == moe.moe_forward_kernel_count(L.shape) == 2      # counter reset + persistent kernel
 
 
-def test_forward_host_matches_forward():
-    L = Layer(moe_synth.get_config("qwen3_decode"))
+@pytest.mark.parametrize("name,T", [("qwen3_decode", 64), ("qwen3_prefill", 8192), ("skewed", 4096),
+                                    ("qwen3_prefill", 3000)])
+def test_forward_host_matches_forward(name, T):
+    # T >= 2048 runs in chunks on the library's copy streams: the same bits
+    L = Layer(moe_synth.get_config(name, T=T))
     ref = L.forward()
     d, c = L.d, L.cfg
     ws = torch.empty(moe.moe_forward_host_workspace_size(L.shape), dtype=torch.uint8, device=DEV)
