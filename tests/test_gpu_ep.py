@@ -37,8 +37,9 @@ def _ranks(cfg, Ts, seed0=100):
 
 
 @pytest.mark.parametrize("R,Ts,extra", [(1, [48], "none"), (2, [16, 40], "none"), (4, [33, 64, 7, 20], "none"),
-                                        (4, [64, 64, 64, 64], "bias0.5"), (8, [8, 1, 17, 64, 32, 5, 11, 40], "none")],
-                         ids=["R1", "R2", "R4", "R4_biased", "R8"])
+                                        (4, [64, 64, 64, 64], "bias0.5"), (8, [8, 1, 17, 64, 32, 5, 11, 40], "none"),
+                                        (2, [0, 24], "none")],
+                         ids=["R1", "R2", "R4", "R4_biased", "R8", "R2_empty_rank"])
 def test_ep_equals_moe_forward_on_each_rank(R, Ts, extra):
     cfg = moe_synth.get_config("qwen3_decode").with_(logit_extra=extra)
     w = moe_synth.gen_inputs(cfg.with_(T=1), seed=0)
