@@ -377,7 +377,9 @@ typedef struct {
 } moe_ep_peers_t;
 
 /* This rank's pairs per expert (from its offsets [E+1]) into row `rank` of
- * every owner's counts. */
+ * every owner's counts; zeros when this rank has no tokens (T = 0: offsets
+ * are not read and may be NULL). Unlike the other entry points it runs for
+ * T = 0, since the other ranks need this rank's row. */
 MOE_API moe_status_t moe_ep_count(const int32_t *offsets, const moe_shape_t *shape, const moe_ep_peers_t *peers,
                                   moe_stream_t stream);
 /* After every rank's count: this rank's permuted rows (hidden [T,H] through

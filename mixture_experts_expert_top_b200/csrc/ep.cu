@@ -49,13 +49,15 @@ EpPtrs ptrs_of(const moe_ep_peers_t *p) {
     return e;
 }
 
-// This rank's pairs per expert, into row `rank` of every owner's count matrix.
-__global__ void __launch_bounds__(kEpThreads) ep_count_kernel(const int32_t *__restrict__ offsets, int E, int E_loc,
-                                                             int rank, int world, const __grid_constant__ EpPtrs p) {
+// This rank's pairs per expert, into row `rank` of every owner's count matrix
+// (zeros for a rank without tokens, whose offsets are never written).
+__global__ void __launch_bounds__(kEpThreads) ep_count_kernel(const int32_t *__restrict__ offsets, int P, int E,
+                                                             int E_loc, int rank, int world,
+                                                             const __grid_constant__ EpPtrs p) {
     griddep_wait();
     for (int e = threadIdx.x; e < E; e += kEpThreads) {
         const int d = e / E_loc, el = e - d * E_loc;
-        p.counts[d][rank * E_loc + el] = offsets[e + 1] - offsets[e];
+        p.counts[d][rank * E_loc + el] = P > 0 ? offsets[e + 1] - offsets[e] : 0;
     }
 }
 
@@ -191,10 +193,11 @@ moe_status_t moe_ep_count(const int32_t *offsets, const moe_shape_t *shape, cons
     int E_loc = 0;
     moe_status_t st = moe::check_ep(shape, peers, E_loc);
     if (st != MOE_OK) return st;
-    if (!offsets) return MOE_ERR_INVALID_ARG;
+    const int P = shape->T * shape->top_k;
+    if (!offsets && P > 0) return MOE_ERR_INVALID_ARG;
     return moe::status_of(moe::launch_pdl(moe::ep_count_kernel, dim3(1), dim3(moe::kEpThreads), 0,
-                                          static_cast<cudaStream_t>(stream), offsets, shape->E, E_loc, peers->rank,
-                                          peers->world, moe::ptrs_of(peers)));
+                                          static_cast<cudaStream_t>(stream), offsets, P, shape->E, E_loc,
+                                          peers->rank, peers->world, moe::ptrs_of(peers)));
 }
 
 moe_status_t moe_ep_dispatch(const moe_bf16_t *hidden, const int32_t *perm, const int32_t *offsets,
