@@ -61,17 +61,48 @@ __global__ void __launch_bounds__(kEpThreads) ep_count_kernel(const int32_t *__r
     }
 }
 
-// Start of this rank's rows of expert e in its owner's receive buffer: all
-// rows of the owner's lower experts, then the lower ranks' rows of e.
-__device__ int dest_base(const EpPtrs &p, int e, int E_loc, int rank, int world) {
-    const int d = e / E_loc, el = e - d * E_loc;
-    const int32_t *c = p.counts[d];
-    int base = 0;
-    for (int s = 0; s < world; ++s) {
-        for (int j = 0; j < el; ++j) base += c[s * E_loc + j];
-        if (s < rank) base += c[s * E_loc + el];
+// base[e] = start of this rank's rows of expert e in its owner's receive
+// buffer: all rows of the owner's lower experts, then the lower ranks' rows
+// of e. One exclusive scan over the E experts' totals over all ranks,
+// restarted at each owner's first expert. Every thread of the CTA calls it;
+// prefix is scratch of E ints.
+__device__ void dest_bases(const EpPtrs &p, int E, int E_loc, int rank, int world, int *prefix, int *base) {
+    __shared__ int chunk_sum[kEpThreads];
+    const int per = (E + kEpThreads - 1) / kEpThreads;     // experts per thread, contiguous
+    const int e0 = threadIdx.x * per;
+    int run = 0;
+    for (int i = 0; i < per && e0 + i < E; ++i) {
+        const int e = e0 + i, d = e / E_loc, el = e - d * E_loc;
+        int t = 0, below = 0;
+        for (int s = 0; s < world; ++s) {
+            const int c = p.counts[d][s * E_loc + el];
+            t += c;
+            if (s < rank) below += c;
+        }
+        prefix[e] = t;                                      // the total, for now
+        base[e] = below;
+        run += t;
     }
-    return base;
+    chunk_sum[threadIdx.x] = run;
+    __syncthreads();
+    if (threadIdx.x == 0) {                                 // exclusive scan of the threads' sums
+        int acc = 0;
+        for (int i = 0; i < kEpThreads; ++i) {
+            const int v = chunk_sum[i];
+            chunk_sum[i] = acc;
+            acc += v;
+        }
+    }
+    __syncthreads();
+    int excl = chunk_sum[threadIdx.x];
+    for (int i = 0; i < per && e0 + i < E; ++i) {
+        const int t = prefix[e0 + i];
+        prefix[e0 + i] = excl;
+        excl += t;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += kEpThreads) base[e] += prefix[e] - prefix[(e / E_loc) * E_loc];
+    __syncthreads();
 }
 
 // Row r of this rank's permutation (expert e, i-th of e's rows) -> row
@@ -85,10 +116,10 @@ __global__ void __launch_bounds__(kEpThreads) ep_dispatch_kernel(const uint4 *__
     extern __shared__ int ep_smem[];
     int *off_s = ep_smem;              // [E + 1]
     int *base_s = off_s + E + 1;       // [E]
+    int *prefix_s = base_s + E;        // [E]
     griddep_wait();
     for (int e = threadIdx.x; e <= E; e += kEpThreads) off_s[e] = offsets[e];
-    for (int e = threadIdx.x; e < E; e += kEpThreads) base_s[e] = dest_base(p, e, E_loc, rank, world);
-    __syncthreads();
+    dest_bases(p, E, E_loc, rank, world, prefix_s, base_s);
     const int lane = threadIdx.x & 31;
     const int warps = gridDim.x * (kEpThreads / 32);
     for (int r = blockIdx.x * (kEpThreads / 32) + (threadIdx.x >> 5); r < P; r += warps) {
@@ -209,7 +240,7 @@ moe_status_t moe_ep_dispatch(const moe_bf16_t *hidden, const int32_t *perm, cons
     const int P = shape->T * shape->top_k;
     if (P == 0) return MOE_OK;
     if (!hidden || !perm || !offsets || reinterpret_cast<uintptr_t>(hidden) % 16) return MOE_ERR_INVALID_ARG;
-    const size_t smem = (2 * static_cast<size_t>(shape->E) + 1) * sizeof(int);
+    const size_t smem = (3 * static_cast<size_t>(shape->E) + 1) * sizeof(int);
     return moe::status_of(moe::launch_pdl(moe::ep_dispatch_kernel, dim3(moe::ep_grid(P)), dim3(moe::kEpThreads),
                                           smem, static_cast<cudaStream_t>(stream),
                                           reinterpret_cast<const uint4 *>(hidden), perm, offsets, P, shape->top_k,
