@@ -7,9 +7,11 @@ tokens, through the C ABI (moe_forward). The headline workload is the
 largest single-GPU one, the Qwen3-30B-A3B-shaped prefill layer: T=8192,
 H=2048, I=768, E=128, top_k=8, bf16 weights. The same run also times the
 other graded workloads (Qwen3 decode, the skewed Zipf layer and the W4A16
-decode layer) and reports them under "workloads". Every workload reads more
-than the 126 MB L2 per step (its expert weights), so no flush is needed
-between steps.
+decode layer) and, ungraded, the MXFP8, MXFP4 and shared-expert decode
+layers, and reports them under "workloads". Every workload reads more than
+the 126 MB L2 per step (its expert weights), so no flush is needed between
+steps. For a bf16 decode batch moe_forward is one persistent kernel (after a
+one-warp counter reset); its roofline is taken over the timed region.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                   [--extra all|none|NAME,...] [--impl ours|reference]
