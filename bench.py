@@ -66,6 +66,7 @@ KERNEL_SOURCES = ["mixture_experts_expert_top_b200/csrc/gemm_sm100.cu",
                   "mixture_experts_expert_top_b200/csrc/gemm_prefill_sm100.cu",
                   "mixture_experts_expert_top_b200/csrc/gemm_wm_pair_sm100.cu",
                   "mixture_experts_expert_top_b200/csrc/gemm_mxfp8_sm100.cu",
+                  "mixture_experts_expert_top_b200/csrc/gemm_int4_warp_sm100.cu",
                   "mixture_experts_expert_top_b200/csrc/gemm_common.cuh",
                   "mixture_experts_expert_top_b200/csrc/common.cuh",
                   "mixture_experts_expert_top_b200/csrc/launch_util.cuh"]

@@ -42,7 +42,37 @@ struct Params {
     const uint16_t *w_scales;   // int4: [E * w_rows, K/128]
     int evict_first_weights;
     int hints;                  // kGemmHint* bits
+    const uint16_t *a;          // the token operand's rows (GemmArgs::a), for kernels that copy them without TMA
 };
+
+// W4A16 decoding of one 32-bit word of packed int4 (K elements 8i..8i+7 of a
+// row; byte b holds element 2b in its low nibble, 2b+1 in its high nibble,
+// two's complement) into four bf16x2 words (elements 2j, 2j+1 in word j):
+//   w = bf16_rne(q * scale)
+// Each nibble pair is placed in the mantissas of a bf16x2 with exponent 2^7
+// and biased to n = q + 8 (the bias is the flip of the nibble's sign bit,
+// folded into the same three-input logic op), giving bf16 (128 + n) exactly;
+// subtracting 136 gives q exactly, and one bf16 multiply by the scale rounds
+// the exact product once, to nearest even.
+__device__ __forceinline__ void dequant_word(uint32_t packed, __nv_bfloat162 scale2, uint32_t *out4) {
+    const uint32_t hi = packed >> 4;                       // odd elements move to the low nibble of each byte
+    const __nv_bfloat162 bias = __floats2bfloat162_rn(136.0f, 136.0f);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        // byte 0 <- element 2j (low nibble of byte j), byte 2 <- element 2j+1
+        const uint32_t r = __byte_perm(packed, hi, static_cast<uint32_t>(j | ((4 + j) << 8)));
+        // bits of 0x000F000F: r ^ 0x00080008 (n = q + 8); other bits: 0x43004300
+        const uint32_t v = (r & 0x000F000Fu) ^ 0x43084308u;
+        const __nv_bfloat162 q = __hsub2(*reinterpret_cast<const __nv_bfloat162 *>(&v), bias);
+        const __nv_bfloat162 w = __hmul2(q, scale2);
+        out4[j] = *reinterpret_cast<const uint32_t *>(&w);
+    }
+}
+
+__device__ __forceinline__ __nv_bfloat162 bf16_pair(uint16_t bits) {
+    const __nv_bfloat16 b = __ushort_as_bfloat16(bits);
+    return __halves2bfloat162(b, b);
+}
 
 // Tile bookkeeping shared by the roles.
 struct TileInfo {
@@ -237,6 +267,7 @@ inline Params make_params(const GemmArgs &g, int BN) {
     Params p;
     p.offsets = g.offsets;
     p.perm = g.perm;
+    p.a = static_cast<const uint16_t *>(g.a);
     p.top_k = g.top_k;
     p.E = g.E;
     p.K = g.K;

@@ -106,6 +106,10 @@ cudaError_t launch_grouped_gemm_prefill(const GemmArgs &g, cudaStream_t s);
 cudaError_t launch_grouped_gemm_wm_pair(const GemmArgs &g, cudaStream_t s);
 cudaError_t launch_dequant_int4(const uint8_t *q, const uint16_t *scales, int rows, int K, uint16_t *out,
                                 cudaStream_t s);
+// ---- gemm_int4_warp_sm100.cu: the W4A16 down GEMM for few rows per expert
+// (P/E <= 24): int4 decoded in registers straight into warp-level MMA
+// fragments (swiglu must be false)
+cudaError_t launch_grouped_gemm_int4_warp(const GemmArgs &g, cudaStream_t s);
 
 // ---- gemm_mxfp8_sm100.cu: MXFP8 weights (E4M3 + one E8M0 scale per 32 K),
 // block-scaled tcgen05 MMA; the token operand is MX-quantised too.

@@ -258,6 +258,12 @@ GEMM_CFGS = [
     moe_synth.get_config("qwen3_prefill", T=1100, H=264, I=200, E=4, k=2),  # CTA-pair, ragged H and I
     moe_synth.get_config("qwen3_decode", T=448, H=1024, I=384, E=64, k=8),  # weights on M, 128-token blocks
     moe_synth.MoeConfig("int4_bn64", T=96, H=1024, I=384, E=24, k=8, fmt="int4_g128"),  # int4, 64-token blocks
+    # int4 with few rows per expert (gate/up decoded into TMEM, down into
+    # warp-level MMA fragments): K = 640 and 384 end half-way through a 256-K
+    # stage
+    moe_synth.MoeConfig("int4_warp_ragged", T=40, H=640, I=384, E=10, k=3, fmt="int4_g128"),
+    # uneven load: empty experts, experts past 32 rows (several token blocks)
+    moe_synth.MoeConfig("int4_warp_zipf", T=64, H=512, I=256, E=16, k=4, fmt="int4_g128", logit_extra="zipf1.2"),
 ]
 
 
