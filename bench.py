@@ -59,7 +59,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NORTH_STAR_HBM_GBS = 8000.0       # the roofline literals the layer's target is stated against
 NORTH_STAR_BF16_TFLOPS = 2250.0
 PROFILE_DIR = os.path.join(ROOT, "profiles")
-# the GEMM kernels' sources: a change to any of them invalidates stored counters
+# Kernel sources whose change invalidates stored counters. A profile summary
+# may name the files its kernel is built from ("kernel_sources: a.cu b.cuh",
+# paths under csrc/); its counters then stand while those files are
+# unchanged. Without that line every file below counts.
+CSRC_DIR = "mixture_experts_expert_top_b200/csrc"
 KERNEL_SOURCES = ["mixture_experts_expert_top_b200/csrc/gemm_sm100.cu",
                   "mixture_experts_expert_top_b200/csrc/fused_decode_sm100.cu",
                   "mixture_experts_expert_top_b200/csrc/route_dev.cuh",
@@ -153,9 +157,11 @@ def host_cpu_model() -> str:
     return platform.processor() or "unknown"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(files=None) -> str:
+    """First 16 hex digits of the SHA-256 of the given source files' bytes,
+    in order (default: KERNEL_SOURCES)."""
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in (files if files is not None else KERNEL_SOURCES):
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -171,7 +177,13 @@ def profiled_traffic(kernel: str, workload: str):
         return None
     m_hash = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]{16})", text)
     m_tr = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m_hash or not m_tr or m_hash.group(1) != kernel_source_hash():
+    m_src = re.search(r"kernel_sources:[ \t]*(\S.*)", text)
+    files = [f"{CSRC_DIR}/{n}" for n in m_src.group(1).split()] if m_src else None
+    try:
+        current = kernel_source_hash(files)
+    except OSError:
+        return None
+    if not m_hash or not m_tr or m_hash.group(1) != current:
         return None
     return float(m_tr.group(1))
 
