@@ -163,7 +163,10 @@ MOE_API moe_status_t moe_grouped_gemm_swiglu(const moe_bf16_t *a, const int32_t 
 /* Grouped GEMM down. InfiniLM PR #500 report §2.2 step 2 (third grouped GEMM).
  *   act     [T*top_k,I] bf16, offsets [E+1]
  *   w_d     MOE_W_BF16: [E,H,I] bf16. MOE_W_INT4_G128: [E,H,I/2] bytes with
- *           w_d_scales [E,H,I/128] bf16.
+ *           w_d_scales [E,H,I/128] bf16; w = bf16(q * scale) is formed on
+ *           chip (in tensor memory, or, with at most 24 rows per expert on
+ *           average, in the registers that feed warp-level MMAs) and never
+ *           reaches HBM.
  *   y       [T*top_k,H] bf16 out: unscaled down projection, permuted row order. */
 MOE_API moe_status_t moe_grouped_gemm_down(const moe_bf16_t *act, const int32_t *offsets,
                                    const void *w_d, const void *w_d_scales,
