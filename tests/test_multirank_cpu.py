@@ -123,3 +123,25 @@ def test_bench_rejects_too_few_warmup_steps():
     import bench
     with pytest.raises(SystemExit):
         bench.parse_args(["--warmup", "2"])
+
+
+def test_stored_traffic_follows_its_kernel_sources(tmp_path, monkeypatch):
+    """A profile summary's DRAM figure is reported while the files it names
+    hash as stored, and dropped (None) once they do not."""
+    sys.path.insert(0, ROOT)
+    import bench
+    files = ["common.cuh", "launch_util.cuh"]
+    h = bench.kernel_source_hash([f"{bench.CSRC_DIR}/{n}" for n in files])
+    monkeypatch.setattr(bench, "PROFILE_DIR", str(tmp_path))
+    body = "dram_bytes_per_launch: 12345\nkernel_sources: {}\nkernel_source_sha256_16: {}\n"
+    (tmp_path / "k_w.md").write_text(body.format(" ".join(files), h))
+    assert bench.profiled_traffic("k", "w") == 12345.0
+    (tmp_path / "k_w.md").write_text(body.format(" ".join(reversed(files)), h))   # other files, other hash
+    assert bench.profiled_traffic("k", "w") is None
+    (tmp_path / "k_w.md").write_text(body.format("no_such_file.cu", h))
+    assert bench.profiled_traffic("k", "w") is None
+    assert bench.profiled_traffic("k", "missing") is None
+    # the committed summaries of the graded workloads carry a source list
+    for name in ("gemm_swiglu_qwen3_prefill", "gemm_swiglu_skewed", "gemm_swiglu_w4a16_decode", "fused_qwen3_decode"):
+        text = open(os.path.join(ROOT, "profiles", name + ".md")).read()
+        assert "kernel_sources:" in text and "kernel_source_sha256_16:" in text
